@@ -1,0 +1,232 @@
+"""CPU oracle for the product-key memory lookup (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library and its Python
+binding never do: the two implementations share no code.
+
+The arithmetic lives in ``pkm_oracle.c`` (plain C, IEEE double, OpenMP over
+(token, head)); this module only compiles it and marshals numpy arrays.
+Each function states which passage of the pages it follows:
+
+* "Memory Layers at Scale" digest, "Product-key 검색": split keys, top-k
+  from 2*sqrt(N) comparisons.
+* "Memory Layers at Scale" digest, "Memory+ 블록": (y ⊙ silu(x W1)) W2 and
+  qk-normalization.
+* "Memory Layers at Scale" digest, "병렬 EmbeddingBag 구현": the weighted bag.
+* "모델 안의 메모리", "작동 방식" and figure D: halves scored against the
+  half-keys, best of each combined, weighted average of the values read.
+
+Parity pins (tests/test_oracle_pins.py) tie every function to something other
+than itself: brute force over all N keys, closed forms, numpy/torch library
+special cases and finite differences.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pkm_oracle.c")
+_HDR = os.path.join(_HERE, "pkm_oracle.h")
+_LIB = os.path.join(_HERE, "liboracle_pkm.so")
+
+F64, F32, BF16 = 0, 1, 2
+NORM_EPS = 1e-12
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle_pkm.so`` (gcc, OpenMP)."""
+    stale = (not os.path.exists(_LIB)) or any(
+        os.path.getmtime(p) > os.path.getmtime(_LIB) for p in (_SRC, _HDR))
+    if force or stale:
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+               "-Wall", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I64, I = ctypes.c_int64, ctypes.c_int
+        lib.orc_half_scores.argtypes = [I64, I, I, I, P, I, P, I, P]
+        lib.orc_topk.argtypes = [P, I, I, P]
+        lib.orc_pkm_select.argtypes = [I64, I, I, I, I, P, I, P, I, P, P, P, P]
+        lib.orc_bruteforce_select.argtypes = [I64, I, I, I, I, P, I, P, I, P, P]
+        lib.orc_softmax.argtypes = [P, I64, I, P]
+        lib.orc_bag.argtypes = [I64, I, I, P, P, P, I, I64, P]
+        lib.orc_memplus.argtypes = [I64, I, I, P, P, I, P, I, P, I, P]
+        lib.orc_pkm_backward.argtypes = [I64, I, I, I, I, I, P, I, P, I, P, I, I64,
+                                         P, P, P, P, I, P, P, P, P, P]
+        lib.orc_num_threads.argtypes = []
+        for f in ("orc_half_scores", "orc_topk", "orc_pkm_select",
+                  "orc_bruteforce_select", "orc_softmax", "orc_bag", "orc_memplus",
+                  "orc_pkm_backward", "orc_num_threads"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _input(x):
+    """(contiguous numpy array, dtype tag) for a numpy array or torch tensor.
+
+    bf16 tensors travel as their raw 16-bit patterns and are decoded exactly
+    by the C code; fp32 and fp64 are passed as they are.
+    """
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return x.view(torch.int16).numpy().view(np.uint16), BF16
+            if x.dtype == torch.float32:
+                return x.numpy(), F32
+            return x.to(torch.float64).numpy(), F64
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, F32
+    if x.dtype == np.uint16:
+        return x, BF16
+    return np.ascontiguousarray(x, dtype=np.float64), F64
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+def half_scores(q, K):
+    """s[t,h,c,a] = sqrt(dh) * <q_c/|q_c|, K_c[a]/|K_c[a]|>  (shape [T,H,2,n])."""
+    qa, qt = _input(q)
+    ka, kt = _input(K)
+    T, H, two, dh = qa.shape
+    n = ka.shape[2]
+    out = np.empty((T, H, 2, n), np.float64)
+    _check(_load().orc_half_scores(T, H, dh, n, _p(qa), qt, _p(ka), kt, _p(out)),
+           "half_scores")
+    return out
+
+
+def topk(s, k: int):
+    """Positions of the k largest entries of the 1-D array s, larger first,
+    equal values -> smaller position first."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    pos = np.empty(k, np.int32)
+    _check(_load().orc_topk(_p(s), s.shape[0], k, _p(pos)), "topk")
+    return pos
+
+
+def pkm_select(q, K, k: int):
+    """Product-key selection.  Returns (idx int64 [T,H,k], S [T,H,k],
+    w [T,H,k], number of half-key dot products evaluated)."""
+    qa, qt = _input(q)
+    ka, kt = _input(K)
+    T, H, _, dh = qa.shape
+    n = ka.shape[2]
+    idx = np.empty((T, H, k), np.int64)
+    S = np.empty((T, H, k), np.float64)
+    w = np.empty((T, H, k), np.float64)
+    dots = ctypes.c_int64(0)
+    _check(_load().orc_pkm_select(T, H, dh, n, k, _p(qa), qt, _p(ka), kt, _p(idx),
+                                  _p(S), _p(w), ctypes.byref(dots)), "pkm_select")
+    return idx, S, w, int(dots.value)
+
+
+def bruteforce_select(q, K, k: int):
+    """Top-k over all N = n*n full keys.  Returns (idx [T,H,k], S [T,H,k])."""
+    qa, qt = _input(q)
+    ka, kt = _input(K)
+    T, H, _, dh = qa.shape
+    n = ka.shape[2]
+    idx = np.empty((T, H, k), np.int64)
+    S = np.empty((T, H, k), np.float64)
+    _check(_load().orc_bruteforce_select(T, H, dh, n, k, _p(qa), qt, _p(ka), kt,
+                                         _p(idx), _p(S)), "bruteforce_select")
+    return idx, S
+
+
+def softmax(S):
+    S = np.ascontiguousarray(S, dtype=np.float64)
+    k = S.shape[-1]
+    w = np.empty_like(S)
+    _check(_load().orc_softmax(_p(S), S.size // k, k, _p(w)), "softmax")
+    return w
+
+
+def bag(idx, w, table):
+    """y[t] = sum_j w[t,j] * table[idx[t,j]]; idx/w [n_bags, B]."""
+    idx = np.ascontiguousarray(idx, dtype=np.int64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    ta, tt = _input(table)
+    n_bags = idx.shape[0]
+    B = int(np.prod(idx.shape[1:]))
+    d = ta.shape[1]
+    y = np.empty((n_bags, d), np.float64)
+    _check(_load().orc_bag(n_bags, B, d, _p(idx), _p(w), _p(ta), tt, ta.shape[0],
+                           _p(y)), "bag")
+    return y
+
+
+def memplus(y, x, W1, W2):
+    """out = (y ⊙ silu(x W1)) W2."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    xa, xt = _input(x)
+    w1, w1t = _input(W1)
+    w2, w2t = _input(W2)
+    T, dm = xa.shape
+    dv = w1.shape[1]
+    out = np.empty((T, dm), np.float64)
+    _check(_load().orc_memplus(T, dm, dv, _p(y), _p(xa), xt, _p(w1), w1t, _p(w2), w2t,
+                               _p(out)), "memplus")
+    return out
+
+
+def pkm_backward(q, K, table, idx, vrow, w, dy, want_dv: bool = True):
+    """Backward of the lookup with the selection held fixed.
+
+    ``idx`` [T,H,k] holds global row ids (a*n+b); ``vrow`` [T,H,k] the
+    position of each selected row in the compact ``table`` [n_rows, d_v].
+    Returns dict(dw, dS [T,H,k], dq [T,H,2,dh], dK [H,2,n,dh],
+    dV [n_rows, d_v] or None).
+    """
+    qa, qt = _input(q)
+    ka, kt = _input(K)
+    ta, tt = _input(table)
+    da, dt = _input(dy)
+    idx = np.ascontiguousarray(idx, dtype=np.int64)
+    vrow = np.ascontiguousarray(vrow, dtype=np.int64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    T, H, _, dh = qa.shape
+    n = ka.shape[2]
+    k = idx.shape[-1]
+    dv = ta.shape[1]
+    dw = np.empty((T, H, k))
+    dS = np.empty((T, H, k))
+    dq = np.empty((T, H, 2, dh))
+    dK = np.empty((H, 2, n, dh))
+    dV = np.empty((ta.shape[0], dv)) if want_dv else None
+    _check(_load().orc_pkm_backward(
+        T, H, dh, n, k, dv, _p(qa), qt, _p(ka), kt, _p(ta), tt, ta.shape[0],
+        _p(idx), _p(vrow), _p(w), _p(da), dt, _p(dw), _p(dS), _p(dq), _p(dK),
+        _p(dV) if want_dv else None), "pkm_backward")
+    return dict(dw=dw, dS=dS, dq=dq, dK=dK, dV=dV)

@@ -1,0 +1,338 @@
+"""Pins of the CPU oracle against things other than itself (no GPU needed).
+
+Each test ties one oracle function to brute force, a closed form, an
+invariant, a library routine on a special case, the pages' printed counts,
+or finite differences.  A plausible slip in the oracle (a wrong scale, a
+swapped half, a transposed weight, a dropped softmax term, a wrong sign in
+the backward) fails at least one of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from sparse_key_value_b200.inputs import WORKLOADS, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g, dtype=torch.float64) * std).numpy()
+
+
+def _problem(T, H, dh, n, seed):
+    q = _rand((T, H, 2, dh), seed)
+    K = _rand((H, 2, n, dh), seed + 1, 1.0 / math.sqrt(dh))
+    return q, K
+
+
+# --------------------------------------------------------------------------
+# half scores: closed forms, invariance, library special case
+# --------------------------------------------------------------------------
+
+def test_half_scores_closed_forms(orc):
+    dh, n = 16, 5
+    q = _rand((1, 1, 2, dh), 3)
+    K = _rand((1, 2, n, dh), 4)
+    K[0, 0, 1] = 3.0 * q[0, 0, 0]       # parallel to the first half -> +sqrt(dh)
+    K[0, 0, 2] = -0.5 * q[0, 0, 0]      # anti-parallel -> -sqrt(dh)
+    v = _rand((dh,), 5)
+    u = q[0, 0, 1]
+    K[0, 1, 3] = v - (v @ u) / (u @ u) * u  # orthogonal to the second half -> 0
+    s = orc.half_scores(q, K)
+    assert s.shape == (1, 1, 2, n)
+    assert s[0, 0, 0, 1] == pytest.approx(math.sqrt(dh), rel=1e-13)
+    assert s[0, 0, 0, 2] == pytest.approx(-math.sqrt(dh), rel=1e-13)
+    assert abs(s[0, 0, 1, 3]) < 1e-12
+    assert np.all(np.abs(s) <= math.sqrt(dh) * (1 + 1e-12))
+
+
+def test_half_scores_scale_invariance(orc):
+    q, K = _problem(6, 2, 8, 7, 10)
+    s = orc.half_scores(q, K)
+    rng = np.random.default_rng(0)
+    q2 = q * rng.uniform(0.01, 100.0, size=q.shape[:-1] + (1,))
+    K2 = K * rng.uniform(0.01, 100.0, size=K.shape[:-1] + (1,))
+    np.testing.assert_allclose(orc.half_scores(q2, K2), s, rtol=1e-12, atol=1e-12)
+
+
+def test_half_scores_match_library_cosine(orc):
+    q, K = _problem(4, 3, 12, 9, 11)
+    s = orc.half_scores(q, K)
+    qt, Kt = torch.from_numpy(q), torch.from_numpy(K)
+    for h in range(3):
+        for c in range(2):
+            cos = torch.nn.functional.cosine_similarity(
+                qt[:, h, c, None, :], Kt[None, h, c, :, :], dim=-1)
+            np.testing.assert_allclose(s[:, h, c, :], math.sqrt(12) * cos.numpy(),
+                                       rtol=1e-12, atol=1e-12)
+
+
+def test_zero_vector_clamp(orc):
+    q = np.zeros((1, 1, 2, 4))
+    K = _rand((1, 2, 3, 4), 12)
+    assert np.all(orc.half_scores(q, K) == 0.0)
+
+
+# --------------------------------------------------------------------------
+# top-k and the tie rule: library sort
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,k", [(1, 1), (7, 3), (64, 64), (100, 17)])
+def test_topk_matches_library_lexsort(orc, n, k):
+    rng = np.random.default_rng(n * 100 + k)
+    s = np.round(rng.normal(size=n), 1)  # many exact ties
+    ref = np.lexsort((np.arange(n), -s))[:k]
+    np.testing.assert_array_equal(orc.topk(s, k), ref)
+
+
+def test_topk_matches_torch_on_distinct(orc):
+    rng = np.random.default_rng(1)
+    s = rng.normal(size=257)
+    ref = torch.topk(torch.from_numpy(s), 31, sorted=True).indices.numpy()
+    np.testing.assert_array_equal(orc.topk(s, 31), ref)
+
+
+# --------------------------------------------------------------------------
+# product-key selection == the definition (brute force over all N keys)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", [2, 3, 8, 16])
+def test_product_key_equals_bruteforce(orc, n):
+    for k in sorted({1, 2, n // 2 or 1, n}):
+        q, K = _problem(9, 2, 8, n, 20 + n * 10 + k)
+        idx, S, w, _ = orc.pkm_select(q, K, k)
+        bidx, bS = orc.bruteforce_select(q, K, k)
+        np.testing.assert_array_equal(idx, bidx)
+        np.testing.assert_allclose(S, bS, rtol=0, atol=1e-12)
+
+
+def test_product_key_equals_bruteforce_tiny_workload(orc):
+    """The tiny fp32 workload (N = 1024 keys): the definition brute-forced."""
+    w = WORKLOADS["tiny"]
+    inp = make_inputs(w.scaled(T=64), "cpu", with_values=False)
+    idx, S, _, _ = orc.pkm_select(inp["query"], inp["subkeys"], w.k)
+    bidx, bS = orc.bruteforce_select(inp["query"], inp["subkeys"], w.k)
+    np.testing.assert_array_equal(idx, bidx)
+    np.testing.assert_allclose(S, bS, rtol=0, atol=1e-12)
+
+
+def test_selection_with_exact_ties(orc):
+    """Duplicate sub-key rows tie exactly; the smaller row id comes first."""
+    q, K = _problem(5, 1, 8, 6, 30)
+    K[0, 0, 4] = K[0, 0, 1]
+    K[0, 1, 5] = K[0, 1, 2]
+    for k in (1, 3, 6):
+        idx, _, _, _ = orc.pkm_select(q, K, k)
+        bidx, _ = orc.bruteforce_select(q, K, k)
+        np.testing.assert_array_equal(idx, bidx)
+
+
+def test_planted_key_row_id_convention(orc):
+    """Sub-key a* of half 1 equal to the first query half and b* of half 2
+    equal to the second give the best full key, row id a* * n + b*."""
+    n, dh = 11, 8
+    q, K = _problem(3, 2, dh, n, 40)
+    plants = {(0, 0): (7, 2), (0, 1): (3, 9), (1, 0): (10, 0), (2, 1): (0, 10)}
+    for (t, h), (a, b) in plants.items():
+        Kp = K.copy()
+        Kp[h, 0, a] = 2.0 * q[t, h, 0]
+        Kp[h, 1, b] = 5.0 * q[t, h, 1]
+        idx, S, _, _ = orc.pkm_select(q, Kp, 1)
+        assert idx[t, h, 0] == a * n + b
+        assert S[t, h, 0] == pytest.approx(2 * math.sqrt(dh), rel=1e-12)
+
+
+def test_k1_is_argmax_of_each_half(orc):
+    q, K = _problem(7, 3, 8, 13, 50)
+    s = orc.half_scores(q, K)
+    idx, _, w, _ = orc.pkm_select(q, K, 1)
+    np.testing.assert_array_equal(idx[..., 0], s[:, :, 0].argmax(-1) * 13 + s[:, :, 1].argmax(-1))
+    assert np.all(w == 1.0)
+
+
+def test_comparison_counts_match_pages(orc):
+    """2*sqrt(N) half-key comparisons per (token, head), as the pages count."""
+    with open(os.path.join(GOLDEN, "comparison_counts.json")) as f:
+        cases = json.load(f)["cases"]
+    for case in cases:
+        n = case["n_sub"]
+        assert n * n == case["cells"]
+        q, K = _problem(2, 1, 4, n, 60)
+        _, _, _, dots = orc.pkm_select(q, K, 2)
+        assert dots == 2 * case["comparisons"]  # 2 (token, head) pairs
+        assert dots // 2 == 2 * math.isqrt(case["cells"])
+
+
+# --------------------------------------------------------------------------
+# softmax weights
+# --------------------------------------------------------------------------
+
+def test_softmax_properties(orc):
+    q, K = _problem(8, 2, 8, 10, 70)
+    idx, S, w, _ = orc.pkm_select(q, K, 6)
+    np.testing.assert_allclose(w.sum(-1), 1.0, rtol=0, atol=1e-14)
+    ref = torch.softmax(torch.from_numpy(S), dim=-1).numpy()
+    np.testing.assert_allclose(w, ref, rtol=1e-14, atol=0)
+    assert np.all(np.diff(w, axis=-1) <= 0)  # scores are in descending order
+    np.testing.assert_allclose(orc.softmax(np.full((3, 5), 2.5)), 0.2, rtol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# weighted bag: library embedding_bag
+# --------------------------------------------------------------------------
+
+def test_bag_matches_library_embedding_bag(orc):
+    rng = np.random.default_rng(2)
+    table = rng.normal(size=(50, 24))
+    idx = rng.integers(0, 50, size=(13, 9))
+    w = rng.uniform(size=(13, 9))
+    y = orc.bag(idx, w, table)
+    ref = torch.nn.functional.embedding_bag(
+        torch.from_numpy(idx), torch.from_numpy(table), mode="sum",
+        per_sample_weights=torch.from_numpy(w)).numpy()
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-15)
+
+
+def test_bag_equal_scores_is_mean(orc):
+    """Equal scores give w = 1/k: the bag is the plain mean of the rows."""
+    rng = np.random.default_rng(3)
+    table = rng.normal(size=(20, 8))
+    idx = rng.integers(0, 20, size=(4, 5))
+    w = orc.softmax(np.zeros((4, 5)))
+    np.testing.assert_allclose(orc.bag(idx, w, table), table[idx].mean(1), rtol=1e-13)
+
+
+def test_bag_bf16_decoding_exact(orc):
+    t = torch.randn(9, 16, dtype=torch.float32).to(torch.bfloat16)
+    idx = np.arange(9).reshape(9, 1)
+    y = orc.bag(idx, np.ones((9, 1)), t)
+    np.testing.assert_array_equal(y, t.double().numpy())
+
+
+# --------------------------------------------------------------------------
+# Memory+ gate: closed forms and library special cases
+# --------------------------------------------------------------------------
+
+def test_memplus_zero_gate(orc):
+    rng = np.random.default_rng(4)
+    y, x = rng.normal(size=(5, 6)), rng.normal(size=(5, 4))
+    out = orc.memplus(y, x, np.zeros((4, 6)), rng.normal(size=(6, 4)))
+    assert np.all(out == 0.0)
+
+
+def test_memplus_identity_projection(orc):
+    """W2 = I and y = 1: out = silu(x W1) (library silu and matmul)."""
+    rng = np.random.default_rng(5)
+    x, W1 = rng.normal(size=(7, 6)), rng.normal(size=(6, 6))
+    out = orc.memplus(np.ones((7, 6)), x, W1, np.eye(6))
+    ref = torch.nn.functional.silu(torch.from_numpy(x) @ torch.from_numpy(W1)).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-15)
+
+
+def test_memplus_identity_gate_weights(orc):
+    """W1 = I (d_model = d_v), y random: out = (y ⊙ silu(x)) W2 with a
+    non-symmetric W2 (a transposed W2 fails)."""
+    rng = np.random.default_rng(6)
+    y, x, W2 = rng.normal(size=(4, 5)), rng.normal(size=(4, 5)), rng.normal(size=(5, 5))
+    out = orc.memplus(y, x, np.eye(5), W2)
+    g = torch.nn.functional.silu(torch.from_numpy(x)).numpy()
+    np.testing.assert_allclose(out, (y * g) @ W2, rtol=1e-13, atol=1e-15)
+    assert not np.allclose(out, (y * g) @ W2.T)
+
+
+def test_memplus_rectangular_shapes(orc):
+    rng = np.random.default_rng(7)
+    y, x = rng.normal(size=(3, 5)), rng.normal(size=(3, 2))
+    W1, W2 = rng.normal(size=(2, 5)), rng.normal(size=(5, 2))
+    out = orc.memplus(y, x, W1, W2)
+    assert out.shape == (3, 2)
+    # linear in y
+    np.testing.assert_allclose(orc.memplus(2.5 * y, x, W1, W2), 2.5 * out, rtol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# backward: central finite differences with the selection held fixed
+# --------------------------------------------------------------------------
+
+def _forward_fixed(orc, q, K, V, idx, n):
+    """y from the oracle's own pieces with a fixed selection idx [T,H,k]."""
+    s = orc.half_scores(q, K)  # [T,H,2,n]
+    a, b = idx // n, idx % n
+    T, H, k = idx.shape
+    S = np.take_along_axis(s[:, :, 0], a, -1) + np.take_along_axis(s[:, :, 1], b, -1)
+    w = orc.softmax(S)
+    return orc.bag(idx.reshape(T, H * k), w.reshape(T, H * k), V)
+
+
+def test_backward_finite_differences(orc):
+    T, H, dh, n, k, dv = 3, 2, 4, 5, 3, 6
+    q, K = _problem(T, H, dh, n, 80)
+    V = _rand((n * n, dv), 81)
+    dy = _rand((T, dv), 82)
+    idx, S, w, _ = orc.pkm_select(q, K, k)
+    g = orc.pkm_backward(q, K, V, idx, idx, w, dy)
+
+    def loss(q_, K_, V_):
+        return float(np.sum(dy * _forward_fixed(orc, q_, K_, V_, idx, n)))
+
+    eps = 1e-6
+    for name, arr, grad in (("q", q, g["dq"]), ("K", K, g["dK"]), ("V", V, g["dV"])):
+        num = np.zeros_like(arr)
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            p, m = arr.copy(), arr.copy()
+            p[i] += eps
+            m[i] -= eps
+            args = {"q": (q, K, V), "K": (q, K, V), "V": (q, K, V)}[name]
+            ap = [p if nm == name else a for nm, a in zip("qKV", args)]
+            am = [m if nm == name else a for nm, a in zip("qKV", args)]
+            num[i] = (loss(*ap) - loss(*am)) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+    # dw = <dy_t, V[idx]>; dS sums to zero per (t, h) (softmax Jacobian)
+    np.testing.assert_allclose(g["dS"].sum(-1), 0.0, atol=1e-14)
+    np.testing.assert_allclose(g["dw"], np.einsum("td,thkd->thk", dy, V[idx]), rtol=1e-13)
+
+
+def test_backward_matches_autograd(orc):
+    """torch.autograd (CPU, fp64) on the same composition, as a second check."""
+    T, H, dh, n, k, dv = 4, 2, 6, 4, 3, 3
+    q, K = _problem(T, H, dh, n, 90)
+    V = _rand((n * n, dv), 91)
+    dy = _rand((T, dv), 92)
+    idx, _, w, _ = orc.pkm_select(q, K, k)
+    g = orc.pkm_backward(q, K, V, idx, idx, w, dy)
+    qt = torch.tensor(q, requires_grad=True)
+    Kt = torch.tensor(K, requires_grad=True)
+    Vt = torch.tensor(V, requires_grad=True)
+    u = qt / qt.norm(dim=-1, keepdim=True)
+    kap = Kt / Kt.norm(dim=-1, keepdim=True)
+    s = math.sqrt(dh) * torch.einsum("thcd,hcnd->thcn", u, kap)
+    it = torch.from_numpy(idx)
+    S = torch.gather(s[:, :, 0], -1, it // n) + torch.gather(s[:, :, 1], -1, it % n)
+    y = (torch.softmax(S, -1).unsqueeze(-1) * Vt[it]).sum((1, 2))
+    (y * torch.from_numpy(dy)).sum().backward()
+    np.testing.assert_allclose(g["dq"], qt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(g["dK"], Kt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(g["dV"], Vt.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_compact_rows(orc):
+    """dV accumulated on a compact table equals the full-table result."""
+    T, H, dh, n, k, dv = 5, 2, 4, 6, 4, 3
+    q, K = _problem(T, H, dh, n, 95)
+    V = _rand((n * n, dv), 96)
+    dy = _rand((T, dv), 97)
+    idx, _, w, _ = orc.pkm_select(q, K, k)
+    full = orc.pkm_backward(q, K, V, idx, idx, w, dy)
+    uniq, inv = np.unique(idx, return_inverse=True)
+    comp = orc.pkm_backward(q, K, V[uniq], idx, inv.reshape(idx.shape), w, dy)
+    np.testing.assert_allclose(comp["dV"], full["dV"][uniq], rtol=1e-13)
+    np.testing.assert_array_equal(comp["dq"], full["dq"])
