@@ -1,0 +1,200 @@
+/*
+ * pkm.h -- C ABI of libpkm.so, a B200 (sm_100a) implementation of the
+ * product-key memory lookup that replaces a transformer FFN, and of its
+ * training backward.
+ *
+ * The method (web pages cited by title and section):
+ *  - "Memory Layers at Scale" digest, "Product-key 검색": every key is the
+ *    concatenation of two sub-keys, so the top-k of N keys is found with
+ *    2*sqrt(N) half-key comparisons instead of N.
+ *  - "모델 안의 메모리", "작동 방식" (and figure D): the query is split into
+ *    a front and a back half, each half is compared with its table of
+ *    sqrt(N) half-keys, the best of each are combined, a few values are read
+ *    and averaged with weights; a gate decides how much passes on.
+ *  - "Memory Layers at Scale" digest, "Memory+ 블록": gated output
+ *    (y ⊙ silu(x W1)) W2; qk-normalization for stability.
+ *  - "Memory Layers at Scale" digest, "병렬 EmbeddingBag 구현": the layer is
+ *    bound by memory bandwidth; its core is a weighted EmbeddingBag.
+ *
+ * Readings where the pages are silent (fixed by this library):
+ *  - qk-normalization: each query half and each sub-key row is divided by
+ *    max(||.||_2, 1e-12); half score s_c[a] = sqrt(d_half) * <q_c, K_c[a]>
+ *    of the normalised vectors.
+ *  - full score S(a, b) = s_1[a] + s_2[b]; value row id = a * n_sub + b.
+ *  - weights: softmax over the k selected full scores.
+ *  - heads: each head h has its own sub-key tables; all heads share one
+ *    value table; the H bags of a token are summed into one output row.
+ *  - order: larger score first; equal scores -> smaller id first.
+ *
+ * Conventions for every entry point:
+ *  - Device pointers are caller-owned, row-major, contiguous and 16-byte
+ *    aligned.  Host pointers are named so.  The library never allocates or
+ *    frees device memory; scratch comes from the caller's workspace.
+ *  - Work is enqueued on `stream` (a cudaStream_t); nothing synchronises
+ *    except pkm_get_device_error.
+ *  - Arguments are validated on the host before any launch; an invalid call
+ *    returns an error and launches nothing.
+ *  - Anomalies found on the device (an out-of-range row id, a spin-wait that
+ *    ran out, a sparse-output overflow) never trap: the offending work is
+ *    skipped and a sticky per-device status word records the first one; read
+ *    and clear it with pkm_get_device_error.
+ *  - dtype applies to query, sub-keys, values, x, W1, W2, dy and out.
+ *    Row ids are int32, weights and gradients fp32.
+ */
+#ifndef PKM_H
+#define PKM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKM_API __attribute__((visibility("default")))
+#else
+#define PKM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pkm_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    PKM_OK = 0,
+    PKM_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer */
+    PKM_ERR_UNSUPPORTED = 2, /* valid but not implemented combination */
+    PKM_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+    PKM_ERR_DEVICE = 4,      /* device status: out-of-range row id or overflow */
+    PKM_ERR_TIMEOUT = 5,     /* device status: a bounded spin-wait ran out */
+    PKM_ERR_WORKSPACE = 6    /* workspace missing or too small */
+} pkm_status;
+
+typedef enum { PKM_F32 = 0, PKM_BF16 = 1 } pkm_dtype;
+
+/*
+ * Forward of one memory layer.
+ *
+ *   query   [T, H, 2, d_half]      the two halves of each head's query
+ *   subkeys [H, 2, n_sub, d_half]  per head, the half-key tables of both halves
+ *   values  [n_sub*n_sub, d_v]     the value table (N = n_sub^2 rows)
+ *   idx     [T, H, k]  out: selected row ids a*n_sub+b, best first
+ *   weights [T, H, k]  out: softmax weights of the selected rows
+ *   out     [T, d_v]   y[t] = sum_h sum_j weights[t,h,j] * values[idx[t,h,j]]
+ *           or, with Memory+ (x, W1, W2 all non-NULL), [T, d_model]
+ *           out = (y ⊙ silu(x W1)) W2 with x [T, d_model], W1 [d_model, d_v],
+ *           W2 [d_v, d_model] (bf16 only).
+ *
+ * Limits: 1 <= k <= min(n_sub, 64); d_half, d_v, d_model multiples of 8;
+ * n_sub*n_sub < 2^31.  T = 0 is a valid empty call.
+ */
+typedef struct {
+    int64_t T;
+    int32_t H, d_half, n_sub, k, d_v;
+    pkm_dtype dtype;
+    const void *query;
+    const void *subkeys;
+    const void *values;
+    const void *x; /* Memory+ gate input, or NULL */
+    const void *W1;
+    const void *W2;
+    int32_t d_model;
+    void *out;
+    int32_t *idx;
+    float *weights;
+    void *workspace; /* device scratch of pkm_forward_workspace_size bytes */
+    size_t workspace_bytes;
+} pkm_fwd_args;
+
+/* Bytes of device workspace pkm_forward needs for these sizes (pointers
+   are not read). */
+PKM_API size_t pkm_forward_workspace_size(const pkm_fwd_args *args);
+
+/* Enqueue the forward on `stream`. */
+PKM_API pkm_status pkm_forward(const pkm_fwd_args *args, pkm_stream_t stream);
+
+/*
+ * Backward of the plain lookup (out = y), selection held fixed (top-k is
+ * piecewise constant).  With w = softmax(S):
+ *   dw_j      = <dy_t, values[idx_j]>
+ *   dS_j      = w_j (dw_j - sum_l w_l dw_l)
+ *   dvalues[r]= sum over (t,h,j) with idx = r of w_j dy_t
+ *   dquery, dsubkeys: dS through S = s_1[a] + s_2[b] and the normalisation.
+ *
+ *   idx, weights  [T, H, k]  as written by pkm_forward
+ *   dy            [T, d_v]   upstream gradient (dtype)
+ *   dquery        [T, H, 2, d_half] fp32 out (overwritten)
+ *   dsubkeys      [H, 2, n_sub, d_half] fp32 out (overwritten)
+ *   value gradient, sparse: uniq_rows int32 [uniq_cap] (ascending row ids),
+ *       grad_rows fp32 [uniq_cap, d_v], *n_uniq (device int64) = rows
+ *       written; uniq_cap >= T*H*k always suffices.  Rows beyond the cap
+ *       are dropped and the device status is set to PKM_ERR_DEVICE.
+ *   and/or dense: dvalues_dense fp32 [n_sub^2, d_v] receives += per row.
+ *   Either may be NULL (not both).  dscores [T,H,k] fp32 (optional) gets dS.
+ * Every sum runs in a fixed order: results are bitwise reproducible.
+ */
+typedef struct {
+    int64_t T;
+    int32_t H, d_half, n_sub, k, d_v;
+    pkm_dtype dtype;
+    const void *query;
+    const void *subkeys;
+    const void *values;
+    const int32_t *idx;
+    const float *weights;
+    const void *dy;
+    float *dquery;
+    float *dsubkeys;
+    int32_t *uniq_rows;
+    float *grad_rows;
+    int64_t *n_uniq;
+    int64_t uniq_cap;
+    float *dvalues_dense;
+    float *dscores;
+    void *workspace;
+    size_t workspace_bytes;
+} pkm_bwd_args;
+
+PKM_API size_t pkm_backward_workspace_size(const pkm_bwd_args *args);
+PKM_API pkm_status pkm_backward(const pkm_bwd_args *args, pkm_stream_t stream);
+
+/*
+ * Generic weighted bags ("병렬 EmbeddingBag 구현"):
+ *   out[t] = (sum_j w[t,j] * table[idx[t,j]]) [⊙ gate[t]]
+ *   table [n_rows, d] (dtype), idx int32 / w fp32 [n_bags, B],
+ *   gate NULL or [n_bags, d] (dtype), out [n_bags, d] (dtype).
+ * Accumulation is fp32 in j order, one rounding at the store.  A row id
+ * outside [0, n_rows) is skipped and sets the device status.
+ */
+PKM_API pkm_status embbag_forward(const void *table, int64_t n_rows, int32_t d, pkm_dtype dtype,
+                          const int32_t *idx, const float *w, int64_t n_bags, int32_t B,
+                          const void *gate, void *out, pkm_stream_t stream);
+
+/*
+ * Backward of embbag_forward without gate:
+ *   dw[t,j]  = <dy[t], table[idx[t,j]]>          (if table and dw non-NULL)
+ *   grad[r]  = sum over (t,j) with idx = r of w[t,j] dy[t]
+ * written sparse (uniq_rows/grad_rows/n_uniq as in pkm_bwd_args) and/or
+ * added into dense_accum [n_rows, d].  Deterministic sorted reduction.
+ */
+PKM_API size_t embbag_backward_workspace_size(int64_t n_bags, int32_t B, int32_t d, int64_t n_rows);
+PKM_API pkm_status embbag_backward(const void *dy, const int32_t *idx, const float *w,
+                           int64_t n_bags, int32_t B, int32_t d, pkm_dtype dtype,
+                           const void *table, int64_t n_rows, float *dw,
+                           int32_t *uniq_rows, float *grad_rows, int64_t *n_uniq,
+                           int64_t uniq_cap, float *dense_accum, void *workspace,
+                           size_t workspace_bytes, pkm_stream_t stream);
+
+/* Synchronise `stream`, then read and clear this device's sticky status
+   word into *code (a pkm_status value; PKM_OK when nothing happened). */
+PKM_API pkm_status pkm_get_device_error(pkm_stream_t stream, int32_t *code);
+
+/* Static description of a status code. */
+PKM_API const char *pkm_status_string(pkm_status status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+PKM_API int32_t pkm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PKM_H */

@@ -230,3 +230,12 @@ def pkm_backward(q, K, table, idx, vrow, w, dy, want_dv: bool = True):
         _p(idx), _p(vrow), _p(w), _p(da), dt, _p(dw), _p(dS), _p(dq), _p(dK),
         _p(dV) if want_dv else None), "pkm_backward")
     return dict(dw=dw, dS=dS, dq=dq, dK=dK, dV=dV)
+
+
+def full_scores(s_half, ids, n: int):
+    """S(id) = s1[id // n] + s2[id % n] for row ids ``ids`` [T,H,m], given
+    the half scores ``s_half`` [T,H,2,n] of ``half_scores``."""
+    ids = np.asarray(ids, dtype=np.int64)
+    a, b = ids // n, ids % n
+    return (np.take_along_axis(s_half[:, :, 0], a, -1)
+            + np.take_along_axis(s_half[:, :, 1], b, -1))

@@ -1,0 +1,201 @@
+"""Product-key memory lookup on B200 (sm_100a): torch-facing binding of
+libpkm.so.
+
+Every function here marshals torch tensors into the C ABI declared in
+include/pkm.h and calls it on the current CUDA stream; the computation runs
+entirely in the library's kernels.  Outputs and workspaces the caller does
+not pass are allocated with torch (device memory only); the library itself
+never allocates.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from ._lib import (PKM_BF16, PKM_F32, PKMError, BwdArgs, FwdArgs, check, load)
+
+__all__ = ["PKMError", "load", "pkm_forward", "pkm_backward", "embbag_forward",
+           "embbag_backward", "forward_workspace_size", "backward_workspace_size",
+           "device_error", "fwd_args"]
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return PKM_BF16
+    if t.dtype == torch.float32:
+        return PKM_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _stream(dev: torch.device, stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libpkm works on CUDA tensors only")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def fwd_args(T, H, d_half, n_sub, k, d_v, dtype=PKM_BF16, d_model=0, memplus=False,
+             **ptrs) -> FwdArgs:
+    a = FwdArgs()
+    a.T, a.H, a.d_half, a.n_sub, a.k, a.d_v, a.dtype = T, H, d_half, n_sub, k, d_v, dtype
+    a.d_model = d_model
+    if memplus:  # the size query only needs to know Memory+ is on
+        a.x = a.W1 = a.W2 = ctypes.c_void_p(16)
+    for name, v in ptrs.items():
+        setattr(a, name, v)
+    return a
+
+
+def forward_workspace_size(T, H, d_half, n_sub, k, d_v, dtype=PKM_BF16, memplus=False,
+                           d_model=0) -> int:
+    a = fwd_args(T, H, d_half, n_sub, k, d_v, dtype, d_model, memplus)
+    return int(load().pkm_forward_workspace_size(ctypes.byref(a)))
+
+
+def pkm_forward(query, subkeys, values, k: int, x=None, W1=None, W2=None, out=None, idx=None,
+                weights=None, workspace=None, stream=None):
+    """Forward of one memory layer (see pkm_forward in include/pkm.h).
+
+    query [T,H,2,d_half], subkeys [H,2,n_sub,d_half], values [n_sub^2, d_v];
+    optional Memory+ gate x [T,d_model], W1 [d_model,d_v], W2 [d_v,d_model].
+    Returns (out, idx, weights)."""
+    _need_cuda(query, subkeys, values, x, W1, W2)
+    T, H, two, dh = query.shape
+    n = subkeys.shape[2]
+    dv = values.shape[1]
+    dev = query.device
+    memplus = x is not None
+    dm = x.shape[1] if memplus else 0
+    if out is None:
+        out = torch.empty(T, dm if memplus else dv, dtype=query.dtype, device=dev)
+    if idx is None:
+        idx = torch.empty(T, H, k, dtype=torch.int32, device=dev)
+    if weights is None:
+        weights = torch.empty(T, H, k, dtype=torch.float32, device=dev)
+    a = fwd_args(T, H, dh, n, k, dv, _dt(query), dm, False, query=_p(query), subkeys=_p(subkeys),
+                 values=_p(values), x=_p(x), W1=_p(W1), W2=_p(W2), out=_p(out), idx=_p(idx),
+                 weights=_p(weights))
+    lib = load()
+    need = int(lib.pkm_forward_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    a.workspace, a.workspace_bytes = _p(workspace), workspace.numel()
+    check(lib.pkm_forward(ctypes.byref(a), _stream(dev, stream)), "pkm_forward")
+    return out, idx, weights
+
+
+def _bwd_args(query, subkeys, values, idx, weights, dy, **kw) -> BwdArgs:
+    T, H, _, dh = query.shape
+    a = BwdArgs()
+    a.T, a.H, a.d_half, a.n_sub, a.k, a.d_v = T, H, dh, subkeys.shape[2], idx.shape[2], \
+        values.shape[1]
+    a.dtype = _dt(query)
+    a.query, a.subkeys, a.values = _p(query), _p(subkeys), _p(values)
+    a.idx, a.weights, a.dy = _p(idx), _p(weights), _p(dy)
+    for name, v in kw.items():
+        setattr(a, name, v)
+    return a
+
+
+def backward_workspace_size(query, subkeys, values, idx, weights, dy) -> int:
+    a = _bwd_args(query, subkeys, values, idx, weights, dy)
+    return int(load().pkm_backward_workspace_size(ctypes.byref(a)))
+
+
+def pkm_backward(query, subkeys, values, idx, weights, dy, sparse: bool = True,
+                 dense: Optional[torch.Tensor] = None, want_dscores: bool = False,
+                 workspace=None, stream=None, uniq_cap: Optional[int] = None):
+    """Backward of the plain lookup (see pkm_backward in include/pkm.h).
+
+    Returns dict(dquery, dsubkeys, uniq_rows, grad_rows, n_uniq, dscores)
+    with the sparse value gradient sliced to its n_uniq rows (a host read of
+    n_uniq) when ``sparse``; ``dense`` [N, d_v] fp32 receives += if given."""
+    _need_cuda(query, subkeys, values, idx, weights, dy, dense)
+    T, H, _, dh = query.shape
+    dev = query.device
+    k = idx.shape[2]
+    R = T * H * k
+    dq = torch.empty(T, H, 2, dh, dtype=torch.float32, device=dev)
+    dK = torch.empty_like(subkeys, dtype=torch.float32)
+    cap = R if uniq_cap is None else uniq_cap
+    uniq = torch.empty(max(cap, 1), dtype=torch.int32, device=dev) if sparse else None
+    grad = torch.empty(max(cap, 1), values.shape[1], dtype=torch.float32, device=dev) \
+        if sparse else None
+    n_uniq = torch.zeros(1, dtype=torch.int64, device=dev) if sparse else None
+    dS = torch.empty(T, H, k, dtype=torch.float32, device=dev) if want_dscores else None
+    a = _bwd_args(query, subkeys, values, idx, weights, dy, dquery=_p(dq), dsubkeys=_p(dK),
+                  uniq_rows=_p(uniq), grad_rows=_p(grad), n_uniq=_p(n_uniq),
+                  uniq_cap=cap if sparse else 0, dvalues_dense=_p(dense), dscores=_p(dS))
+    lib = load()
+    need = int(lib.pkm_backward_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    a.workspace, a.workspace_bytes = _p(workspace), workspace.numel()
+    check(lib.pkm_backward(ctypes.byref(a), _stream(dev, stream)), "pkm_backward")
+    res = dict(dquery=dq, dsubkeys=dK, dscores=dS, n_uniq=n_uniq)
+    if sparse:
+        u = int(n_uniq.item())
+        res.update(uniq_rows=uniq[:u], grad_rows=grad[:u])
+    return res
+
+
+def embbag_forward(table, idx, w, gate=None, out=None, stream=None):
+    """out[t] = (sum_j w[t,j] table[idx[t,j]]) (⊙ gate[t]); idx int32, w fp32 [n_bags, B]."""
+    _need_cuda(table, idx, w, gate)
+    n_bags, B = idx.shape
+    d = table.shape[1]
+    if out is None:
+        out = torch.empty(n_bags, d, dtype=table.dtype, device=table.device)
+    check(load().embbag_forward(_p(table), table.shape[0], d, _dt(table), _p(idx), _p(w),
+                                n_bags, B, _p(gate), _p(out), _stream(table.device, stream)),
+          "embbag_forward")
+    return out
+
+
+def embbag_backward(dy, idx, w, table=None, n_rows=None, sparse=True, dense=None,
+                    want_dw=False, stream=None):
+    """Backward of embbag_forward (no gate); see include/pkm.h."""
+    _need_cuda(dy, idx, w, table, dense)
+    n_bags, B = idx.shape
+    d = dy.shape[1]
+    dev = dy.device
+    n_rows = table.shape[0] if n_rows is None else n_rows
+    R = n_bags * B
+    dw = torch.empty(n_bags, B, dtype=torch.float32, device=dev) if want_dw else None
+    uniq = torch.empty(max(R, 1), dtype=torch.int32, device=dev) if sparse else None
+    grad = torch.empty(max(R, 1), d, dtype=torch.float32, device=dev) if sparse else None
+    n_uniq = torch.zeros(1, dtype=torch.int64, device=dev) if sparse else None
+    lib = load()
+    need = int(lib.embbag_backward_workspace_size(n_bags, B, d, n_rows))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    check(lib.embbag_backward(_p(dy), _p(idx), _p(w), n_bags, B, d, _dt(dy), _p(table), n_rows,
+                              _p(dw), _p(uniq), _p(grad), _p(n_uniq), R if sparse else 0,
+                              _p(dense), _p(ws), ws.numel(), _stream(dev, stream)),
+          "embbag_backward")
+    res = dict(dw=dw)
+    if sparse:
+        u = int(n_uniq.item())
+        res.update(uniq_rows=uniq[:u], grad_rows=grad[:u])
+    return res
+
+
+def device_error(stream=None, device=None) -> int:
+    """Synchronise and read-and-clear the device status word (0 = none)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    code = ctypes.c_int32(0)
+    check(load().pkm_get_device_error(_stream(dev, stream), ctypes.byref(code)),
+          "pkm_get_device_error")
+    return int(code.value)

@@ -1,0 +1,91 @@
+"""ctypes binding of libpkm.so (argument marshalling only).
+
+Every step of the lookup runs in the library's CUDA kernels; this module
+only turns torch tensors into pointers and sizes and raises on a non-OK
+status.  It fails loudly if the library is missing: there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libpkm.so")
+
+PKM_OK = 0
+STATUS = {0: "PKM_OK", 1: "PKM_ERR_INVALID_ARG", 2: "PKM_ERR_UNSUPPORTED", 3: "PKM_ERR_CUDA",
+          4: "PKM_ERR_DEVICE", 5: "PKM_ERR_TIMEOUT", 6: "PKM_ERR_WORKSPACE"}
+PKM_F32, PKM_BF16 = 0, 1
+
+P = ctypes.c_void_p
+I32, I64, SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+
+class PKMError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+
+
+class FwdArgs(ctypes.Structure):
+    _fields_ = [("T", I64), ("H", I32), ("d_half", I32), ("n_sub", I32), ("k", I32),
+                ("d_v", I32), ("dtype", ctypes.c_int), ("query", P), ("subkeys", P),
+                ("values", P), ("x", P), ("W1", P), ("W2", P), ("d_model", I32), ("out", P),
+                ("idx", P), ("weights", P), ("workspace", P), ("workspace_bytes", SZ)]
+
+
+class BwdArgs(ctypes.Structure):
+    _fields_ = [("T", I64), ("H", I32), ("d_half", I32), ("n_sub", I32), ("k", I32),
+                ("d_v", I32), ("dtype", ctypes.c_int), ("query", P), ("subkeys", P),
+                ("values", P), ("idx", P), ("weights", P), ("dy", P), ("dquery", P),
+                ("dsubkeys", P), ("uniq_rows", P), ("grad_rows", P), ("n_uniq", P),
+                ("uniq_cap", I64), ("dvalues_dense", P), ("dscores", P), ("workspace", P),
+                ("workspace_bytes", SZ)]
+
+
+EXPORTS = ("pkm_forward_workspace_size", "pkm_forward", "pkm_backward_workspace_size",
+           "pkm_backward", "embbag_forward", "embbag_backward_workspace_size",
+           "embbag_backward", "pkm_get_device_error", "pkm_status_string", "pkm_version")
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libpkm.so and declare its signatures (raises if it is missing)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libpkm.so not built at {path}; run python -m sparse_key_value_b200.build")
+    lib = ctypes.CDLL(path)
+    FA, BA = ctypes.POINTER(FwdArgs), ctypes.POINTER(BwdArgs)
+    lib.pkm_forward_workspace_size.argtypes = [FA]
+    lib.pkm_forward_workspace_size.restype = SZ
+    lib.pkm_forward.argtypes = [FA, P]
+    lib.pkm_forward.restype = ctypes.c_int
+    lib.pkm_backward_workspace_size.argtypes = [BA]
+    lib.pkm_backward_workspace_size.restype = SZ
+    lib.pkm_backward.argtypes = [BA, P]
+    lib.pkm_backward.restype = ctypes.c_int
+    lib.embbag_forward.argtypes = [P, I64, I32, ctypes.c_int, P, P, I64, I32, P, P, P]
+    lib.embbag_forward.restype = ctypes.c_int
+    lib.embbag_backward_workspace_size.argtypes = [I64, I32, I32, I64]
+    lib.embbag_backward_workspace_size.restype = SZ
+    lib.embbag_backward.argtypes = [P, P, P, I64, I32, I32, ctypes.c_int, P, I64, P, P, P, P,
+                                    I64, P, P, SZ, P]
+    lib.embbag_backward.restype = ctypes.c_int
+    lib.pkm_get_device_error.argtypes = [P, ctypes.POINTER(I32)]
+    lib.pkm_get_device_error.restype = ctypes.c_int
+    lib.pkm_status_string.argtypes = [ctypes.c_int]
+    lib.pkm_status_string.restype = ctypes.c_char_p
+    lib.pkm_version.argtypes = []
+    lib.pkm_version.restype = I32
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def check(code: int, what: str):
+    if code != PKM_OK:
+        raise PKMError(code, what)

@@ -1,0 +1,107 @@
+// k_gemm.cu -- dense pieces of the Memory+ block ("Memory Layers at
+// Scale" digest, "Memory+ 블록": out = (y ⊙ silu(x W1)) W2).
+//
+// The weights arrive row-major ([d_model, d_v] and [d_v, d_model]); a small
+// transpose puts each into the K-major layout both GEMM operands use.  The
+// GEMM runs on the tensor cores (k_gemm_tc.cu) when the shape allows it,
+// else on this SIMT kernel.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pkm {
+
+__global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src, int rows, int cols,
+                                      __nv_bfloat16* __restrict__ dst) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = src[(int64_t)r * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int c = c0 + i, r = r0 + threadIdx.x;  // dst[c][r] = src[r][c]
+    if (r < rows && c < cols) dst[(int64_t)c * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,
+                                  cudaStream_t stream) {
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32), block(32, 8);
+  transpose_bf16_kernel<<<grid, block, 0, stream>>>((const __nv_bfloat16*)src, rows, cols,
+                                                    (__nv_bfloat16*)dst);
+  return cudaGetLastError();
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+// C[M,N] = epi(sum_k A[m,k] B[n,k]); 64x64 tile, 256 threads, 4x4 each.
+__global__ void __launch_bounds__(256) gemm_simt_kernel(const __nv_bfloat16* __restrict__ A,
+                                                        const __nv_bfloat16* __restrict__ B,
+                                                        int64_t M, int N, int K, int epi,
+                                                        __nv_bfloat16* __restrict__ C) {
+  __shared__ float As[16][64 + 1];
+  __shared__ float Bs[16][64 + 1];
+  const int64_t m0 = (int64_t)blockIdx.y * 64;
+  const int n0 = blockIdx.x * 64;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      int r = i / 16, kk = i % 16;
+      int64_t m = m0 + r;
+      int nn = n0 + r;
+      As[kk][r] = (m < M && k0 + kk < K) ? __bfloat162float(A[m * K + k0 + kk]) : 0.f;
+      Bs[kk][r] = (nn < N && k0 + kk < K) ? __bfloat162float(B[(int64_t)nn * K + k0 + kk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int64_t m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int nn = n0 + tx * 4 + j;
+      if (nn >= N) continue;
+      float v = acc[i][j];
+      if (epi == 1) v = silu_f(v);
+      C[m * N + nn] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+cudaError_t launch_gemm_simt(const void* A, const void* B, int64_t M, int N, int K, int epi,
+                             void* C, cudaStream_t stream) {
+  dim3 grid((N + 63) / 64, (unsigned)((M + 63) / 64));
+  gemm_simt_kernel<<<grid, 256, 0, stream>>>((const __nv_bfloat16*)A, (const __nv_bfloat16*)B,
+                                             M, N, K, epi, (__nv_bfloat16*)C);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
+                           void* C, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
+                             void* C, int32_t* status, cudaStream_t stream) {
+  if (M <= 0) return cudaSuccess;
+  if (gemm_tc_supported(M, N, K)) return launch_gemm_tc(A, B, M, N, K, epi, C, status, stream);
+  return launch_gemm_simt(A, B, M, N, K, epi, C, stream);
+}
+
+}  // namespace pkm

@@ -1,0 +1,66 @@
+// kernels.h -- internal launchers of libpkm.so (host side, C++).  Each
+// launcher enqueues its kernel(s) on `stream` and returns the launch error.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pkm.h"
+
+namespace pkm {
+
+// r[i] = 1 / max(||x[i, :]||_2, 1e-12) for rows of d elements.
+cudaError_t launch_row_rnorm(const void* x, pkm_dtype dt, int64_t rows, int d, float* r,
+                             cudaStream_t stream);
+
+// Per-half top-k lists of the sub-key scores, SIMT cores (any dtype, k <= 64).
+//   hv/hi [T, H, 2, k]: s_c and the sub-key position a, best first.
+cudaError_t launch_score_topk_simt(const void* q, const void* K, pkm_dtype dt, int64_t T,
+                                   int H, int dh, int n, int k, const float* rq,
+                                   const float* rk, float* hv, int32_t* hi,
+                                   cudaStream_t stream);
+
+// Same lists on the tensor cores (tcgen05, bf16, k <= 32).  `splits` > 1
+// cuts each sub-key table into that many column ranges, written as
+// separate lists hv/hi [splits][T, H, 2, k] that the combine step merges.
+bool score_tc_supported(pkm_dtype dt, int dh, int n, int k);
+int score_tc_splits(int64_t T, int H, int n);
+cudaError_t launch_score_topk_tc(const void* q, const void* K, int64_t T, int H, int dh, int n,
+                                 int k, int splits, const float* rq, const float* rk, float* hv,
+                                 int32_t* hi, int32_t* status, cudaStream_t stream);
+
+// Merge the split lists, combine the two halves' k x k candidates, keep the
+// top k, softmax -> idx [T,H,k] (a*n+b), w [T,H,k].
+cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64_t T, int H,
+                           int n, int k, int32_t* idx, float* w, cudaStream_t stream);
+
+// out[t] = sum_j w[t,j] * table[idx[t,j]] (⊙ gate[t])
+cudaError_t launch_embbag_fwd(const void* table, int64_t n_rows, int d, pkm_dtype dt,
+                              const int32_t* idx, const float* w, int64_t n_bags, int B,
+                              const void* gate, void* out, int32_t* status,
+                              cudaStream_t stream);
+
+// Memory+ helpers (bf16).
+cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,
+                                  cudaStream_t stream);
+// C[M,N] = epi(A[M,K] * B[N,K]^T), A/B bf16 K-major; epi: 0 none, 1 silu.
+// Optional `mul` [M,N] bf16 multiplies the result after the epilogue.
+bool gemm_tc_supported(int64_t M, int N, int K);
+cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
+                             void* C, int32_t* status, cudaStream_t stream);
+
+// ---------------------------------------------------------------- backward
+// dw[t,j] = <dy[t], table[idx[t,j]]>; with H>0 also dS = w (dw - sum w dw)
+// per (t, h) group of k.
+cudaError_t launch_bag_dw(const void* dy, const void* table, int64_t n_rows, int d,
+                          pkm_dtype dt, const int32_t* idx, const float* w, int64_t n_bags,
+                          int B, int group, float* dw, float* dS, int32_t* status,
+                          cudaStream_t stream);
+
+// Stable LSD radix sort of (key, value) pairs, key < 2^key_bits.
+size_t radix_sort_workspace(int64_t n);
+cudaError_t launch_radix_sort(const uint32_t* keys_in, const uint32_t* vals_in, int64_t n,
+                              int key_bits, uint32_t* keys_out, uint32_t* vals_out,
+                              void* workspace, cudaStream_t stream);
+
+}  // namespace pkm

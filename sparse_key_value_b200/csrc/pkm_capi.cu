@@ -1,0 +1,209 @@
+// pkm_capi.cu -- the C ABI of libpkm.so: argument validation, workspace
+// carving and the launch sequence of each entry point (see include/pkm.h).
+#include <mutex>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pkm {
+
+__device__ int32_t g_status = 0;  // sticky per-device status word
+
+static std::mutex g_status_mu;
+static int32_t* g_status_ptr[64] = {nullptr};
+
+// Device address of this device's status word (looked up once per device).
+static int32_t* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------ forward ----
+
+struct FwdLayout {
+  size_t rq, rk, hv, hi, w1t, w2t, g, z, total;
+  int splits;
+  bool tc;
+};
+
+static bool has_memplus(const pkm_fwd_args* a) { return a->x || a->W1 || a->W2; }
+
+static FwdLayout fwd_layout(const pkm_fwd_args* a) {
+  FwdLayout L{};
+  const size_t T = (size_t)(a->T > 0 ? a->T : 0);
+  const size_t H = (size_t)a->H, n = (size_t)a->n_sub, k = (size_t)a->k;
+  L.tc = score_tc_supported(a->dtype, a->d_half, a->n_sub, a->k);
+  L.splits = L.tc ? score_tc_splits(a->T, a->H, a->n_sub) : 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = round_up(off + bytes, 256);
+    return o;
+  };
+  L.rq = take(T * H * 2 * sizeof(float));
+  L.rk = take(H * 2 * n * sizeof(float));
+  L.hv = take((size_t)L.splits * T * H * 2 * k * sizeof(float));
+  L.hi = take((size_t)L.splits * T * H * 2 * k * sizeof(int32_t));
+  if (has_memplus(a)) {
+    const size_t dm = (size_t)a->d_model, dv = (size_t)a->d_v;
+    L.w1t = take(dv * dm * 2);
+    L.w2t = take(dm * dv * 2);
+    L.g = take(T * dv * 2);
+    L.z = take(T * dv * 2);
+  }
+  L.total = off;
+  return L;
+}
+
+static pkm_status validate_fwd(const pkm_fwd_args* a) {
+  if (!a) return PKM_ERR_INVALID_ARG;
+  if (a->T < 0 || a->H < 1 || a->n_sub < 1 || a->k < 1 || a->k > 64 || a->k > a->n_sub)
+    return PKM_ERR_INVALID_ARG;
+  if (a->d_half < 8 || a->d_half % 8 || a->d_v < 8 || a->d_v % 8) return PKM_ERR_INVALID_ARG;
+  if ((int64_t)a->n_sub * a->n_sub >= (int64_t(1) << 31)) return PKM_ERR_INVALID_ARG;
+  if (a->dtype != PKM_F32 && a->dtype != PKM_BF16) return PKM_ERR_INVALID_ARG;
+  if (a->H * a->k > 4096) return PKM_ERR_INVALID_ARG;
+  if (a->d_half > 2048) return PKM_ERR_UNSUPPORTED;
+  if (a->T == 0) return PKM_OK;
+  const void* need[] = {a->query, a->subkeys, a->values, a->out, a->idx, a->weights};
+  for (const void* p : need)
+    if (!p || !aligned16(p)) return PKM_ERR_INVALID_ARG;
+  if (has_memplus(a)) {
+    if (!a->x || !a->W1 || !a->W2) return PKM_ERR_INVALID_ARG;
+    if (!aligned16(a->x) || !aligned16(a->W1) || !aligned16(a->W2)) return PKM_ERR_INVALID_ARG;
+    if (a->d_model < 8 || a->d_model % 8) return PKM_ERR_INVALID_ARG;
+    if (a->dtype != PKM_BF16) return PKM_ERR_UNSUPPORTED;
+  }
+  const FwdLayout L = fwd_layout(a);
+  if (!a->workspace || !aligned16(a->workspace) || a->workspace_bytes < L.total)
+    return PKM_ERR_WORKSPACE;
+  return PKM_OK;
+}
+
+#define PKM_TRY(expr)                          \
+  do {                                         \
+    cudaError_t e_ = (expr);                   \
+    if (e_ != cudaSuccess) return PKM_ERR_CUDA; \
+  } while (0)
+
+static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
+  int32_t* status = status_ptr();
+  if (!status) return PKM_ERR_CUDA;
+  const FwdLayout L = fwd_layout(a);
+  char* ws = static_cast<char*>(a->workspace);
+  float* rq = reinterpret_cast<float*>(ws + L.rq);
+  float* rk = reinterpret_cast<float*>(ws + L.rk);
+  float* hv = reinterpret_cast<float*>(ws + L.hv);
+  int32_t* hi = reinterpret_cast<int32_t*>(ws + L.hi);
+  const int64_t T = a->T;
+  const int H = a->H, dh = a->d_half, n = a->n_sub, k = a->k;
+
+  // a1: qk-normalisation factors
+  PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
+  PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
+  // a2 + a3: sub-key scores and per-half top-k
+  if (L.tc)
+    PKM_TRY(launch_score_topk_tc(a->query, a->subkeys, T, H, dh, n, k, L.splits, rq, rk, hv, hi,
+                                 status, st));
+  else
+    PKM_TRY(launch_score_topk_simt(a->query, a->subkeys, a->dtype, T, H, dh, n, k, rq, rk, hv,
+                                   hi, st));
+  // a4 + a5: k x k combine, top-k, softmax
+  PKM_TRY(launch_combine(hv, hi, L.splits, T, H, n, k, a->idx, a->weights, st));
+  // a6 (+ a7): bag gather over the H*k selected rows of each token
+  const int64_t N = (int64_t)n * n;
+  if (!has_memplus(a)) {
+    PKM_TRY(launch_embbag_fwd(a->values, N, a->d_v, a->dtype, a->idx, a->weights, T, H * k,
+                              nullptr, a->out, status, st));
+    return PKM_OK;
+  }
+  void* w1t = ws + L.w1t;
+  void* w2t = ws + L.w2t;
+  void* g = ws + L.g;
+  void* z = ws + L.z;
+  const int dm = a->d_model, dv = a->d_v;
+  PKM_TRY(launch_transpose_bf16(a->W1, dm, dv, w1t, st));  // [dv, dm]
+  PKM_TRY(launch_transpose_bf16(a->W2, dv, dm, w2t, st));  // [dm, dv]
+  PKM_TRY(launch_gemm_bf16(a->x, w1t, T, dv, dm, /*silu*/ 1, g, status, st));
+  PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g, z,
+                            status, st));
+  PKM_TRY(launch_gemm_bf16(z, w2t, T, dm, dv, /*none*/ 0, a->out, status, st));
+  return PKM_OK;
+}
+
+}  // namespace pkm
+
+using namespace pkm;
+
+extern "C" {
+
+size_t pkm_forward_workspace_size(const pkm_fwd_args* args) {
+  if (!args) return 0;
+  return fwd_layout(args).total;
+}
+
+pkm_status pkm_forward(const pkm_fwd_args* args, pkm_stream_t stream) {
+  pkm_status s = validate_fwd(args);
+  if (s != PKM_OK || args->T == 0) return s;
+  return forward_impl(args, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pkm_status embbag_forward(const void* table, int64_t n_rows, int32_t d, pkm_dtype dtype,
+                          const int32_t* idx, const float* w, int64_t n_bags, int32_t B,
+                          const void* gate, void* out, pkm_stream_t stream) {
+  if (n_bags < 0 || n_rows < 1 || d < 8 || d % 8 || B < 1 || B > 4096)
+    return PKM_ERR_INVALID_ARG;
+  if (dtype != PKM_F32 && dtype != PKM_BF16) return PKM_ERR_INVALID_ARG;
+  if (n_bags == 0) return PKM_OK;
+  if (!table || !idx || !w || !out || !aligned16(table) || !aligned16(out) ||
+      (gate && !aligned16(gate)))
+    return PKM_ERR_INVALID_ARG;
+  int32_t* status = status_ptr();
+  if (!status) return PKM_ERR_CUDA;
+  cudaError_t e = launch_embbag_fwd(table, n_rows, d, dtype, idx, w, n_bags, B, gate, out,
+                                    status, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
+}
+
+pkm_status pkm_get_device_error(pkm_stream_t stream, int32_t* code) {
+  if (!code) return PKM_ERR_INVALID_ARG;
+  int32_t* status = status_ptr();
+  if (!status) return PKM_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, status, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return PKM_ERR_CUDA;
+  if (cudaMemsetAsync(status, 0, sizeof v, st) != cudaSuccess) return PKM_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PKM_ERR_CUDA;
+  *code = v;
+  return PKM_OK;
+}
+
+const char* pkm_status_string(pkm_status s) {
+  switch (s) {
+    case PKM_OK: return "ok";
+    case PKM_ERR_INVALID_ARG: return "invalid argument";
+    case PKM_ERR_UNSUPPORTED: return "unsupported combination";
+    case PKM_ERR_CUDA: return "CUDA call failed";
+    case PKM_ERR_DEVICE: return "device anomaly: row id out of range or output overflow";
+    case PKM_ERR_TIMEOUT: return "device spin-wait ran out";
+    case PKM_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int32_t pkm_version(void) { return 100; }
+
+}  // extern "C"

@@ -55,6 +55,12 @@ class Workload:
     zipf_alpha: float = 0.0
     zipf_beta: float = 0.0
     zipf_gamma: float = 0.0
+    # seed of the parameter tables (sub-keys, values, W1, W2); defaults to seed
+    table_seed_: int = -1
+
+    @property
+    def table_seed(self) -> int:
+        return self.seed if self.table_seed_ < 0 else self.table_seed_
 
     @property
     def N(self) -> int:
@@ -98,7 +104,7 @@ WORKLOADS = {
                       zipf_alpha=0.5, zipf_beta=1.0, zipf_gamma=1.0),
     "decode": Workload("decode", T=8, H=4, d_half=512, n_sub=4096, k=32, d_v=1024,
                        dtype="bf16", seed=1005, memplus=True, d_model=1024,
-                       decode_steps=256),
+                       decode_steps=256, table_seed_=1003),
 }
 
 _DEVICE_GEN_BYTES = 64 << 20
@@ -120,11 +126,11 @@ def value_table(w: Workload, device) -> torch.Tensor:
     rows, d = w.N, w.d_v
     out = torch.empty(rows, d, dtype=w.torch_dtype, device=device)
     if device.type == "cpu" or rows * d * w.elem_bytes <= _DEVICE_GEN_BYTES:
-        g = _cpu_gen(w.seed + 7)
+        g = _cpu_gen(w.table_seed + 7)
         out.copy_(_randn((rows, d), 0.02, g))
         return out
     g = torch.Generator(device=device)
-    g.manual_seed(w.seed + 7)
+    g.manual_seed(w.table_seed + 7)
     chunk = max(1, (32 << 20) // d)  # 32 Mi elements per draw
     for r0 in range(0, rows, chunk):
         r1 = min(rows, r0 + chunk)
@@ -140,29 +146,35 @@ def _zipf_direction(w: Workload, g: torch.Generator) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, device="cpu", with_values: bool = True) -> dict:
-    """All inputs of one forward (and, for ``train``, backward) of ``w``."""
-    g = _cpu_gen(w.seed)
+    """All inputs of one forward (and, for ``train``, backward) of ``w``.
+
+    Each tensor family has its own generator stream, so the tables do not
+    depend on T: the decode workload reuses the Memory+ tables exactly.
+    """
+    ts = w.table_seed
     dt = w.torch_dtype
-    q = _randn((w.T, w.H, 2, w.d_half), 1.0, g)
-    K = _randn((w.H, 2, w.n_sub, w.d_half), 1.0 / math.sqrt(w.d_half), g)
+    q = _randn((w.T, w.H, 2, w.d_half), 1.0, _cpu_gen(w.seed))
+    gk = _cpu_gen(ts + 1)
+    K = _randn((w.H, 2, w.n_sub, w.d_half), 1.0 / math.sqrt(w.d_half), gk)
     if w.zipf_beta > 0.0:
-        e = _zipf_direction(w, g)  # [H, 2, d_half]
+        e = _zipf_direction(w, gk)  # [H, 2, d_half]
         rank = torch.empty(w.H, 2, w.n_sub, dtype=torch.float32)
         for h in range(w.H):
             for c in range(2):
-                perm = torch.randperm(w.n_sub, generator=g)
+                perm = torch.randperm(w.n_sub, generator=gk)
                 rank[h, c, perm] = torch.arange(w.n_sub, dtype=torch.float32)
         amp = w.zipf_beta * (rank + 1.0).pow(-w.zipf_alpha)  # [H,2,n]
         K = K + amp.unsqueeze(-1) * e.unsqueeze(2)
         q = q + w.zipf_gamma * e.unsqueeze(0)
     out = dict(query=q.to(dt).to(device), subkeys=K.to(dt).to(device))
     if w.memplus:
-        out["x"] = _randn((w.T, w.d_model), 1.0, g).to(dt).to(device)
+        out["x"] = _randn((w.T, w.d_model), 1.0, _cpu_gen(w.seed + 2)).to(dt).to(device)
+        gw = _cpu_gen(ts + 3)
         s = 1.0 / math.sqrt(1024.0)
-        out["W1"] = _randn((w.d_model, w.d_v), s, g).to(dt).to(device)
-        out["W2"] = _randn((w.d_v, w.d_model), s, g).to(dt).to(device)
+        out["W1"] = _randn((w.d_model, w.d_v), s, gw).to(dt).to(device)
+        out["W2"] = _randn((w.d_v, w.d_model), s, gw).to(dt).to(device)
     if w.train:
-        out["dy"] = _randn((w.T, w.d_v), 1.0, g).to(dt).to(device)
+        out["dy"] = _randn((w.T, w.d_v), 1.0, _cpu_gen(w.seed + 4)).to(dt).to(device)
     if with_values:
         out["values"] = value_table(w, device)
     return out

@@ -1,0 +1,117 @@
+"""The C ABI on the host: the library loads without a GPU, exports every
+symbol the header declares, and rejects invalid arguments before any launch
+(no compute call is made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_key_value_b200 import build
+    build.build()
+    from sparse_key_value_b200 import _lib
+    return _lib.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"PKM_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ("pkm_forward", "pkm_backward", "embbag_forward", "embbag_backward",
+              "pkm_forward_workspace_size", "pkm_backward_workspace_size",
+              "embbag_backward_workspace_size", "pkm_get_device_error", "pkm_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} not exported"
+    from sparse_key_value_b200 import _lib
+    assert set(_lib.EXPORTS) <= set(declared_symbols())
+
+
+def test_only_the_c_abi_is_exported():
+    from sparse_key_value_b200 import _lib
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert exported == set(declared_symbols())
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.pkm_status_string(code)
+    assert lib.pkm_version() >= 100
+
+
+def _fwd(**kw):
+    from sparse_key_value_b200 import fwd_args
+    base = dict(T=64, H=2, d_half=64, n_sub=32, k=8, d_v=64)
+    base.update(kw)
+    fake = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced on the host
+    a = fwd_args(**base, query=fake, subkeys=fake, values=fake, out=fake, idx=fake,
+                 weights=fake, workspace=fake)
+    return a
+
+
+@pytest.mark.parametrize("bad", [dict(k=0), dict(k=33, n_sub=32), dict(k=65, n_sub=100),
+                                 dict(d_half=60), dict(d_v=12), dict(H=0), dict(n_sub=0),
+                                 dict(n_sub=46341), dict(T=-1), dict(dtype=7)])
+def test_forward_rejects_bad_sizes(lib, bad):
+    a = _fwd(**bad)
+    a.workspace_bytes = 1 << 40
+    assert lib.pkm_forward(ctypes.byref(a), None) == 1
+
+
+def test_forward_rejects_null_and_misaligned(lib):
+    a = _fwd()
+    a.workspace_bytes = 1 << 40
+    a.query = None
+    assert lib.pkm_forward(ctypes.byref(a), None) == 1
+    a = _fwd()
+    a.workspace_bytes = 1 << 40
+    a.values = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.pkm_forward(ctypes.byref(a), None) == 1
+
+
+def test_forward_workspace_checks(lib):
+    a = _fwd()
+    need = lib.pkm_forward_workspace_size(ctypes.byref(a))
+    assert need > 0
+    a.workspace_bytes = need - 1
+    assert lib.pkm_forward(ctypes.byref(a), None) == 6
+    bigger = _fwd(T=128)
+    assert lib.pkm_forward_workspace_size(ctypes.byref(bigger)) > need
+
+
+def test_forward_empty_batch_is_ok_without_gpu(lib):
+    a = _fwd(T=0)
+    assert lib.pkm_forward(ctypes.byref(a), None) == 0
+
+
+def test_memplus_requires_all_three_and_bf16(lib):
+    a = _fwd(d_model=64)
+    a.workspace_bytes = 1 << 40
+    a.x = ctypes.c_void_p(1 << 20)
+    assert lib.pkm_forward(ctypes.byref(a), None) == 1  # W1, W2 missing
+    a.W1 = a.W2 = ctypes.c_void_p(1 << 20)
+    a.dtype = 0  # fp32 Memory+
+    assert lib.pkm_forward(ctypes.byref(a), None) == 2
+
+
+def test_embbag_rejects_bad_args(lib):
+    P = ctypes.c_void_p
+    f = P(1 << 20)
+    assert lib.embbag_forward(f, 10, 12, 1, f, f, 4, 3, None, f, None) == 1   # d % 8
+    assert lib.embbag_forward(f, 10, 16, 1, f, f, 4, 0, None, f, None) == 1   # B = 0
+    assert lib.embbag_forward(None, 10, 16, 1, f, f, 4, 3, None, f, None) == 1
+    assert lib.embbag_forward(f, 10, 16, 1, f, f, 0, 3, None, f, None) == 0   # no bags

@@ -1,0 +1,175 @@
+"""GPU parity of the forward path against the CPU oracle (through the C ABI)."""
+
+import numpy as np
+import pytest
+import torch
+
+from parity import RTOL, W_RTOL, close, forward_reference, weights_close
+
+pytestmark = pytest.mark.gpu
+
+skv = pytest.importorskip("sparse_key_value_b200")
+from sparse_key_value_b200.inputs import WORKLOADS, make_inputs, random_bags  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    skv.load()
+    yield
+    assert skv.device_error() == 0
+
+
+def run_forward(w, inp=None, sample=None):
+    """Run the GPU forward of workload ``w`` and check it against the oracle
+    on the tokens ``sample`` (all tokens by default)."""
+    import oracle
+
+    if inp is None:
+        inp = make_inputs(w, "cuda")
+    mp = w.memplus
+    out, idx, wts = skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k,
+                                    x=inp.get("x") if mp else None,
+                                    W1=inp.get("W1") if mp else None,
+                                    W2=inp.get("W2") if mp else None)
+    torch.cuda.synchronize()
+    assert skv.device_error() == 0
+    if sample is None:
+        sample = torch.arange(w.T)
+    sample = torch.as_tensor(sample, dtype=torch.long)
+    sd = sample.to("cuda")
+    idx_g = idx[sd].cpu().numpy().astype(np.int64)
+    rows = np.unique(idx_g)
+    table_rows = inp["values"][torch.from_numpy(rows).to("cuda")].cpu()
+    ref = forward_reference(inp["query"][sd].cpu(), inp["subkeys"].cpu(), w.k, idx_g,
+                            table_rows, rows, w.n_sub,
+                            x=inp["x"][sd].cpu() if mp else None,
+                            W1=inp["W1"].cpu() if mp else None,
+                            W2=inp["W2"].cpu() if mp else None)
+    weights_close(wts[sd].cpu().numpy(), ref["w_ref"], W_RTOL[w.dtype])
+    err = close(out[sd].float().cpu().numpy(), ref["out_ref"], RTOL[w.dtype], "out")
+    n_th = len(sample) * w.H
+    assert ref["exempt"] <= max(1, 0.01 * n_th), f"{ref['exempt']} tie exemptions of {n_th}"
+    return dict(ref=ref, idx=idx_g, err=err, inp=inp)
+
+
+SMALL = [
+    # name, T, H, d_half, n_sub, k, d_v, dtype
+    ("bf16-ragged", 300, 2, 64, 64, 16, 128, "bf16"),
+    ("bf16-k32-odd-n", 129, 3, 128, 100, 32, 64, "bf16"),
+    ("bf16-minimal", 1, 1, 8, 3, 1, 8, "bf16"),
+    ("bf16-wide", 37, 4, 512, 300, 32, 2048, "bf16"),
+    ("f32-k64", 70, 2, 32, 64, 64, 40, "f32"),
+    ("f32-k-equals-n", 33, 1, 16, 5, 5, 24, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_forward_small(case):
+    name, T, H, dh, n, k, dv, dt = case
+    w = WORKLOADS["pkm"].scaled(name=name, T=T, H=H, d_half=dh, n_sub=n, k=k, d_v=dv, dtype=dt,
+                                seed=sum(map(ord, name)))
+    run_forward(w)
+
+
+def test_forward_tiny_workload_and_bruteforce():
+    """The tiny fp32 workload end to end; the selection also equals the
+    brute-force top-k over all 1024 full keys."""
+    import oracle
+
+    w = WORKLOADS["tiny"]
+    r = run_forward(w)
+    bidx, _ = oracle.bruteforce_select(r["inp"]["query"].cpu(), r["inp"]["subkeys"].cpu(), w.k)
+    assert r["ref"]["exempt"] == 0
+    np.testing.assert_array_equal(r["idx"], bidx)
+
+
+def test_forward_memplus_small():
+    w = WORKLOADS["memplus"].scaled(T=200, H=2, d_half=64, n_sub=64, k=8, d_v=256, d_model=128)
+    run_forward(w)
+
+
+def test_forward_empty_batch():
+    w = WORKLOADS["pkm"].scaled(T=0, H=2, d_half=64, n_sub=16, k=4, d_v=64)
+    inp = make_inputs(w, "cuda")
+    out, idx, wts = skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k)
+    assert out.shape == (0, 64)
+
+
+def test_forward_deterministic():
+    w = WORKLOADS["pkm"].scaled(T=257, H=2, d_half=64, n_sub=128, k=32, d_v=256)
+    inp = make_inputs(w, "cuda")
+    a = skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k)
+    b = skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+# ------------------------------------------------------------ bag gather --
+
+BAGS = [(1, 1, 8, "bf16"), (513, 128, 2048, "bf16"), (77, 33, 1024, "bf16"),
+        (50, 7, 24, "f32"), (31, 128, 4096, "bf16"), (200, 5, 8, "f32")]
+
+
+@pytest.mark.parametrize("n_bags,B,d,dt", BAGS)
+@pytest.mark.parametrize("gate", [False, True])
+def test_embbag_forward(n_bags, B, d, dt, gate):
+    import oracle
+
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    n_rows = 1000
+    g = torch.Generator().manual_seed(n_bags * 7 + B)
+    table = (torch.randn(n_rows, d, generator=g) * 0.02).to(tdt).cuda()
+    idx, w = random_bags(n_bags, B, n_rows, seed=B + d)
+    gt = torch.randn(n_bags, d, generator=g).to(tdt).cuda() if gate else None
+    out = skv.embbag_forward(table, idx.cuda(), w.cuda(), gate=gt)
+    ref = oracle.bag(idx.numpy(), w.double().numpy(), table.cpu())
+    if gate:
+        ref = ref * gt.double().cpu().numpy()
+    close(out.double().cpu().numpy(), ref, RTOL[dt], "embbag")
+
+
+def test_embbag_bad_index_sets_status():
+    table = torch.randn(10, 16, dtype=torch.bfloat16, device="cuda")
+    idx = torch.tensor([[0, 1, 10], [2, -1, 3]], dtype=torch.int32, device="cuda")
+    w = torch.full((2, 3), 0.5, device="cuda")
+    out = skv.embbag_forward(table, idx, w)
+    assert skv.device_error() == 4  # PKM_ERR_DEVICE
+    assert skv.device_error() == 0  # cleared on read
+    ref = 0.5 * (table[0].float() + table[1].float())
+    torch.testing.assert_close(out[0].float(), ref, rtol=2e-2, atol=1e-2)
+
+
+# ------------------------------------------------- full-size workloads --
+
+def _sample(T, m, seed):
+    g = torch.Generator().manual_seed(seed)
+    s = torch.randperm(T, generator=g)[: m - 2]
+    return torch.cat([torch.tensor([0, T - 1]), s]).sort().values
+
+
+def test_forward_pkm_full_size_sampled():
+    w = WORKLOADS["pkm"]
+    run_forward(w, sample=_sample(w.T, 64, 1))
+
+
+def test_forward_memplus_full_size_sampled():
+    w = WORKLOADS["memplus"]
+    r = run_forward(w, sample=_sample(w.T, 32, 2))
+    del r
+    torch.cuda.empty_cache()
+
+
+def test_decode_steps():
+    """Decode-shaped lookups (8 tokens per step) against the 16.8M-key tables."""
+    from sparse_key_value_b200.inputs import decode_step_inputs
+
+    w = WORKLOADS["decode"]
+    base = make_inputs(w.scaled(T=8), "cuda")
+    for step in (0, 1, 255):
+        inp = dict(base)
+        inp.update(decode_step_inputs(w, step, "cuda"))
+        run_forward(w, inp=inp)
+    del base
+    torch.cuda.empty_cache()
