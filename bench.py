@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the product-key memory lookup forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload pkm]
+                    [--impl ours|reference]
+
+One step = one pkm_forward over a batch of the workload (norms, sub-key
+scoring + per-half top-k, k x k combine + softmax, bag gather [+ Memory+
+GEMMs]).  For N > 1 the script runs under torch.distributed.run, one rank
+per GPU: every rank holds a replica of the tables and processes its own
+batch (weak scaling, no data-path collective); the timing is the maximum
+over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (plain fp64 C, all host cores) on a
+bounded token sample per step, rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "memory-layer lookup tokens/sec; bag-gather HBM GB/s vs B200 ~8 TB/s peak"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="pkm",
+                   choices=["pkm", "memplus", "tiny", "decode"])
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="target CPU time of the oracle baseline sample")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------ plumbing --
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return rank, world, local  # rank 0 alone works; no process group
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+class Clocks:
+    """nvidia-smi samples (200 ms) of this GPU during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"pkm_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.remove(self.path)
+        loaded = [s for s in sm if smax and s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def measured_peaks():
+    for p in (os.path.join(ROOT, "MEASURED_PEAKS.json"),):
+        if os.path.exists(p):
+            d = json.load(open(p))
+            return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def gather_bytes_per_token(w) -> int:
+    """Algorithmic bytes of the bag gather per token: every selected value row
+    (H*k rows of d_v elements), its row id and weight (8 B), the output row
+    and, with Memory+, the gate row read."""
+    b = w.elem_bytes
+    per = w.H * w.k * (w.d_v * b + 8) + w.d_v * b
+    if w.memplus:
+        per += w.d_v * b
+    return per
+
+
+def traffic_record(workload: str):
+    """dram bytes per gather launch from the committed ncu summary, or None
+    when the gather kernel's source changed since it was captured."""
+    path = os.path.join(PROFILES, "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(workload)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "sparse_key_value_b200", "csrc", rec["source"])
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["dram_bytes_per_launch"] if sha == rec["source_sha"] else None
+
+
+# ------------------------------------------------------------ our arm --
+
+def run_ours(args, rank, world, local):
+    import sparse_key_value_b200 as skv
+    from sparse_key_value_b200.inputs import WORKLOADS, make_inputs
+
+    skv.load()
+    w = WORKLOADS[args.workload]
+    if args.workload == "decode":
+        w = w.scaled(T=8)
+    # each rank: its own token batch, a replica of the tables
+    wr = w.scaled(seed=w.seed + 7919 * rank, table_seed_=w.table_seed)
+    inp = make_inputs(wr, "cuda")
+    mp = w.memplus
+    kw = dict(x=inp["x"], W1=inp["W1"], W2=inp["W2"]) if mp else {}
+    T = w.T
+    out = torch.empty(T, w.d_out, dtype=w.torch_dtype, device="cuda")
+    idx = torch.empty(T, w.H, w.k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(T, w.H, w.k, dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(16, skv.forward_workspace_size(
+        T, w.H, w.d_half, w.n_sub, w.k, w.d_v, 1 if w.dtype == "bf16" else 0, mp, w.d_model)),
+        dtype=torch.uint8, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    lib = skv.load()
+
+    def step(events=None):
+        skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k, out=out, idx=idx,
+                        weights=wts, workspace=ws, phase_events=events, **kw)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert skv.device_error() == 0
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
+    for e in sum(ev, []):
+        e.record()  # creates the event handles the library records into
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = lib.pkm_launch_count()
+    with Clocks(local) as clk:
+        for i in range(K):
+            flush.zero_()  # L2 flush between timed steps (outside the events)
+            step(ev[i])
+        torch.cuda.synchronize()
+    launches = lib.pkm_launch_count() - launches0
+    barrier(world)
+    step_ms = [e[0].elapsed_time(e[6]) for e in ev]
+    phase_ms = [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(6)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    assert skv.device_error() == 0
+    ms_per_step = total_ms / K
+    value = world * T / (ms_per_step / 1e3)
+
+    # roofline of the dominant kernel: the bag gather (phase 4 -> 5)
+    gather_ms = statistics.mean(phase_ms[4])
+    bytes_per_launch = gather_bytes_per_token(w) * T
+    achieved = bytes_per_launch / (gather_ms / 1e3) / 1e9
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    traffic = traffic_record(args.workload)
+    roof = {"kernel": "embbag_fwd_kernel (bag gather)", "bound": "hbm",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_bytes_per_launch": bytes_per_launch,
+            "traffic": traffic, "gather_us": round(gather_ms * 1e3, 2)}
+    phases = dict(zip(["norms", "score_topk", "combine_softmax", "gate_gemm", "gather",
+                       "out_gemm"], [round(statistics.mean(p) * 1e3, 2) for p in phase_ms]))
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world)
+
+    clocks = clk.summary()
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded generators; no dataset)",
+        "config": dict(w.describe(), l2="256 MiB L2 flush write before every timed step",
+                       parallelism=f"replicas x{world}: one token batch per GPU, tables "
+                                   f"replicated, no data-path collective"),
+        "roofline": roof, "phases_us": phases,
+        "gather_GBps": round(achieved, 1), "clocks": clocks,
+        "gpu_launches": int(launches), "e2e": e2e,
+    }
+    return res, w, inp
+
+
+def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world):
+    """Same metric through the public API with host buffers: every step
+    copies the step's query (and x) from pinned host memory, runs the
+    forward and copies the output back."""
+    import sparse_key_value_b200 as skv
+
+    hq = inp["query"].cpu().pin_memory()
+    hx = inp["x"].cpu().pin_memory() if w.memplus else None
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq = torch.empty_like(inp["query"])
+    dx = torch.empty_like(inp["x"]) if w.memplus else None
+    kw2 = dict(kw)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        if dx is not None:
+            dx.copy_(hx, non_blocking=True)
+            kw2["x"] = dx
+        skv.pkm_forward(dq, inp["subkeys"], inp["values"], w.k, out=out, idx=idx, weights=wts,
+                        workspace=ws, **kw2)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    tot = 0.0
+    barrier(world)
+    for _ in range(K):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    tot = max_over_ranks(tot, world)
+    ms = tot / K
+    h2d = hq.numel() * hq.element_size() + (hx.numel() * hx.element_size() if hx is not None else 0)
+    d2h = hout.numel() * hout.element_size()
+    return {"value": round(world * w.T / (ms / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4)}
+
+
+# --------------------------------------------------------- oracle timing --
+
+def oracle_tokens_per_s(w, inp, tokens, values_dev):
+    """Run the CPU oracle (selection, bag, Memory+) on ``tokens``; returns
+    (seconds of oracle work, threads).  Value rows are fetched from the
+    device table between the oracle's steps (not timed)."""
+    import numpy as np
+
+    import oracle
+
+    q = inp["query"][tokens].cpu()
+    K = inp["subkeys"].cpu()
+    t0 = time.perf_counter()
+    idx, S, wt, _ = oracle.pkm_select(q, K, w.k)
+    t_sel = time.perf_counter() - t0
+    rows = np.unique(idx)
+    dev = values_dev.device
+    table = values_dev[torch.from_numpy(rows).to(dev)].cpu()
+    pos = np.searchsorted(rows, idx).reshape(len(tokens), -1)
+    t0 = time.perf_counter()
+    y = oracle.bag(pos, wt.reshape(len(tokens), -1), table)
+    if w.memplus:
+        oracle.memplus(y, inp["x"][tokens].cpu(), inp["W1"].cpu(), inp["W2"].cpu())
+    t_rest = time.perf_counter() - t0
+    return t_sel + t_rest, oracle.num_threads()
+
+
+def cpu_baseline(args, w, inp):
+    """The oracle as it stands, on a bounded token sample (about
+    --cpu-seconds of CPU work)."""
+    import oracle
+
+    oracle.build()
+    T = w.T
+    m, secs = 4, 0.0
+    while True:
+        tokens = torch.arange(m) * (T // m)
+        secs, cores = oracle_tokens_per_s(w, inp, tokens, inp["values"])
+        if secs >= args.cpu_seconds / 4 or m >= T:
+            break
+        m = min(T, m * max(2, int(args.cpu_seconds / 4 / max(secs, 1e-3))))
+    return {"value": round(m / secs, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{m} of {T} tokens (evenly spaced) of the {w.name} workload; "
+                      f"fp64 selection + bag{' + Memory+' if w.memplus else ''}; "
+                      f"{secs:.2f} s"}
+
+
+# ---------------------------------------------------------- reference arm --
+
+def run_reference(args, rank, world):
+    """The oracle on the host cores as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    from sparse_key_value_b200.inputs import WORKLOADS, make_inputs
+
+    oracle.build()
+    w = WORKLOADS[args.workload]
+    if args.workload == "decode":
+        w = w.scaled(T=8)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(w, dev)
+    per_step = 8 if w.T >= 8 else w.T
+    spacing = max(1, w.T // (per_step * max(1, args.steps + args.warmup)))
+    times, cores = [], 1
+    for i in range(args.warmup + args.steps):
+        tokens = (torch.arange(per_step) * spacing * (args.steps + args.warmup) + i * spacing) % w.T
+        s, cores = oracle_tokens_per_s(w, inp, tokens, inp["values"])
+        if i >= args.warmup:
+            times.append(s)
+    sec = sum(times) / len(times)
+    value = per_step / sec
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generators; no dataset)",
+        "config": dict(w.describe(), parallelism="host cores of rank 0"),
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{per_step} tokens per step of the {w.name} workload"},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            res, w, inp = run_ours(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(args, w, inp)
+            else:
+                res["cpu_baseline"] = None
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

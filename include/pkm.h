@@ -103,7 +103,16 @@ typedef struct {
     float *weights;
     void *workspace; /* device scratch of pkm_forward_workspace_size bytes */
     size_t workspace_bytes;
+    /* Optional instrumentation: NULL, or PKM_FWD_N_EVENTS cudaEvent_t
+       handles (host array) recorded on `stream` at the phase boundaries:
+       [0] start, [1] after the norms, [2] after scoring + per-half top-k,
+       [3] after combine + softmax, [4] after the gate GEMM, [5] after the
+       bag gather, [6] after the output GEMM ([4] and [6] repeat the
+       previous boundary without Memory+). */
+    void **phase_events;
 } pkm_fwd_args;
+
+#define PKM_FWD_N_EVENTS 7
 
 /* Bytes of device workspace pkm_forward needs for these sizes (pointers
    are not read). */
@@ -193,6 +202,10 @@ PKM_API const char *pkm_status_string(pkm_status status);
 
 /* Library version: major*10000 + minor*100 + patch. */
 PKM_API int32_t pkm_version(void);
+
+/* Instrumentation: number of kernels this process has launched through the
+   library so far (host-side counter, all devices). */
+PKM_API uint64_t pkm_launch_count(void);
 
 #ifdef __cplusplus
 }

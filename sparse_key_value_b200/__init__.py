@@ -66,11 +66,13 @@ def forward_workspace_size(T, H, d_half, n_sub, k, d_v, dtype=PKM_BF16, memplus=
 
 
 def pkm_forward(query, subkeys, values, k: int, x=None, W1=None, W2=None, out=None, idx=None,
-                weights=None, workspace=None, stream=None):
+                weights=None, workspace=None, stream=None, phase_events=None):
     """Forward of one memory layer (see pkm_forward in include/pkm.h).
 
     query [T,H,2,d_half], subkeys [H,2,n_sub,d_half], values [n_sub^2, d_v];
     optional Memory+ gate x [T,d_model], W1 [d_model,d_v], W2 [d_v,d_model].
+    ``phase_events``: optional list of 7 torch.cuda.Event recorded at the
+    phase boundaries (see pkm_fwd_args.phase_events).
     Returns (out, idx, weights)."""
     _need_cuda(query, subkeys, values, x, W1, W2)
     T, H, two, dh = query.shape
@@ -93,6 +95,11 @@ def pkm_forward(query, subkeys, values, k: int, x=None, W1=None, W2=None, out=No
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     a.workspace, a.workspace_bytes = _p(workspace), workspace.numel()
+    if phase_events is not None:
+        if len(phase_events) != 7 or any(e.cuda_event == 0 for e in phase_events):
+            raise ValueError("phase_events: 7 events, each recorded once before use")
+        arr = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
+        a.phase_events = ctypes.cast(arr, ctypes.c_void_p)
     check(lib.pkm_forward(ctypes.byref(a), _stream(dev, stream)), "pkm_forward")
     return out, idx, weights
 

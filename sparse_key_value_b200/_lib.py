@@ -32,7 +32,11 @@ class FwdArgs(ctypes.Structure):
     _fields_ = [("T", I64), ("H", I32), ("d_half", I32), ("n_sub", I32), ("k", I32),
                 ("d_v", I32), ("dtype", ctypes.c_int), ("query", P), ("subkeys", P),
                 ("values", P), ("x", P), ("W1", P), ("W2", P), ("d_model", I32), ("out", P),
-                ("idx", P), ("weights", P), ("workspace", P), ("workspace_bytes", SZ)]
+                ("idx", P), ("weights", P), ("workspace", P), ("workspace_bytes", SZ),
+                ("phase_events", P)]
+
+
+FWD_N_EVENTS = 7
 
 
 class BwdArgs(ctypes.Structure):
@@ -46,7 +50,8 @@ class BwdArgs(ctypes.Structure):
 
 EXPORTS = ("pkm_forward_workspace_size", "pkm_forward", "pkm_backward_workspace_size",
            "pkm_backward", "embbag_forward", "embbag_backward_workspace_size",
-           "embbag_backward", "pkm_get_device_error", "pkm_status_string", "pkm_version")
+           "embbag_backward", "pkm_get_device_error", "pkm_status_string", "pkm_version",
+           "pkm_launch_count")
 
 _lib = None
 
@@ -81,6 +86,8 @@ def load(path: str = LIB_PATH):
     lib.pkm_status_string.restype = ctypes.c_char_p
     lib.pkm_version.argtypes = []
     lib.pkm_version.restype = I32
+    lib.pkm_launch_count.argtypes = []
+    lib.pkm_launch_count.restype = ctypes.c_uint64
     if path == LIB_PATH:
         _lib = lib
     return lib

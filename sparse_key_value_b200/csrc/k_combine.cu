@@ -129,6 +129,7 @@ cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64
   if (TH <= 0) return cudaSuccess;
   dim3 grid((unsigned)((TH + kCombWarps - 1) / kCombWarps));
   combine_kernel<<<grid, kCombWarps * 32, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -116,6 +116,7 @@ static cudaError_t launch_embbag_t(const void* table, int64_t n_rows, int d, con
   dim3 grid((unsigned)((n_bags + bags_per_cta - 1) / bags_per_cta));
   fn<<<grid, kBagThreads, smem, stream>>>((const T*)table, n_rows, d, idx, w, n_bags, B,
                                           (const T*)gate, (T*)out, bags_per_cta, status);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -32,6 +32,7 @@ cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst
   dim3 grid((cols + 31) / 32, (rows + 31) / 32), block(32, 8);
   transpose_bf16_kernel<<<grid, block, 0, stream>>>((const __nv_bfloat16*)src, rows, cols,
                                                     (__nv_bfloat16*)dst);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -91,6 +92,7 @@ cudaError_t launch_gemm_simt(const void* A, const void* B, int64_t M, int N, int
   dim3 grid((N + 63) / 64, (unsigned)((M + 63) / 64));
   gemm_simt_kernel<<<grid, 256, 0, stream>>>((const __nv_bfloat16*)A, (const __nv_bfloat16*)B,
                                              M, N, K, epi, (__nv_bfloat16*)C);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -47,6 +47,7 @@ cudaError_t launch_row_rnorm(const void* x, pkm_dtype dt, int64_t rows, int d, f
         (const __nv_bfloat16*)x, rows, d, r);
   else
     row_rnorm_kernel<PKM_F32><<<grid, warps * 32, 0, stream>>>((const float*)x, rows, d, r);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -148,12 +149,14 @@ cudaError_t launch_score_topk_simt(const void* q, const void* K, pkm_dtype dt, i
     if (e != cudaSuccess) return e;
     fn<<<grid, 256, smem, stream>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)K, T, H, dh,
                                     n, k, rq, rk, hv, hi);
+    note_launch();
   } else {
     auto fn = score_topk_simt_kernel<PKM_F32>;
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     fn<<<grid, 256, smem, stream>>>((const float*)q, (const float*)K, T, H, dh, n, k, rq, rk,
                                     hv, hi);
+    note_launch();
   }
   return cudaGetLastError();
 }

@@ -1,21 +1,408 @@
-// k_score_tc.cu -- sub-key scoring on the tensor cores (tcgen05): placeholder
-// until the kernel lands; the SIMT path serves every shape meanwhile.
+// k_score_tc.cu -- sub-key scoring on the tensor cores with the per-half
+// top-k fused into the epilogue.
+//
+// "모델 안의 메모리", "작동 방식": each half of the query is compared with all
+// of its ~sqrt(N) half-keys and the best are kept; "Memory Layers at Scale"
+// digest, "Product-key 검색": 2*sqrt(N) comparisons per lookup.  For one
+// (head h, half c) the comparisons of 128 tokens against 256 half-keys form
+// the GEMM tile D[128 x 256] = Q_c[128 x d_half] * K_c[256 x d_half]^T.
+//
+// Per CTA: 128 tokens x one (h, c) x a range of 256-column chunks.
+//   warp 0     TMA producer: per chunk and 64-wide k-block, the query tile
+//              [128 x 64] and the sub-key tile [256 x 64] (bf16, 128-byte
+//              swizzle) into a 4-stage ring.
+//   warp 1     TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128,
+//              N=256, K=16, fp32 accumulators in two TMEM buffers of 256
+//              columns (the MMAs of chunk i+1 overlap the epilogue of chunk i).
+//   warps 2-5  epilogue, one thread per token row (TMEM lane): reads its
+//              row's 256 scores with tcgen05.ld, scales them,
+//                s = (acc * rk[a]) * (sqrt(d_half) * rq),
+//              and keeps a running top-k: scores above the current k-th
+//              best go to a per-thread buffer in shared memory; when any
+//              thread's buffer nears full the warp sorts each buffer with a
+//              bitonic network in registers and merges it into the sorted
+//              register list (a 64-bit key: order-preserving score bits,
+//              then the complemented column, so ties favour the smaller id).
+// The raw bf16 inputs feed the MMA (products exact in fp32); the
+// normalisation is applied in fp32 in the epilogue.
+//
+// Every spin-wait is bounded: on a timeout the CTA records PKM_ERR_TIMEOUT,
+// stops issuing work, waits (bounded) for its copies and MMAs in flight,
+// frees its TMEM and exits.
+#include <math.h>
+
+#include "common.cuh"
 #include "kernels.h"
+#include "tmap.h"
 
 namespace pkm {
 
-bool score_tc_supported(pkm_dtype, int, int, int) { return false; }
-int score_tc_splits(int64_t, int, int) { return 1; }
-cudaError_t launch_score_topk_tc(const void*, const void*, int64_t, int, int, int, int, int,
-                                 const float*, const float*, float*, int32_t*, int32_t*,
-                                 cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace sc {
+constexpr int kM = 128;           // tokens per tile (TMEM lanes)
+constexpr int kN = 256;           // sub-key columns per chunk
+constexpr int kKB = 64;           // k-block width (128 bytes of bf16)
+constexpr int kStages = 4;
+constexpr int kABytes = kM * kKB * 2;   // 16 KiB
+constexpr int kBBytes = kN * kKB * 2;   // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kBuf = 16;          // pending candidates per row
+constexpr int kFlushAt = kBuf - 8;
+constexpr int kThreads = 192;
+constexpr int kMaxK = 32;
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + (size_t)kStages * kStageBytes +
+                              (size_t)kBuf * kM * 8 /*buffers*/ + 256 /*barriers*/;
+}  // namespace sc
+
+struct ScoreSmemCtl {
+  uint64_t full[sc::kStages];
+  uint64_t empty[sc::kStages];
+  uint64_t accf[2];
+  uint64_t acce[2];
+  uint64_t drain;
+  uint32_t tmem;
+  volatile int abort;
+};
+
+// bounded wait that also gives up when another role of the CTA aborted
+__device__ __forceinline__ bool wait_ctl(uint64_t* bar, uint32_t parity, ScoreSmemCtl* ctl,
+                                         int32_t* status) {
+  for (unsigned long long i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 255 && ctl->abort) return false;
+  }
+  ctl->abort = 1;
+  set_status(status, PKM_ERR_TIMEOUT);
+  return false;
 }
 
-bool gemm_tc_supported(int64_t, int, int) { return false; }
-cudaError_t launch_gemm_tc(const void*, const void*, int64_t, int, int, int, void*, int32_t*,
-                           cudaStream_t) {
-  return cudaErrorNotSupported;
+__device__ __forceinline__ uint32_t ord_f32(float s) {
+  uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unord_f32(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+__device__ __forceinline__ uint64_t pack_key(float s, int32_t id) {
+  return ((uint64_t)ord_f32(s) << 32) | (uint64_t)(0xffffffffu - (uint32_t)id);
+}
+
+#define CAS_DESC(a, b)                 \
+  {                                    \
+    uint64_t x_ = (a), y_ = (b);       \
+    (a) = x_ > y_ ? x_ : y_;           \
+    (b) = x_ > y_ ? y_ : x_;           \
+  }
+
+// sort 32 keys descending (bitonic network, fully unrolled)
+__device__ __forceinline__ void sort32_desc(uint64_t* v) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          if ((i & size) == 0) {
+            CAS_DESC(v[i], v[j]);
+          } else {
+            CAS_DESC(v[j], v[i]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// sort 16 keys descending
+__device__ __forceinline__ void sort16_desc(uint64_t* v) {
+#pragma unroll
+  for (int size = 2; size <= 16; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          if ((i & size) == 0) {
+            CAS_DESC(v[i], v[j]);
+          } else {
+            CAS_DESC(v[j], v[i]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// L (sorted desc, 32) <- top 32 of L u B (B sorted desc, 16)
+__device__ __forceinline__ void merge16_desc(uint64_t* L, const uint64_t* B) {
+#pragma unroll
+  for (int i = 16; i < 32; ++i) L[i] = L[i] > B[31 - i] ? L[i] : B[31 - i];
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & stride) == 0) CAS_DESC(L[i], L[i + stride]);
+    }
+  }
+}
+
+// L (sorted desc) <- top 32 of L u B (B sorted desc)
+__device__ __forceinline__ void merge32_desc(uint64_t* L, const uint64_t* B) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) L[i] = L[i] > B[31 - i] ? L[i] : B[31 - i];
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & stride) == 0) CAS_DESC(L[i], L[i + stride]);
+    }
+  }
+}
+
+// Merge the thread's pending candidates (bv/bi, cnt of them, stride kM)
+// into its sorted list L and refresh the threshold (score of entry k-1).
+__device__ __forceinline__ void flush_pending(uint64_t (&L)[32], const float* bv,
+                                              const int32_t* bi, int& cnt, float& thr, int k) {
+  uint64_t B[sc::kBuf];
+#pragma unroll
+  for (int j = 0; j < sc::kBuf; ++j)
+    B[j] = j < cnt ? pack_key(bv[j * sc::kM], bi[j * sc::kM]) : 0ull;
+  sort16_desc(B);
+  merge16_desc(L, B);
+  cnt = 0;
+  uint64_t kth = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (i == k - 1) kth = L[i];
+  thr = kth ? unord_f32((uint32_t)(kth >> 32)) : -INFINITY;
+}
+
+__global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t T,
+    int H, int dh, int n, int k, int chunks_per_split, const float* __restrict__ rq,
+    const float* __restrict__ rk, float* __restrict__ hv, int32_t* __restrict__ hi,
+    int32_t* status) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* stages = base;
+  float* bufv = reinterpret_cast<float*>(base + sc::kStages * sc::kStageBytes);
+  int32_t* bufi = reinterpret_cast<int32_t*>(bufv + sc::kBuf * sc::kM);
+  ScoreSmemCtl* ctl = reinterpret_cast<ScoreSmemCtl*>(bufi + sc::kBuf * sc::kM);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hc = blockIdx.y;
+  const int64_t m0 = (int64_t)blockIdx.x * sc::kM;
+  const int n_chunks = (n + sc::kN - 1) / sc::kN;
+  const int c_begin = blockIdx.z * chunks_per_split;
+  const int c_end = min(n_chunks, c_begin + chunks_per_split);
+  const int KB = dh / sc::kKB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < sc::kStages; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->accf[b], 1);
+      mbar_init(&ctl->acce[b], 4);
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_par = 0;
+      bool ok = true;
+      for (int c = c_begin; c < c_end && ok; ++c) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!wait_ctl(&ctl->empty[stage], phase ^ 1, ctl, status)) { ok = false; break; }
+          unsigned char* sa = stages + stage * sc::kStageBytes;
+          mbar_arrive_expect_tx(&ctl->full[stage], sc::kStageBytes);
+          tma_load_3d(sa, &tmA, &ctl->full[stage], kb * sc::kKB, hc, (int32_t)m0);
+          tma_load_3d(sa + sc::kABytes, &tmB, &ctl->full[stage], kb * sc::kKB, c * sc::kN, hc);
+          issued_mask |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == sc::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {  // let every copy in flight land before the CTA exits
+        for (int s = 0; s < sc::kStages; ++s)
+          if (issued_mask & (1u << s)) {
+            for (unsigned long long i = 0; i < kSpinLimit; ++i)
+              if (mbar_try_wait(&ctl->full[s], (issued_par >> s) & 1)) break;
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(sc::kM, sc::kN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int c = c_begin; c < c_end && ok; ++c, ++it) {
+        const int buf = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1) & 1;
+        if (!wait_ctl(&ctl->acce[buf], use ^ 1, ctl, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + buf * sc::kN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!wait_ctl(&ctl->full[stage], phase, ctl, status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stages + stage * sc::kStageBytes);
+          const uint32_t sb = sa + sc::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < sc::kKB / 16; ++kk) {
+            tc_mma_f16(d_tmem, smem_desc_k128(sa + kk * 32), smem_desc_k128(sb + kk * 32), idesc,
+                       (kb | kk) != 0);
+          }
+          tc_commit(&ctl->empty[stage]);  // the stage is free once these MMAs finish
+          if (++stage == sc::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (ok) tc_commit(&ctl->accf[buf]);
+      }
+      // every MMA issued must complete before TMEM is released
+      tc_commit(&ctl->drain);
+      for (unsigned long long i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(&ctl->drain, 0)) break;
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may read
+    const int row = quarter * 32 + lane;
+    const int64_t t = m0 + row;
+    const float rowf = t < T ? sqrtf((float)dh) * rq[t * H * 2 + hc] : 0.f;
+    const float* rkc = rk + (int64_t)hc * n;
+    float* bv = bufv + row;
+    int32_t* bi = bufi + row;
+    uint64_t L[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) L[i] = 0;
+    float thr = -INFINITY;
+    float rkg = 0.f;
+    int cnt = 0;
+
+    int it = 0;
+    bool ok = true;
+    for (int c = c_begin; c < c_end; ++c, ++it) {
+      const int buf = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1) & 1;
+      const bool got = wait_ctl(&ctl->accf[buf], use, ctl, status);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      for (int g = 0; g < sc::kN / 8; ++g) {
+        const int col0 = c * sc::kN + g * 8;
+        if (col0 >= n) break;
+        uint32_t r[8];
+        tmem_ld_32x32b_x8(tmem + ((uint32_t)(quarter * 32) << 16) + buf * sc::kN + g * 8, r);
+        if ((g & 3) == 0) rkg = col0 + lane < n ? rkc[col0 + lane] : 0.f;
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float rkj = __shfl_sync(0xffffffffu, rkg, (g & 3) * 8 + j);
+          const float s = __uint_as_float(r[j]) * rkj * rowf;
+          if (col0 + j < n && s > thr) {
+            bv[cnt * sc::kM] = s;
+            bi[cnt * sc::kM] = col0 + j;
+            ++cnt;
+          }
+        }
+        if (__any_sync(0xffffffffu, cnt > sc::kFlushAt)) flush_pending(L, bv, bi, cnt, thr, k);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->acce[buf]);
+    }
+    if (ok) {
+      if (__any_sync(0xffffffffu, cnt > 0)) flush_pending(L, bv, bi, cnt, thr, k);
+      if (t < T) {
+        const int64_t orow = ((int64_t)blockIdx.z * T + t) * H * 2 + hc;
+        float* ov = hv + orow * k;
+        int32_t* oi = hi + orow * k;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (i < k) {
+            const uint64_t key = L[i];
+            ov[i] = key ? unord_f32((uint32_t)(key >> 32)) : -INFINITY;
+            oi[i] = key ? (int32_t)(0xffffffffu - (uint32_t)key) : 0x7fffffff;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+bool score_tc_supported(pkm_dtype dt, int dh, int n, int k) {
+  return dt == PKM_BF16 && dh % sc::kKB == 0 && dh <= 2048 && n >= sc::kN && k <= sc::kMaxK;
+}
+
+int score_tc_splits(int64_t T, int H, int n) {
+  const int64_t tiles = (T + sc::kM - 1) / sc::kM * H * 2;
+  const int chunks = (n + sc::kN - 1) / sc::kN;
+  int splits = 1;
+  // split the sub-key columns when the grid would not fill the 148 SMs
+  while (splits < 32 && splits * 2 <= chunks && tiles * splits < 148) splits *= 2;
+  // every split gets the same number of chunks
+  const int per = (chunks + splits - 1) / splits;
+  return (chunks + per - 1) / per;
+}
+
+cudaError_t launch_score_topk_tc(const void* q, const void* K, int64_t T, int H, int dh, int n,
+                                 int k, int splits, const float* rq, const float* rk, float* hv,
+                                 int32_t* hi, int32_t* status, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  CUtensorMap tmA, tmB;
+  {
+    const uint64_t dims[3] = {(uint64_t)dh, (uint64_t)H * 2, (uint64_t)T};
+    const uint64_t strides[2] = {(uint64_t)dh * 2, (uint64_t)H * 2 * dh * 2};
+    const uint32_t box[3] = {(uint32_t)sc::kKB, 1, (uint32_t)sc::kM};
+    if (!make_tmap_bf16(&tmA, q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)dh, (uint64_t)n, (uint64_t)H * 2};
+    const uint64_t strides[2] = {(uint64_t)dh * 2, (uint64_t)n * dh * 2};
+    const uint32_t box[3] = {(uint32_t)sc::kKB, (uint32_t)sc::kN, 1};
+    if (!make_tmap_bf16(&tmB, K, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  const int chunks = (n + sc::kN - 1) / sc::kN;
+  const int per = (chunks + splits - 1) / splits;
+  cudaError_t e = cudaFuncSetAttribute(score_topk_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sc::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((T + sc::kM - 1) / sc::kM), (unsigned)(H * 2), (unsigned)splits);
+  score_topk_tc_kernel<<<grid, sc::kThreads, sc::kSmemBytes, stream>>>(
+      tmA, tmB, T, H, dh, n, k, per, rq, rk, hv, hi, status);
+  note_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace pkm

@@ -9,6 +9,9 @@
 
 namespace pkm {
 
+// Host-side count of kernels this library has launched (instrumentation).
+void note_launch(int n = 1);
+
 // r[i] = 1 / max(||x[i, :]||_2, 1e-12) for rows of d elements.
 cudaError_t launch_row_rnorm(const void* x, pkm_dtype dt, int64_t rows, int d, float* r,
                              cudaStream_t stream);

@@ -1,5 +1,6 @@
 // pkm_capi.cu -- the C ABI of libpkm.so: argument validation, workspace
 // carving and the launch sequence of each entry point (see include/pkm.h).
+#include <atomic>
 #include <mutex>
 #include <stdio.h>
 
@@ -9,6 +10,9 @@
 namespace pkm {
 
 __device__ int32_t g_status = 0;  // sticky per-device status word
+
+static std::atomic<unsigned long long> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
 static std::mutex g_status_mu;
 static int32_t* g_status_ptr[64] = {nullptr};
@@ -98,6 +102,11 @@ static pkm_status validate_fwd(const pkm_fwd_args* a) {
     if (e_ != cudaSuccess) return PKM_ERR_CUDA; \
   } while (0)
 
+static void mark(const pkm_fwd_args* a, int i, cudaStream_t st) {
+  if (a->phase_events && a->phase_events[i])
+    cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), st);
+}
+
 static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   int32_t* status = status_ptr();
   if (!status) return PKM_ERR_CUDA;
@@ -111,8 +120,10 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   const int H = a->H, dh = a->d_half, n = a->n_sub, k = a->k;
 
   // a1: qk-normalisation factors
+  mark(a, 0, st);
   PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
   PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
+  mark(a, 1, st);
   // a2 + a3: sub-key scores and per-half top-k
   if (L.tc)
     PKM_TRY(launch_score_topk_tc(a->query, a->subkeys, T, H, dh, n, k, L.splits, rq, rk, hv, hi,
@@ -120,13 +131,18 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   else
     PKM_TRY(launch_score_topk_simt(a->query, a->subkeys, a->dtype, T, H, dh, n, k, rq, rk, hv,
                                    hi, st));
+  mark(a, 2, st);
   // a4 + a5: k x k combine, top-k, softmax
   PKM_TRY(launch_combine(hv, hi, L.splits, T, H, n, k, a->idx, a->weights, st));
+  mark(a, 3, st);
   // a6 (+ a7): bag gather over the H*k selected rows of each token
   const int64_t N = (int64_t)n * n;
   if (!has_memplus(a)) {
+    mark(a, 4, st);
     PKM_TRY(launch_embbag_fwd(a->values, N, a->d_v, a->dtype, a->idx, a->weights, T, H * k,
                               nullptr, a->out, status, st));
+    mark(a, 5, st);
+    mark(a, 6, st);
     return PKM_OK;
   }
   void* w1t = ws + L.w1t;
@@ -137,9 +153,12 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   PKM_TRY(launch_transpose_bf16(a->W1, dm, dv, w1t, st));  // [dv, dm]
   PKM_TRY(launch_transpose_bf16(a->W2, dv, dm, w2t, st));  // [dm, dv]
   PKM_TRY(launch_gemm_bf16(a->x, w1t, T, dv, dm, /*silu*/ 1, g, status, st));
+  mark(a, 4, st);
   PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g, z,
                             status, st));
+  mark(a, 5, st);
   PKM_TRY(launch_gemm_bf16(z, w2t, T, dm, dv, /*none*/ 0, a->out, status, st));
+  mark(a, 6, st);
   return PKM_OK;
 }
 
@@ -205,5 +224,7 @@ const char* pkm_status_string(pkm_status s) {
 }
 
 int32_t pkm_version(void) { return 100; }
+
+uint64_t pkm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

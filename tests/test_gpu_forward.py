@@ -60,6 +60,9 @@ SMALL = [
     ("bf16-k32-odd-n", 129, 3, 128, 100, 32, 64, "bf16"),
     ("bf16-minimal", 1, 1, 8, 3, 1, 8, "bf16"),
     ("bf16-wide", 37, 4, 512, 300, 32, 2048, "bf16"),
+    ("tc-two-chunks", 300, 2, 128, 512, 16, 64, "bf16"),
+    ("tc-k32-many-tiles", 1000, 1, 64, 1024, 32, 128, "bf16"),
+    ("tc-k1", 130, 2, 64, 256, 1, 16, "bf16"),
     ("f32-k64", 70, 2, 32, 64, 64, 40, "f32"),
     ("f32-k-equals-n", 33, 1, 16, 5, 5, 24, "f32"),
 ]
