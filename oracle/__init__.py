@@ -68,10 +68,11 @@ def _load():
         lib.orc_memplus.argtypes = [I64, I, I, P, P, I, P, I, P, I, P]
         lib.orc_pkm_backward.argtypes = [I64, I, I, I, I, I, P, I, P, I, P, I, I64,
                                          P, P, P, P, I, P, P, P, P, P]
+        lib.orc_value_grad_rows.argtypes = [I64, I, I, I, P, P, P, I, P, I64, P]
         lib.orc_num_threads.argtypes = []
         for f in ("orc_half_scores", "orc_topk", "orc_pkm_select",
                   "orc_bruteforce_select", "orc_softmax", "orc_bag", "orc_memplus",
-                  "orc_pkm_backward", "orc_num_threads"):
+                  "orc_pkm_backward", "orc_num_threads", "orc_value_grad_rows"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -239,3 +240,18 @@ def full_scores(s_half, ids, n: int):
     a, b = ids // n, ids % n
     return (np.take_along_axis(s_half[:, :, 0], a, -1)
             + np.take_along_axis(s_half[:, :, 1], b, -1))
+
+
+def value_grad_rows(idx, w, dy, rows):
+    """dV[r] = sum over slots with idx == r of w * dy[t], for the row ids
+    ``rows`` only; idx/w [T,H,k], dy [T, d_v]."""
+    idx = np.ascontiguousarray(idx, dtype=np.int64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    da, dt = _input(dy)
+    T, H, k = idx.shape
+    dv = da.shape[1]
+    out = np.empty((rows.shape[0], dv))
+    _check(_load().orc_value_grad_rows(T, H, k, dv, _p(idx), _p(w), _p(da), dt, _p(rows),
+                                       rows.shape[0], _p(out)), "value_grad_rows")
+    return out

@@ -510,3 +510,25 @@ int orc_num_threads(void) {
     return 1;
 #endif
 }
+
+/*
+ * Value-table gradient of selected rows only: for each requested row id
+ * rows[u], out[u] = sum over (t,h,j) with idx[t,h,j] == rows[u] of
+ * w[t,h,j] * dy[t], accumulated in (t, h, j) order.
+ */
+int orc_value_grad_rows(int64_t T, int H, int k, int dv, const int64_t *idx, const double *w,
+                        const void *dy, int dy_dtype, const int64_t *rows, int64_t n_rows,
+                        double *out) {
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t u = 0; u < n_rows; u++) {
+        double *o = out + u * dv;
+        for (int i = 0; i < dv; i++) o[i] = 0.0;
+        for (int64_t s = 0; s < T * H * k; s++) {
+            if (idx[s] != rows[u]) continue;
+            int64_t t = s / ((int64_t)H * k);
+            for (int i = 0; i < dv; i++) o[i] += w[s] * ld(dy, dy_dtype, t * dv + i);
+        }
+    }
+    return err;
+}

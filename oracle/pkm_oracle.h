@@ -61,6 +61,11 @@ int orc_pkm_backward(int64_t T, int H, int dh, int n, int k, int dv,
                      const void *dy, int dy_dtype, double *dw_out, double *dS_out,
                      double *dq_out, double *dK_out, double *dv_out);
 
+/* dV rows for the requested row ids only: out [n_rows, dv] */
+int orc_value_grad_rows(int64_t T, int H, int k, int dv, const int64_t *idx, const double *w,
+                        const void *dy, int dy_dtype, const int64_t *rows, int64_t n_rows,
+                        double *out);
+
 int orc_num_threads(void);
 
 #ifdef __cplusplus

@@ -6,48 +6,119 @@
 // and its value row is a * n_sub + b.  The weights are a softmax over the k
 // kept scores ("작동 방식": a weighted average of the values read).
 //
-// One warp per (token, head).  Both candidate sets are walks over sorted
-// queues: queue i yields its entries best first, and the warp repeatedly
-// takes the best queue head (a k-way merge), so no k^2 buffer is formed.
+// One warp per (token, head).  With both half lists sorted best first, cell
+// (i, j) of the k x k grid is beaten by every cell (i', j') with i' <= i and
+// j' <= j, so only the cells with (i+1)(j+1) <= k can be among the k best
+// (119 cells for k = 32; all cells when k <= 3).  The warp packs those cells
+// as 64-bit keys (order-preserving score bits, then the complemented row
+// id, so equal scores favour the smaller id), sorts them with a bitonic
+// network spread over its lanes, and keeps the first k.  When the per-half
+// lists come in several column splits, the warp first merges each half's
+// splits the same way.
 #include <math.h>
 
+#include "common.cuh"
 #include "kernels.h"
-#include "warp_topk.cuh"
 
 namespace pkm {
 
-// warp-wide best of (s, id) pairs; returns the winning lane
-__device__ __forceinline__ int warp_best(float& s, int32_t& id) {
-  const int lane = threadIdx.x & 31;
-  int who = lane;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-    int32_t i2 = __shfl_xor_sync(0xffffffffu, id, o);
-    int w2 = __shfl_xor_sync(0xffffffffu, who, o);
-    if (better(s2, i2, s, id)) {
-      s = s2;
-      id = i2;
-      who = w2;
-    }
-  }
-  return who;
-}
+namespace {
 
 constexpr int kCombWarps = 8;
+constexpr int kMaxSlots = 16;  // keys per lane: up to 512 candidates per warp
 
-// lists: smem per warp: l1v/l1i (half 1), l2v/l2i (half 2), k entries each
+__device__ __forceinline__ uint32_t ordf(float s) {
+  uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unordf(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+__device__ __forceinline__ uint64_t key_of(float s, int32_t id) {
+  return ((uint64_t)ordf(s) << 32) | (uint64_t)(0xffffffffu - (uint32_t)id);
+}
+
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int m) {
+  uint32_t lo = (uint32_t)v, hi = (uint32_t)(v >> 32);
+  lo = __shfl_xor_sync(0xffffffffu, lo, m);
+  hi = __shfl_xor_sync(0xffffffffu, hi, m);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Bitonic sort, descending, of the 32*S keys held as v[s] on lane l at
+// position p = s * 32 + l.  S is a power of two <= kMaxSlots.
+template <int S>
+__device__ __forceinline__ void warp_sort_desc(uint64_t (&v)[S]) {
+  const int lane = threadIdx.x & 31;
+  constexpr int NT = 32 * S;
+#pragma unroll
+  for (int size = 2; size <= NT; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 32) {  // partner in another slot of the same lane
+        const int ds = stride >> 5;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+          if ((s & ds) == 0) {
+            const int p = s * 32 + lane;
+            const bool desc = (p & size) == 0;
+            uint64_t a = v[s], b = v[s + ds];
+            const bool sw = desc ? (a < b) : (a > b);
+            v[s] = sw ? b : a;
+            v[s + ds] = sw ? a : b;
+          }
+        }
+      } else {  // partner on lane ^ stride
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+          const int p = s * 32 + lane;
+          const bool desc = (p & size) == 0;
+          const bool lower = (lane & stride) == 0;
+          const uint64_t o = shfl_xor64(v[s], stride);
+          // the lower position keeps the larger key in a descending block
+          const bool keep_max = (lower == desc);
+          const uint64_t mx = v[s] > o ? v[s] : o, mn = v[s] > o ? o : v[s];
+          v[s] = keep_max ? mx : mn;
+        }
+      }
+    }
+  }
+}
+
+// number of candidate cells (i, j), i, j < k, with (i+1)(j+1) <= k
+__host__ __device__ __forceinline__ int pruned_cells(int k) {
+  int c = 0;
+  for (int i = 1; i <= k; ++i) c += k / i;
+  return c;
+}
+
+template <int S>
 __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(
     const float* __restrict__ hv, const int32_t* __restrict__ hi, int splits, int64_t T, int H,
     int n, int k, int32_t* __restrict__ idx, float* __restrict__ wout) {
   __shared__ float lv[kCombWarps][2][64];
   __shared__ int32_t li[kCombWarps][2][64];
+  __shared__ uint8_t cell_i[32 * kMaxSlots];
+  __shared__ uint8_t cell_j[32 * kMaxSlots];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t th = (int64_t)blockIdx.x * kCombWarps + warp;  // t * H + h
-  if (th >= T * H) return;
   const int64_t TH2 = T * H * 2;
 
-  // 1. per half: the k best over the split lists (a walk over `splits` queues)
+  // candidate cells (i, j) with (i+1)(j+1) <= k, row-major, shared by the CTA
+  const int ncells = pruned_cells(k);
+  for (int p = threadIdx.x; p < ncells; p += blockDim.x) {
+    int i = 0, acc = 0;
+    while (acc + k / (i + 1) <= p) {
+      acc += k / (i + 1);
+      ++i;
+    }
+    cell_i[p] = (uint8_t)i;
+    cell_j[p] = (uint8_t)(p - acc);
+  }
+  __syncthreads();
+  if (th >= T * H) return;
+
+  // 1. each half's k best, merging the column splits when there are several
   for (int c = 0; c < 2; ++c) {
     const int64_t row = th * 2 + c;
     if (splits == 1) {
@@ -56,79 +127,83 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(
         li[warp][c][j] = hi[row * k + j];
       }
     } else {
-      int p = 0;  // this lane's position in its split list (lane < splits)
-      for (int r = 0; r < k; ++r) {
-        float s = -INFINITY;
-        int32_t id = 0x7fffffff;
-        if (lane < splits && p < k) {
-          const int64_t off = ((int64_t)lane * TH2 + row) * k + p;
-          s = hv[off];
-          id = hi[off];
+      uint64_t v[S];
+#pragma unroll
+      for (int s = 0; s < S; ++s) {
+        const int p = s * 32 + lane;
+        const int sp = p / k, j = p - sp * k;
+        v[s] = 0;
+        if (sp < splits) {
+          const int64_t off = ((int64_t)sp * TH2 + row) * k + j;
+          const int32_t iv = hi[off];
+          if (iv != 0x7fffffff) v[s] = key_of(hv[off], iv);
         }
-        int who = warp_best(s, id);
-        if (lane == 0) {
-          lv[warp][c][r] = s;
-          li[warp][c][r] = id;
+      }
+      warp_sort_desc<S>(v);
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int p = s * 32 + lane;
+        if (p < k) {
+          lv[warp][c][p] = unordf((uint32_t)(v[s] >> 32));
+          li[warp][c][p] = (int32_t)(0xffffffffu - (uint32_t)v[s]);
         }
-        if (lane == who) ++p;
       }
     }
   }
   __syncwarp();
 
-  // 2. k x k combine: queue i (lane i and lane i + 32) walks b over half 2
-  float s1a = -INFINITY, s1b = -INFINITY;
-  int32_t a1a = 0, a1b = 0;
-  if (lane < k) { s1a = lv[warp][0][lane]; a1a = li[warp][0][lane]; }
-  if (lane + 32 < k) { s1b = lv[warp][0][lane + 32]; a1b = li[warp][0][lane + 32]; }
-  int pa = 0, pb = 0;
-  float outS0 = 0.f, outS1 = 0.f;
-  int32_t outI0 = 0, outI1 = 0;
-  for (int r = 0; r < k; ++r) {
-    float sa = -INFINITY, sb = -INFINITY;
-    int32_t ia = 0x7fffffff, ib = 0x7fffffff;
-    if (lane < k && pa < k) {
-      sa = s1a + lv[warp][1][pa];
-      ia = a1a * n + li[warp][1][pa];
-    }
-    if (lane + 32 < k && pb < k) {
-      sb = s1b + lv[warp][1][pb];
-      ib = a1b * n + li[warp][1][pb];
-    }
-    const bool takeb = better(sb, ib, sa, ia);
-    float s = takeb ? sb : sa;
-    int32_t id = takeb ? ib : ia;
-    int who = warp_best(s, id);
-    if (lane == who) {
-      if (takeb) ++pb; else ++pa;
-    }
-    if (lane == (r & 31)) {
-      if (r < 32) { outS0 = s; outI0 = id; } else { outS1 = s; outI1 = id; }
+  // 2. pack the candidate cells and sort them
+  uint64_t v[S];
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int p = s * 32 + lane;
+    v[s] = 0;
+    if (p < ncells) {
+      const int i = cell_i[p], j = cell_j[p];
+      const float Sc = lv[warp][0][i] + lv[warp][1][j];
+      const int32_t id = li[warp][0][i] * n + li[warp][1][j];
+      v[s] = key_of(Sc, id);
     }
   }
+  warp_sort_desc<S>(v);
 
   // 3. softmax over the k kept scores (entry 0 is the maximum)
-  const float m = __shfl_sync(0xffffffffu, outS0, 0);
-  float e0 = lane < k ? expf(outS0 - m) : 0.f;
-  float e1 = lane + 32 < k ? expf(outS1 - m) : 0.f;
+  const float S0 = unordf((uint32_t)(v[0] >> 32));  // lane's entry `lane`
+  const float S1 = unordf((uint32_t)(v[1] >> 32));  // entry `lane + 32`
+  const float m = __shfl_sync(0xffffffffu, S0, 0);
+  const float e0 = lane < k ? expf(S0 - m) : 0.f;
+  const float e1 = lane + 32 < k ? expf(S1 - m) : 0.f;
   const float z = warp_sum(e0 + e1);
   const float inv = 1.0f / z;
   if (lane < k) {
-    idx[th * k + lane] = outI0;
+    idx[th * k + lane] = (int32_t)(0xffffffffu - (uint32_t)v[0]);
     wout[th * k + lane] = e0 * inv;
   }
   if (lane + 32 < k) {
-    idx[th * k + lane + 32] = outI1;
+    idx[th * k + lane + 32] = (int32_t)(0xffffffffu - (uint32_t)v[1]);
     wout[th * k + lane + 32] = e1 * inv;
   }
 }
+
+}  // namespace
 
 cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64_t T, int H,
                            int n, int k, int32_t* idx, float* w, cudaStream_t stream) {
   const int64_t TH = T * H;
   if (TH <= 0) return cudaSuccess;
+  const int need = max(pruned_cells(k), splits > 1 ? splits * k : 0);
   dim3 grid((unsigned)((TH + kCombWarps - 1) / kCombWarps));
-  combine_kernel<<<grid, kCombWarps * 32, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
+  const int threads = kCombWarps * 32;
+  if (need <= 64)
+    combine_kernel<2><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
+  else if (need <= 128)
+    combine_kernel<4><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
+  else if (need <= 256)
+    combine_kernel<8><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
+  else if (need <= 512)
+    combine_kernel<16><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
+  else
+    return cudaErrorInvalidValue;
   note_launch();
   return cudaGetLastError();
 }

@@ -12,6 +12,9 @@ namespace pkm {
 // Host-side count of kernels this library has launched (instrumentation).
 void note_launch(int n = 1);
 
+// Device address of the current device's sticky status word.
+int32_t* status_ptr();
+
 // r[i] = 1 / max(||x[i, :]||_2, 1e-12) for rows of d elements.
 cudaError_t launch_row_rnorm(const void* x, pkm_dtype dt, int64_t rows, int d, float* r,
                              cudaStream_t stream);
@@ -59,6 +62,34 @@ cudaError_t launch_bag_dw(const void* dy, const void* table, int64_t n_rows, int
                           pkm_dtype dt, const int32_t* idx, const float* w, int64_t n_bags,
                           int B, int group, float* dw, float* dS, int32_t* status,
                           cudaStream_t stream);
+
+cudaError_t launch_iota(uint32_t* v, int64_t n, cudaStream_t stream);
+cudaError_t launch_sanitize_keys(const int32_t* idx, int64_t n, int64_t limit, uint32_t* keys,
+                                 int32_t* status, cudaStream_t stream);
+
+// dq of one (token, head) per warp: d_half must be a multiple of 32 x
+// (elements per 16 bytes), at most 2048.
+bool backward_dh_supported(pkm_dtype dt, int dh);
+cudaError_t launch_dq(const void* q, const void* K, pkm_dtype dt, const float* rq,
+                      const float* rk, const int32_t* idx, const float* dS, int64_t T, int H,
+                      int dh, int n, int k, float* dq, cudaStream_t stream);
+
+// Sub-key gradient entries (distinct positions per token, head and half).
+cudaError_t launch_dk_entries(const int32_t* idx, const float* dS, const float* rq, int64_t T,
+                              int H, int dh, int n, int k, uint32_t mark, uint32_t* keys,
+                              float* coef, cudaStream_t stream);
+cudaError_t launch_dk_jacobian(const void* K, pkm_dtype dt, const float* rk, int64_t rows, int dh,
+                               float* g, cudaStream_t stream);
+
+// Deterministic segmented sums over sorted (key, entry) pairs.
+size_t segsum_workspace(int64_t n, int d);
+cudaError_t launch_segsum(const uint32_t* skey, const uint32_t* sval, int64_t n, uint32_t mark,
+                          const float* coef, const void* src, pkm_dtype dt, int64_t div, int d,
+                          int32_t* uniq_rows, float* grad_rows, int64_t cap, int64_t* n_uniq,
+                          float* dense_add, float* dense_set, void* workspace, int32_t* status,
+                          cudaStream_t stream);
+cudaError_t launch_scan_exclusive(uint32_t* data, int64_t len, uint32_t* total, int64_t* total64,
+                                  cudaStream_t stream);
 
 // Stable LSD radix sort of (key, value) pairs, key < 2^key_bits.
 size_t radix_sort_workspace(int64_t n);

@@ -18,7 +18,7 @@ static std::mutex g_status_mu;
 static int32_t* g_status_ptr[64] = {nullptr};
 
 // Device address of this device's status word (looked up once per device).
-static int32_t* status_ptr() {
+int32_t* status_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(g_status_mu);

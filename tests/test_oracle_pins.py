@@ -336,3 +336,17 @@ def test_backward_compact_rows(orc):
     comp = orc.pkm_backward(q, K, V[uniq], idx, inv.reshape(idx.shape), w, dy)
     np.testing.assert_allclose(comp["dV"], full["dV"][uniq], rtol=1e-13)
     np.testing.assert_array_equal(comp["dq"], full["dq"])
+
+
+def test_value_grad_rows_matches_backward(orc):
+    """The row-sampled value gradient equals the (finite-difference pinned)
+    full backward's dV on the same rows."""
+    T, H, dh, n, k, dv = 6, 2, 4, 5, 3, 7
+    q, K = _problem(T, H, dh, n, 98)
+    V = _rand((n * n, dv), 99)
+    dy = _rand((T, dv), 100)
+    idx, _, w, _ = orc.pkm_select(q, K, k)
+    full = orc.pkm_backward(q, K, V, idx, idx, w, dy)
+    rows = np.array(sorted(set(idx.ravel().tolist()))[::2] + [n * n - 1])
+    got = orc.value_grad_rows(idx, w, dy, rows)
+    np.testing.assert_allclose(got, full["dV"][rows], rtol=1e-13, atol=1e-15)
