@@ -1,13 +1,218 @@
-// k_gemm_tc.cu -- tensor-core GEMM for the Memory+ block (placeholder: the
-// SIMT GEMM in k_gemm.cu serves every shape until this kernel lands).
+// k_gemm_tc.cu -- the dense GEMMs of the Memory+ block on the tensor cores
+// ("Memory Layers at Scale" digest, "Memory+ 블록": out = (y ⊙ silu(x W1)) W2).
+//
+//   C[M, N] = epi(A[M, K] * B[N, K]^T),  A, B bf16 K-major, C bf16 row-major,
+//   epi = silu (gate) or identity (output projection), fp32 accumulation.
+//
+// One CTA per 128 x 256 output tile:
+//   warp 0     TMA producer: 64-wide k-blocks of A [128 x 64] and B [256 x 64]
+//              (128-byte swizzle) into a 4-stage ring.
+//   warp 1     TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128, N=256.
+//   warps 2-5  epilogue: one thread per output row reads 32 accumulator
+//              columns at a time (tcgen05.ld), applies the epilogue, rounds to
+//              bf16 (nearest even) and stores 64 contiguous bytes.
+// Spin-waits are bounded; on a timeout the CTA records PKM_ERR_TIMEOUT,
+// drains what it issued, frees its TMEM and exits.
+#include <math.h>
+
+#include "common.cuh"
 #include "kernels.h"
+#include "tmap.h"
 
 namespace pkm {
 
-bool gemm_tc_supported(int64_t, int, int) { return false; }
-cudaError_t launch_gemm_tc(const void*, const void*, int64_t, int, int, int, void*, int32_t*,
-                           cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace gm {
+constexpr int kM = 128, kN = 256, kKB = 64, kStages = 4;
+constexpr int kABytes = kM * kKB * 2, kBBytes = kN * kKB * 2;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256;
+}  // namespace gm
+
+struct GemmCtl {
+  uint64_t full[gm::kStages];
+  uint64_t empty[gm::kStages];
+  uint64_t accf;
+  uint64_t drain;
+  uint32_t tmem;
+  volatile int abort;
+};
+
+__device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, GemmCtl* ctl,
+                                          int32_t* status) {
+  for (unsigned long long i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 255 && ctl->abort) return false;
+  }
+  ctl->abort = 1;
+  set_status(status, PKM_ERR_TIMEOUT);
+  return false;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t M,
+    int N, int K, __nv_bfloat16* __restrict__ C, int32_t* status) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* stages = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(stages + gm::kStages * gm::kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = (int64_t)blockIdx.x * gm::kM;
+  const int n0 = blockIdx.y * gm::kN;
+  const int KB = (K + gm::kKB - 1) / gm::kKB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < gm::kStages; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    mbar_init(&ctl->accf, 1);
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem, gm::kN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t issued_mask = 0, issued_par = 0;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int stage = kb % gm::kStages;
+        const uint32_t phase = (uint32_t)(kb / gm::kStages) & 1;
+        if (!gemm_wait(&ctl->empty[stage], phase ^ 1, ctl, status)) { ok = false; break; }
+        unsigned char* sa = stages + stage * gm::kStageBytes;
+        mbar_arrive_expect_tx(&ctl->full[stage], gm::kStageBytes);
+        tma_load_2d(sa, &tmA, &ctl->full[stage], kb * gm::kKB, (int32_t)m0);
+        tma_load_2d(sa + gm::kABytes, &tmB, &ctl->full[stage], kb * gm::kKB, n0);
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+      }
+      if (!ok) {
+        for (int s = 0; s < gm::kStages; ++s)
+          if (issued_mask & (1u << s))
+            for (unsigned long long i = 0; i < kSpinLimit; ++i)
+              if (mbar_try_wait(&ctl->full[s], (issued_par >> s) & 1)) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(gm::kM, gm::kN);
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int stage = kb % gm::kStages;
+        const uint32_t phase = (uint32_t)(kb / gm::kStages) & 1;
+        if (!gemm_wait(&ctl->full[stage], phase, ctl, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(stages + stage * gm::kStageBytes);
+        const uint32_t sb = sa + gm::kABytes;
+#pragma unroll
+        for (int kk = 0; kk < gm::kKB / 16; ++kk)
+          tc_mma_f16(tmem, smem_desc_k128(sa + kk * 32), smem_desc_k128(sb + kk * 32), idesc,
+                     (kb | kk) != 0);
+        tc_commit(&ctl->empty[stage]);
+      }
+      if (ok) tc_commit(&ctl->accf);
+      tc_commit(&ctl->drain);
+      for (unsigned long long i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(&ctl->drain, 0)) break;
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int64_t m = m0 + row;
+    const bool got = gemm_wait(&ctl->accf, 0, ctl, status);
+    if (__all_sync(0xffffffffu, got)) {
+      tc_fence_after();
+      for (int g = 0; g < gm::kN / 32; ++g) {
+        const int col0 = n0 + g * 32;
+        if (col0 >= N) break;
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + g * 32, r);
+        tmem_ld_wait();
+        if (m < M) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float a = __uint_as_float(r[2 * j]), b = __uint_as_float(r[2 * j + 1]);
+            if (EPI == 1) {
+              a = a / (1.0f + expf(-a));
+              b = b / (1.0f + expf(-b));
+            }
+            packed[j] = pack_bf16x2(a, b);
+          }
+          __nv_bfloat16* dst = C + m * N + col0;
+          if (col0 + 32 <= N) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              reinterpret_cast<uint4*>(dst)[j] =
+                  make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          } else {
+            for (int j = 0; j < 16 && col0 + 2 * j < N; ++j)
+              reinterpret_cast<uint32_t*>(dst)[j] = packed[j];  // N % 8 == 0
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, gm::kN);
+  }
+}
+
+bool gemm_tc_supported(int64_t M, int N, int K) {
+  return M >= 1 && N >= 16 && K >= gm::kKB && N % 8 == 0 && K % 8 == 0;
+}
+
+cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
+                           void* C, int32_t* status, cudaStream_t stream) {
+  if (M <= 0) return cudaSuccess;
+  CUtensorMap tmA, tmB;
+  {
+    const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
+    const uint64_t strides[1] = {(uint64_t)K * 2};
+    const uint32_t box[2] = {(uint32_t)gm::kKB, (uint32_t)gm::kM};
+    if (!make_tmap_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)K, (uint64_t)N};
+    const uint64_t strides[1] = {(uint64_t)K * 2};
+    const uint32_t box[2] = {(uint32_t)gm::kKB, (uint32_t)gm::kN};
+    if (!make_tmap_bf16(&tmB, B, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  dim3 grid((unsigned)((M + gm::kM - 1) / gm::kM), (unsigned)((N + gm::kN - 1) / gm::kN));
+  cudaError_t e;
+  if (epi == 1) {
+    e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)gm::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    gemm_tc_kernel<1><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(
+        tmA, tmB, M, N, K, (__nv_bfloat16*)C, status);
+  } else {
+    e = cudaFuncSetAttribute(gemm_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)gm::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    gemm_tc_kernel<0><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(
+        tmA, tmB, M, N, K, (__nv_bfloat16*)C, status);
+  }
+  note_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace pkm

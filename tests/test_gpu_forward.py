@@ -88,8 +88,19 @@ def test_forward_tiny_workload_and_bruteforce():
     np.testing.assert_array_equal(r["idx"], bidx)
 
 
-def test_forward_memplus_small():
-    w = WORKLOADS["memplus"].scaled(T=200, H=2, d_half=64, n_sub=64, k=8, d_v=256, d_model=128)
+MEMPLUS = [
+    # T, H, d_half, n_sub, k, d_v, d_model
+    (200, 2, 64, 64, 8, 256, 128),     # output projection N < tile
+    (300, 1, 128, 256, 16, 512, 320),  # ragged N, tensor-core scoring
+    (50, 2, 64, 16, 4, 80, 40),        # K below one k-block: SIMT GEMM
+]
+
+
+@pytest.mark.parametrize("shape", MEMPLUS)
+def test_forward_memplus_small(shape):
+    T, H, dh, n, k, dv, dm = shape
+    w = WORKLOADS["memplus"].scaled(T=T, H=H, d_half=dh, n_sub=n, k=k, d_v=dv, d_model=dm,
+                                    seed=T + dv)
     run_forward(w)
 
 

@@ -1,0 +1,68 @@
+"""Properties of the synthetic workloads (CPU, no GPU needed)."""
+
+import math
+
+import pytest
+import torch
+
+from sparse_key_value_b200.inputs import WORKLOADS, decode_step_inputs, make_inputs
+
+
+def _selected_rows(w):
+    """Rows the product-key lookup selects (fp32 torch on the CPU; a
+    statistic of the inputs, not a parity reference)."""
+    inp = make_inputs(w, "cpu", with_values=False)
+    q, K = inp["query"].float(), inp["subkeys"].float()
+    T, H = q.shape[:2]
+    n, k = K.shape[2], w.k
+    u = q / q.norm(dim=-1, keepdim=True)
+    kap = K / K.norm(dim=-1, keepdim=True)
+    out = []
+    for h in range(H):
+        v1, a1 = (u[:, h, 0] @ kap[h, 0].T).topk(k, dim=-1)
+        v2, a2 = (u[:, h, 1] @ kap[h, 1].T).topk(k, dim=-1)
+        top = (v1[:, :, None] + v2[:, None, :]).view(T, -1).topk(k, dim=-1).indices
+        out.append(torch.gather(a1, 1, top // k) * n + torch.gather(a2, 1, top % k))
+    return torch.cat(out).view(-1)
+
+
+def test_train_workload_follows_zipf_1_1():
+    torch.set_num_threads(max(1, torch.get_num_threads()))
+    w = WORKLOADS["train"]
+    ids = _selected_rows(w)
+    cnt = torch.bincount(ids, minlength=w.N).double()
+    c = torch.sort(cnt, descending=True).values[:10000].clamp_min(0.5)
+    r = torch.arange(1, 10001, dtype=torch.float64)
+    X = torch.stack([torch.ones_like(r), r.log()], 1)
+    slope = torch.linalg.lstsq(X, c.log().unsqueeze(1)).solution[1, 0].item()
+    assert -slope == pytest.approx(1.1, abs=0.05)
+    assert 5e4 < int((cnt > 0).sum()) < 5e5
+
+
+def test_workload_shapes():
+    assert WORKLOADS["pkm"].N == 1 << 20
+    assert WORKLOADS["memplus"].N == 1 << 24
+    assert WORKLOADS["pkm"].N * WORKLOADS["pkm"].d_v * 2 == 4 << 30
+    assert WORKLOADS["memplus"].N * WORKLOADS["memplus"].d_v * 2 == 32 << 30
+    t = WORKLOADS["tiny"]
+    assert (t.T, t.H, t.d_half, t.n_sub, t.k, t.d_v, t.dtype, t.seed) == \
+        (512, 1, 128, 32, 8, 256, "f32", 0)
+
+
+def test_decode_reuses_memplus_tables():
+    m, d = WORKLOADS["memplus"], WORKLOADS["decode"]
+    a = make_inputs(m.scaled(T=4), "cpu", with_values=False)
+    b = make_inputs(d.scaled(T=8), "cpu", with_values=False)
+    assert torch.equal(a["subkeys"], b["subkeys"])
+    assert torch.equal(a["W1"], b["W1"]) and torch.equal(a["W2"], b["W2"])
+    s0, s1 = decode_step_inputs(d, 0), decode_step_inputs(d, 1)
+    assert s0["query"].shape == (8, 4, 2, 512)
+    assert not torch.equal(s0["query"], s1["query"])
+
+
+def test_distributions():
+    w = WORKLOADS["pkm"].scaled(T=512, n_sub=64, d_v=64)
+    inp = make_inputs(w, "cpu")
+    assert abs(inp["query"].float().std().item() - 1.0) < 0.02
+    assert abs(inp["subkeys"].float().std().item() - 1 / math.sqrt(512)) < 0.002
+    assert abs(inp["values"].float().std().item() - 0.02) < 0.001
