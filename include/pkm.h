@@ -104,11 +104,11 @@ typedef struct {
     void *workspace; /* device scratch of pkm_forward_workspace_size bytes */
     size_t workspace_bytes;
     /* Optional instrumentation: NULL, or PKM_FWD_N_EVENTS cudaEvent_t
-       handles (host array) recorded on `stream` at the phase boundaries:
+       handles (host array) recorded at the phase boundaries:
        [0] start, [1] after the norms, [2] after scoring + per-half top-k,
-       [3] after combine + softmax, [4] after the gate GEMM, [5] after the
-       bag gather, [6] after the output GEMM ([4] and [6] repeat the
-       previous boundary without Memory+). */
+       [3] after combine + softmax, [4] before the bag gather (after the
+       Memory+ gate GEMM), [5] after the bag gather, [6] end (after the
+       Memory+ output GEMM). */
     void **phase_events;
 } pkm_fwd_args;
 

@@ -185,12 +185,113 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(
   }
 }
 
+// One thread per (token, head), used when each half has a single list.  The
+// k x k grid S[i][j] = s1[i] + s2[j] decreases along rows and columns, so its
+// cells can be taken best first with a max-heap frontier: start at (0, 0);
+// taking (i, j) admits (i, j+1) and, on the first column, (i+1, 0).  Lists
+// and heap live in shared memory as [slot][thread] (conflict-free).
+constexpr int kThreadCombine = 64;
+
+__global__ void __launch_bounds__(kThreadCombine) combine_thread_kernel(
+    const float* __restrict__ hv, const int32_t* __restrict__ hi, int64_t TH, int n, int k,
+    int32_t* __restrict__ idx, float* __restrict__ wout) {
+  extern __shared__ unsigned char sm[];
+  const int tid = threadIdx.x;
+  constexpr int B = kThreadCombine;
+  float* s1 = reinterpret_cast<float*>(sm);          // [k][B]
+  float* s2 = s1 + k * B;                            // [k][B]
+  int32_t* a1 = reinterpret_cast<int32_t*>(s2 + k * B);
+  int32_t* b2 = a1 + k * B;
+  uint64_t* hk = reinterpret_cast<uint64_t*>(b2 + k * B);  // heap keys [k+2][B]
+  uint16_t* hc = reinterpret_cast<uint16_t*>(hk + (k + 2) * B);  // heap cells
+  float* outS = reinterpret_cast<float*>(hc + (k + 2) * B);      // [k][B]
+  const int64_t th = (int64_t)blockIdx.x * B + tid;
+  if (th >= TH) return;
+  for (int j = 0; j < k; ++j) {
+    s1[j * B + tid] = hv[(th * 2) * k + j];
+    a1[j * B + tid] = hi[(th * 2) * k + j];
+    s2[j * B + tid] = hv[(th * 2 + 1) * k + j];
+    b2[j * B + tid] = hi[(th * 2 + 1) * k + j];
+  }
+  auto key_at = [&](int i, int j) {
+    return key_of(s1[i * B + tid] + s2[j * B + tid], a1[i * B + tid] * n + b2[j * B + tid]);
+  };
+  int size = 0;
+  auto push = [&](uint64_t key, int cell) {
+    int pos = ++size;
+    while (pos > 1) {
+      const int par = pos >> 1;
+      const uint64_t pk = hk[par * B + tid];
+      if (pk >= key) break;
+      hk[pos * B + tid] = pk;
+      hc[pos * B + tid] = hc[par * B + tid];
+      pos = par;
+    }
+    hk[pos * B + tid] = key;
+    hc[pos * B + tid] = (uint16_t)cell;
+  };
+  push(key_at(0, 0), 0);
+  for (int r = 0; r < k; ++r) {
+    const uint64_t top = hk[1 * B + tid];
+    const int cell = hc[1 * B + tid];
+    // pop
+    const uint64_t lk = hk[size * B + tid];
+    const uint16_t lc = hc[size * B + tid];
+    --size;
+    int pos = 1;
+    while (true) {
+      int ch = pos * 2;
+      if (ch > size) break;
+      uint64_t ck = hk[ch * B + tid];
+      if (ch < size) {
+        const uint64_t rk2 = hk[(ch + 1) * B + tid];
+        if (rk2 > ck) {
+          ck = rk2;
+          ++ch;
+        }
+      }
+      if (ck <= lk) break;
+      hk[pos * B + tid] = ck;
+      hc[pos * B + tid] = hc[ch * B + tid];
+      pos = ch;
+    }
+    if (size > 0 || pos > 1) {
+      hk[pos * B + tid] = lk;
+      hc[pos * B + tid] = lc;
+    }
+    // emit
+    idx[th * k + r] = (int32_t)(0xffffffffu - (uint32_t)top);
+    outS[r * B + tid] = unordf((uint32_t)(top >> 32));
+    const int i = cell >> 6, j = cell & 63;
+    if (j + 1 < k) push(key_at(i, j + 1), i * 64 + j + 1);
+    if (j == 0 && i + 1 < k) push(key_at(i + 1, 0), (i + 1) * 64);
+  }
+  // softmax over the k kept scores (entry 0 is the maximum)
+  const float m = outS[tid];
+  float z = 0.f;
+  for (int r = 0; r < k; ++r) z += expf(outS[r * B + tid] - m);
+  const float inv = 1.0f / z;
+  for (int r = 0; r < k; ++r) wout[th * k + r] = expf(outS[r * B + tid] - m) * inv;
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64_t T, int H,
                            int n, int k, int32_t* idx, float* w, cudaStream_t stream) {
   const int64_t TH = T * H;
   if (TH <= 0) return cudaSuccess;
+  if (splits == 1) {
+    const size_t smem = (size_t)kThreadCombine *
+                        ((size_t)k * 16 + (size_t)(k + 2) * 10 + (size_t)k * 4);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(combine_thread_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    combine_thread_kernel<<<(unsigned)((TH + kThreadCombine - 1) / kThreadCombine),
+                            kThreadCombine, smem, stream>>>(hv, hi, TH, n, k, idx, w);
+    note_launch();
+    return cudaGetLastError();
+  }
   const int need = max(pruned_cells(k), splits > 1 ? splits * k : 0);
   dim3 grid((unsigned)((TH + kCombWarps - 1) / kCombWarps));
   const int threads = kCombWarps * 32;

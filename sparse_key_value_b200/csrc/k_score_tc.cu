@@ -41,23 +41,24 @@ namespace sc {
 constexpr int kM = 128;           // tokens per tile (TMEM lanes)
 constexpr int kN = 256;           // sub-key columns per chunk
 constexpr int kKB = 64;           // k-block width (128 bytes of bf16)
-constexpr int kStages = 4;
+constexpr int kStages = 2;
 constexpr int kABytes = kM * kKB * 2;   // 16 KiB
 constexpr int kBBytes = kN * kKB * 2;   // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kBuf = 16;          // pending candidates per row
 constexpr int kFlushAt = kBuf - 8;
 constexpr int kThreads = 192;
+constexpr int kCtasPerSm = 2;     // two CTAs share an SM: their MMAs and epilogues interleave
 constexpr int kMaxK = 32;
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + (size_t)kStages * kStageBytes +
-                              (size_t)kBuf * kM * 8 /*buffers*/ + 256 /*barriers*/;
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + (size_t)kBuf * kM * 8 /*buffers*/ +
+                              128 /*barriers*/;
 }  // namespace sc
 
 struct ScoreSmemCtl {
   uint64_t full[sc::kStages];
   uint64_t empty[sc::kStages];
-  uint64_t accf[2];
-  uint64_t acce[2];
+  uint64_t accf;
+  uint64_t acce;
   uint64_t drain;
   uint32_t tmem;
   volatile int abort;
@@ -161,14 +162,16 @@ __device__ __forceinline__ void merge32_desc(uint64_t* L, const uint64_t* B) {
   }
 }
 
-// Merge the thread's pending candidates (bv/bi, cnt of them, stride kM)
-// into its sorted list L and refresh the threshold (score of entry k-1).
-__device__ __forceinline__ void flush_pending(uint64_t (&L)[32], const float* bv,
-                                              const int32_t* bi, int& cnt, float& thr, int k) {
+// Merge the thread's pending candidates (pairs (score, column) at stride kM,
+// cnt of them) into its sorted list L and refresh the filter threshold.
+__device__ __forceinline__ void flush_pending(uint64_t (&L)[32], const float2* pend, int& cnt,
+                                              float& thr_raw, int k, float rowf) {
   uint64_t B[sc::kBuf];
 #pragma unroll
-  for (int j = 0; j < sc::kBuf; ++j)
-    B[j] = j < cnt ? pack_key(bv[j * sc::kM], bi[j * sc::kM]) : 0ull;
+  for (int j = 0; j < sc::kBuf; ++j) {
+    const float2 e = pend[j * sc::kM];
+    B[j] = j < cnt ? pack_key(e.x, __float_as_int(e.y)) : 0ull;
+  }
   sort16_desc(B);
   merge16_desc(L, B);
   cnt = 0;
@@ -176,21 +179,28 @@ __device__ __forceinline__ void flush_pending(uint64_t (&L)[32], const float* bv
 #pragma unroll
   for (int i = 0; i < 32; ++i)
     if (i == k - 1) kth = L[i];
-  thr = kth ? unord_f32((uint32_t)(kth >> 32)) : -INFINITY;
+  // The filter compares the unscaled product acc * rk[a] against thr / rowf
+  // lowered by 2^-20 relative, so it keeps a superset of the exact
+  // candidates s = (acc * rk[a]) * rowf > thr; the exact key decides later.
+  if (kth != 0) {
+    const float thr = unord_f32((uint32_t)(kth >> 32));
+    const float r = thr / rowf;
+    const float t = r - fabsf(r) * 9.5367431640625e-7f;
+    if (fabsf(t) < INFINITY) thr_raw = fmaxf(thr_raw, t);  // overflow: keep the old one
+  }
 }
 
-__global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
+__global__ void __launch_bounds__(sc::kThreads, sc::kCtasPerSm) score_topk_tc_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t T,
     int H, int dh, int n, int k, int chunks_per_split, const float* __restrict__ rq,
     const float* __restrict__ rk, float* __restrict__ hv, int32_t* __restrict__ hi,
     int32_t* status) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* stages = base;
-  float* bufv = reinterpret_cast<float*>(base + sc::kStages * sc::kStageBytes);
-  int32_t* bufi = reinterpret_cast<int32_t*>(bufv + sc::kBuf * sc::kM);
-  ScoreSmemCtl* ctl = reinterpret_cast<ScoreSmemCtl*>(bufi + sc::kBuf * sc::kM);
+  // dynamic shared memory starts 1024-byte aligned (required by the 128-byte
+  // swizzle of the TMA tiles); checked below
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* stages = smem_raw;
+  float2* pend = reinterpret_cast<float2*>(smem_raw + sc::kStages * sc::kStageBytes);
+  ScoreSmemCtl* ctl = reinterpret_cast<ScoreSmemCtl*>(pend + sc::kBuf * sc::kM);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hc = blockIdx.y;
@@ -198,17 +208,21 @@ __global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
   const int n_chunks = (n + sc::kN - 1) / sc::kN;
   const int c_begin = blockIdx.z * chunks_per_split;
   const int c_end = min(n_chunks, c_begin + chunks_per_split);
+  const int nch = c_end - c_begin;
+  const int iters = nch;
   const int KB = dh / sc::kKB;
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // uniform: every thread leaves
+    if (threadIdx.x == 0) set_status(status, PKM_ERR_DEVICE);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < sc::kStages; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&ctl->accf[b], 1);
-      mbar_init(&ctl->acce[b], 4);
-    }
+    mbar_init(&ctl->accf, 1);
+    mbar_init(&ctl->acce, 4);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_barrier_init();
@@ -218,7 +232,7 @@ __global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem, 512);
+    tmem_alloc(&ctl->tmem, sc::kN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -233,7 +247,8 @@ __global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
-      for (int c = c_begin; c < c_end && ok; ++c) {
+      for (int it = 0; it < iters && ok; ++it) {
+        const int c = c_begin + it % nch;
         for (int kb = 0; kb < KB; ++kb) {
           if (!wait_ctl(&ctl->empty[stage], phase ^ 1, ctl, status)) { ok = false; break; }
           unsigned char* sa = stages + stage * sc::kStageBytes;
@@ -260,13 +275,11 @@ __global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int c = c_begin; c < c_end && ok; ++c, ++it) {
-        const int buf = it & 1;
-        const uint32_t use = (uint32_t)(it >> 1) & 1;
-        if (!wait_ctl(&ctl->acce[buf], use ^ 1, ctl, status)) { ok = false; break; }
+      uint32_t use = 0;
+      for (int it = 0; it < iters && ok; ++it, use ^= 1) {
+        // the accumulator is free once the epilogue has read the last chunk
+        if (!wait_ctl(&ctl->acce, use ^ 1, ctl, status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + buf * sc::kN;
         for (int kb = 0; kb < KB; ++kb) {
           if (!wait_ctl(&ctl->full[stage], phase, ctl, status)) { ok = false; break; }
           tc_fence_after();
@@ -274,13 +287,13 @@ __global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
           const uint32_t sb = sa + sc::kABytes;
 #pragma unroll
           for (int kk = 0; kk < sc::kKB / 16; ++kk) {
-            tc_mma_f16(d_tmem, smem_desc_k128(sa + kk * 32), smem_desc_k128(sb + kk * 32), idesc,
+            tc_mma_f16(tmem, smem_desc_k128(sa + kk * 32), smem_desc_k128(sb + kk * 32), idesc,
                        (kb | kk) != 0);
           }
           tc_commit(&ctl->empty[stage]);  // the stage is free once these MMAs finish
           if (++stage == sc::kStages) { stage = 0; phase ^= 1; }
         }
-        if (ok) tc_commit(&ctl->accf[buf]);
+        if (ok) tc_commit(&ctl->accf);
       }
       // every MMA issued must complete before TMEM is released
       tc_commit(&ctl->drain);
@@ -292,51 +305,65 @@ __global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
     const int quarter = warp & 3;  // TMEM lanes this warp may read
     const int row = quarter * 32 + lane;
     const int64_t t = m0 + row;
-    const float rowf = t < T ? sqrtf((float)dh) * rq[t * H * 2 + hc] : 0.f;
+    const bool live = t < T;
+    const float rowf = live ? sqrtf((float)dh) * rq[t * H * 2 + hc] : 0.f;
     const float* rkc = rk + (int64_t)hc * n;
-    float* bv = bufv + row;
-    int32_t* bi = bufi + row;
+    float2* pd = pend + row;
     uint64_t L[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) L[i] = 0;
-    float thr = -INFINITY;
+    // rows past the end of the batch (or with a zero query) keep nothing
+    float thr_raw = live && rowf > 0.f ? -INFINITY : INFINITY;
     float rkg = 0.f;
     int cnt = 0;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
 
-    int it = 0;
+    uint32_t use = 0;
     bool ok = true;
-    for (int c = c_begin; c < c_end; ++c, ++it) {
-      const int buf = it & 1;
-      const uint32_t use = (uint32_t)(it >> 1) & 1;
-      const bool got = wait_ctl(&ctl->accf[buf], use, ctl, status);
+    for (int it = 0; it < iters; ++it, use ^= 1) {
+      const int c = c_begin + it % nch;
+      const bool got = wait_ctl(&ctl->accf, use, ctl, status);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
+      const int c0 = c * sc::kN;
+      const int ncols = min(sc::kN, n - c0);
       for (int g = 0; g < sc::kN / 8; ++g) {
-        const int col0 = c * sc::kN + g * 8;
-        if (col0 >= n) break;
+        const int col0 = c0 + g * 8;
+        if (g * 8 >= ncols) break;
         uint32_t r[8];
-        tmem_ld_32x32b_x8(tmem + ((uint32_t)(quarter * 32) << 16) + buf * sc::kN + g * 8, r);
-        if ((g & 3) == 0) rkg = col0 + lane < n ? rkc[col0 + lane] : 0.f;
+        tmem_ld_32x32b_x8(tmem + lane_base + g * 8, r);
+        if ((g & 3) == 0) rkg = g * 8 + lane < ncols ? rkc[col0 + lane] : 0.f;
         tmem_ld_wait();
+        if (g * 8 + 8 <= ncols) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float rkj = __shfl_sync(0xffffffffu, rkg, (g & 3) * 8 + j);
-          const float s = __uint_as_float(r[j]) * rkj * rowf;
-          if (col0 + j < n && s > thr) {
-            bv[cnt * sc::kM] = s;
-            bi[cnt * sc::kM] = col0 + j;
-            ++cnt;
+          for (int j = 0; j < 8; ++j) {
+            const float rkj = __shfl_sync(0xffffffffu, rkg, (g & 3) * 8 + j);
+            const float p = __uint_as_float(r[j]) * rkj;
+            if (p > thr_raw) {
+              pd[cnt * sc::kM] = make_float2(p * rowf, __int_as_float(col0 + j));
+              ++cnt;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float rkj = __shfl_sync(0xffffffffu, rkg, (g & 3) * 8 + j);
+            const float p = __uint_as_float(r[j]) * rkj;
+            if (g * 8 + j < ncols && p > thr_raw) {
+              pd[cnt * sc::kM] = make_float2(p * rowf, __int_as_float(col0 + j));
+              ++cnt;
+            }
           }
         }
-        if (__any_sync(0xffffffffu, cnt > sc::kFlushAt)) flush_pending(L, bv, bi, cnt, thr, k);
+        if (__any_sync(0xffffffffu, cnt > sc::kFlushAt)) flush_pending(L, pd, cnt, thr_raw, k, rowf);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->acce[buf]);
+      if (lane == 0) mbar_arrive(&ctl->acce);
     }
     if (ok) {
-      if (__any_sync(0xffffffffu, cnt > 0)) flush_pending(L, bv, bi, cnt, thr, k);
-      if (t < T) {
+      if (__any_sync(0xffffffffu, cnt > 0)) flush_pending(L, pd, cnt, thr_raw, k, rowf);
+      if (live) {
         const int64_t orow = ((int64_t)blockIdx.z * T + t) * H * 2 + hc;
         float* ov = hv + orow * k;
         int32_t* oi = hi + orow * k;
@@ -356,7 +383,7 @@ __global__ void __launch_bounds__(sc::kThreads, 1) score_topk_tc_kernel(
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, sc::kN);
   }
 }
 

@@ -40,11 +40,12 @@ cudaError_t launch_score_topk_tc(const void* q, const void* K, int64_t T, int H,
 cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64_t T, int H,
                            int n, int k, int32_t* idx, float* w, cudaStream_t stream);
 
-// out[t] = sum_j w[t,j] * table[idx[t,j]] (⊙ gate[t])
+// out[t] = sum_j w[t,j] * table[idx[t,j]] (⊙ gate[t]); a persistent grid of
+// at most ctas_per_sm CTAs per SM (fewer leave room for concurrent kernels).
 cudaError_t launch_embbag_fwd(const void* table, int64_t n_rows, int d, pkm_dtype dt,
                               const int32_t* idx, const float* w, int64_t n_bags, int B,
-                              const void* gate, void* out, int32_t* status,
-                              cudaStream_t stream);
+                              const void* gate, void* out, int32_t* status, cudaStream_t stream,
+                              int ctas_per_sm = 8);
 
 // Memory+ helpers (bf16).
 cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,

@@ -118,12 +118,20 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   int32_t* hi = reinterpret_cast<int32_t*>(ws + L.hi);
   const int64_t T = a->T;
   const int H = a->H, dh = a->d_half, n = a->n_sub, k = a->k;
+  const int64_t N = (int64_t)n * n;
+  const bool mp = has_memplus(a);
+  const int dm = a->d_model, dv = a->d_v;
+  void* w1t = mp ? ws + L.w1t : nullptr;
+  void* w2t = mp ? ws + L.w2t : nullptr;
+  char* g = mp ? ws + L.g : nullptr;
+  char* z = mp ? ws + L.z : nullptr;
 
   // a1: qk-normalisation factors
   mark(a, 0, st);
   PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
   PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
   mark(a, 1, st);
+
   // a2 + a3: sub-key scores and per-half top-k
   if (L.tc)
     PKM_TRY(launch_score_topk_tc(a->query, a->subkeys, T, H, dh, n, k, L.splits, rq, rk, hv, hi,
@@ -135,29 +143,17 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   // a4 + a5: k x k combine, top-k, softmax
   PKM_TRY(launch_combine(hv, hi, L.splits, T, H, n, k, a->idx, a->weights, st));
   mark(a, 3, st);
-  // a6 (+ a7): bag gather over the H*k selected rows of each token
-  const int64_t N = (int64_t)n * n;
-  if (!has_memplus(a)) {
-    mark(a, 4, st);
-    PKM_TRY(launch_embbag_fwd(a->values, N, a->d_v, a->dtype, a->idx, a->weights, T, H * k,
-                              nullptr, a->out, status, st));
-    mark(a, 5, st);
-    mark(a, 6, st);
-    return PKM_OK;
+  // (a7) gate GEMM, a6 bag gather over the H*k selected rows of each token
+  if (mp) {
+    PKM_TRY(launch_transpose_bf16(a->W1, dm, dv, w1t, st));  // [dv, dm]
+    PKM_TRY(launch_transpose_bf16(a->W2, dv, dm, w2t, st));  // [dm, dv]
+    PKM_TRY(launch_gemm_bf16(a->x, w1t, T, dv, dm, /*silu*/ 1, g, status, st));
   }
-  void* w1t = ws + L.w1t;
-  void* w2t = ws + L.w2t;
-  void* g = ws + L.g;
-  void* z = ws + L.z;
-  const int dm = a->d_model, dv = a->d_v;
-  PKM_TRY(launch_transpose_bf16(a->W1, dm, dv, w1t, st));  // [dv, dm]
-  PKM_TRY(launch_transpose_bf16(a->W2, dv, dm, w2t, st));  // [dm, dv]
-  PKM_TRY(launch_gemm_bf16(a->x, w1t, T, dv, dm, /*silu*/ 1, g, status, st));
   mark(a, 4, st);
-  PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g, z,
-                            status, st));
+  PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g,
+                            mp ? z : a->out, status, st));
   mark(a, 5, st);
-  PKM_TRY(launch_gemm_bf16(z, w2t, T, dm, dv, /*none*/ 0, a->out, status, st));
+  if (mp) PKM_TRY(launch_gemm_bf16(z, w2t, T, dm, dv, /*none*/ 0, a->out, status, st));
   mark(a, 6, st);
   return PKM_OK;
 }
