@@ -114,6 +114,24 @@ typedef struct {
 
 #define PKM_FWD_N_EVENTS 7
 
+/*
+ * pkm_forward_noalloc: the same forward for callers that cannot allocate
+ * device memory (a C program linking only this library with no allocator,
+ * a runtime whose memory budget is fixed at start-up, a serving loop that
+ * must not call the synchronising cudaMalloc).  There is no counterpart on
+ * the source pages: it is a service of this library.
+ *
+ * Arguments as for pkm_forward; `workspace` and `workspace_bytes` are
+ * ignored.  The scratch is a fixed 32 MiB array inside the library on each
+ * device (held by every device that loads the library until exit); calls
+ * whose pkm_forward_workspace_size exceeds 32 MiB return PKM_ERR_WORKSPACE
+ * and launch nothing.  The first call on a device looks up the array's
+ * address on that device (make that first call before any stream capture).
+ * All calls share the array: calls whose GPU work overlaps race.  Nothing is
+ * allocated or freed.
+ */
+PKM_API pkm_status pkm_forward_noalloc(const pkm_fwd_args *args, pkm_stream_t stream);
+
 /* Bytes of device workspace pkm_forward needs for these sizes (pointers
    are not read). */
 PKM_API size_t pkm_forward_workspace_size(const pkm_fwd_args *args);

@@ -51,7 +51,7 @@ class BwdArgs(ctypes.Structure):
 EXPORTS = ("pkm_forward_workspace_size", "pkm_forward", "pkm_backward_workspace_size",
            "pkm_backward", "embbag_forward", "embbag_backward_workspace_size",
            "embbag_backward", "pkm_get_device_error", "pkm_status_string", "pkm_version",
-           "pkm_launch_count")
+           "pkm_launch_count", "pkm_forward_noalloc")
 
 _lib = None
 
@@ -86,6 +86,8 @@ def load(path: str = LIB_PATH):
     lib.pkm_status_string.restype = ctypes.c_char_p
     lib.pkm_version.argtypes = []
     lib.pkm_version.restype = I32
+    lib.pkm_forward_noalloc.argtypes = [FA, P]
+    lib.pkm_forward_noalloc.restype = ctypes.c_int
     lib.pkm_launch_count.argtypes = []
     lib.pkm_launch_count.restype = ctypes.c_uint64
     if path == LIB_PATH:

@@ -15,6 +15,11 @@ void note_launch(int n = 1);
 // Device address of the current device's sticky status word.
 int32_t* status_ptr();
 
+// pkm_forward with a library-chosen workspace, and the workspace size it needs.
+pkm_status forward_into(const pkm_fwd_args* a, void* workspace, size_t workspace_bytes,
+                        cudaStream_t st);
+size_t forward_workspace_bytes(const pkm_fwd_args* a);
+
 // r[i] = 1 / max(||x[i, :]||_2, 1e-12) for rows of d elements.
 cudaError_t launch_row_rnorm(const void* x, pkm_dtype dt, int64_t rows, int d, float* r,
                              cudaStream_t stream);

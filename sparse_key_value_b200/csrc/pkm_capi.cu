@@ -158,6 +158,21 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   return PKM_OK;
 }
 
+// The forward with a workspace chosen inside the library (the allocation-free
+// entry point in pkm_noalloc.cu passes its static scratch array here).
+pkm_status forward_into(const pkm_fwd_args* a, void* workspace, size_t workspace_bytes,
+                        cudaStream_t st) {
+  if (!a) return PKM_ERR_INVALID_ARG;
+  pkm_fwd_args b = *a;
+  b.workspace = workspace;
+  b.workspace_bytes = workspace_bytes;
+  pkm_status s = validate_fwd(&b);
+  if (s != PKM_OK || b.T == 0) return s;
+  return forward_impl(&b, st);
+}
+
+size_t forward_workspace_bytes(const pkm_fwd_args* a) { return a ? fwd_layout(a).total : 0; }
+
 }  // namespace pkm
 
 using namespace pkm;
