@@ -44,7 +44,9 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default="pkm",
-                   choices=["pkm", "memplus", "tiny", "decode"])
+                   choices=["pkm", "memplus", "tiny", "decode", "train"])
+    p.add_argument("--graph", action="store_true",
+                   help="capture one step in a CUDA graph and replay it (default for decode)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -159,6 +161,24 @@ def gather_bytes_per_token(w) -> int:
     return per
 
 
+def backward_bytes(w, U: int) -> int:
+    """Algorithmic bytes of the training backward: the value rows re-gathered
+    (R rows), ids and weights (8 B per slot), dy, q and K read, dq and dK
+    written (fp32), the sparse value gradient written (U rows of fp32 plus ids)."""
+    b = w.elem_bytes
+    R = w.T * w.H * w.k
+    return (R * (w.d_v * b + 8) + w.T * w.d_v * b + w.T * w.H * 2 * w.d_half * (b + 4)
+            + w.H * 2 * w.n_sub * w.d_half * (b + 4) + U * (w.d_v * 4 + 4))
+
+
+def graph_launches(lib, step) -> int:
+    """Kernels one step launches (counted on an eager run)."""
+    c0 = lib.pkm_launch_count()
+    step()
+    torch.cuda.synchronize()
+    return lib.pkm_launch_count() - c0
+
+
 def traffic_record(workload: str):
     """dram bytes per gather launch from the committed ncu summary, or None
     when the gather kernel's source changed since it was captured."""
@@ -199,80 +219,147 @@ def run_ours(args, rank, world, local):
     stream = torch.cuda.current_stream()
     lib = skv.load()
 
-    def step(events=None):
+    train = w.train
+    if train:
+        R = T * w.H * w.k
+        dq = torch.empty(T, w.H, 2, w.d_half, dtype=torch.float32, device="cuda")
+        dK = torch.empty(w.H, 2, w.n_sub, w.d_half, dtype=torch.float32, device="cuda")
+        uniq = torch.empty(R, dtype=torch.int32, device="cuda")
+        grad = torch.empty(R, w.d_v, dtype=torch.float32, device="cuda")
+        n_uniq = torch.zeros(1, dtype=torch.int64, device="cuda")
+        bargs = skv._bwd_args(inp["query"], inp["subkeys"], inp["values"], idx, wts, inp["dy"],
+                              dquery=skv._p(dq), dsubkeys=skv._p(dK), uniq_rows=skv._p(uniq),
+                              grad_rows=skv._p(grad), n_uniq=skv._p(n_uniq), uniq_cap=R)
+        bws = torch.empty(max(16, lib.pkm_backward_workspace_size(skv.ctypes.byref(bargs))),
+                          dtype=torch.uint8, device="cuda")
+        bargs.workspace, bargs.workspace_bytes = skv._p(bws), bws.numel()
+        sptr = skv.ctypes.c_void_p(stream.cuda_stream)
+
+    def step(events=None, bev=None):
         skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k, out=out, idx=idx,
                         weights=wts, workspace=ws, phase_events=events, **kw)
+        if train:
+            if bev is not None:
+                bev[0].record()
+            skv.check(lib.pkm_backward(skv.ctypes.byref(bargs), sptr), "pkm_backward")
+            if bev is not None:
+                bev[1].record()
 
+    use_graph = args.graph or args.workload == "decode"
+    flush_between = args.workload != "decode"
     for _ in range(args.warmup):
-        flush.zero_()
+        if flush_between:
+            flush.zero_()
         step()
     torch.cuda.synchronize()
     assert skv.device_error() == 0
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
-    for e in sum(ev, []):
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for e in sum(ev, []) + sum(bev, []):
         e.record()  # creates the event handles the library records into
     barrier(world)
     torch.cuda.synchronize()
     launches0 = lib.pkm_launch_count()
     with Clocks(local) as clk:
         for i in range(K):
-            flush.zero_()  # L2 flush between timed steps (outside the events)
-            step(ev[i])
+            if flush_between:
+                flush.zero_()  # L2 flush between timed steps (outside the events)
+            if graph is not None:
+                ev[i][0].record()
+                graph.replay()
+                ev[i][6].record()
+            else:
+                step(ev[i], bev[i] if train else None)
         torch.cuda.synchronize()
     launches = lib.pkm_launch_count() - launches0
+    if graph is not None:  # kernels replayed from the graph: one step's launches x K
+        launches = graph_launches(lib, step) * K
     barrier(world)
-    step_ms = [e[0].elapsed_time(e[6]) for e in ev]
-    phase_ms = [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(6)]
+    step_ms = [(e[0].elapsed_time(e[6]) if not train else e[0].elapsed_time(b[1]))
+               for e, b in zip(ev, bev)]
+    phase_ms = None if graph is not None else \
+        [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(6)]
     total_ms = max_over_ranks(sum(step_ms), world)
     assert skv.device_error() == 0
     ms_per_step = total_ms / K
     value = world * T / (ms_per_step / 1e3)
 
     # roofline of the dominant kernel: the bag gather (phase 4 -> 5)
-    gather_ms = statistics.mean(phase_ms[4])
-    bytes_per_launch = gather_bytes_per_token(w) * T
-    achieved = bytes_per_launch / (gather_ms / 1e3) / 1e9
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
+    bytes_per_launch = gather_bytes_per_token(w) * T
     traffic = traffic_record(args.workload)
-    roof = {"kernel": "embbag_fwd_kernel (bag gather)", "bound": "hbm",
-            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-            "algorithmic_bytes_per_launch": bytes_per_launch,
-            "traffic": traffic, "gather_us": round(gather_ms * 1e3, 2)}
-    phases = dict(zip(["norms", "score_topk", "combine_softmax", "gate_gemm", "gather",
-                       "out_gemm"], [round(statistics.mean(p) * 1e3, 2) for p in phase_ms]))
+    if phase_ms is not None:
+        gather_ms = statistics.mean(phase_ms[4])
+        achieved = bytes_per_launch / (gather_ms / 1e3) / 1e9
+        roof = {"kernel": "embbag_fwd_kernel (bag gather)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": bytes_per_launch,
+                "traffic": traffic, "gather_us": round(gather_ms * 1e3, 2)}
+        phases = dict(zip(["norms", "score_topk", "combine_softmax", "gate_gemm", "gather",
+                           "out_gemm"], [round(statistics.mean(p) * 1e3, 2) for p in phase_ms]))
+    else:  # graph replay: only whole steps are timed
+        achieved = bytes_per_launch / (ms_per_step / 1e3) / 1e9
+        roof = {"kernel": "whole step (graph replay)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": bytes_per_launch, "traffic": traffic}
+        phases = None
+    extra = {}
+    if train:
+        bwd_ms = statistics.mean([b[0].elapsed_time(b[1]) for b in bev])
+        U = int(n_uniq.item())
+        bbytes = backward_bytes(w, U)
+        extra["backward"] = {"us": round(bwd_ms * 1e3, 1), "distinct_rows": U,
+                             "algorithmic_bytes": bbytes,
+                             "GBps": round(bbytes / (bwd_ms / 1e3) / 1e9, 1),
+                             "frac": round(bbytes / (bwd_ms / 1e3) / 1e9 / peak, 4)}
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world)
+        e2e = run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world,
+                      backward=(lambda: skv.check(lib.pkm_backward(skv.ctypes.byref(bargs), sptr),
+                                                  "pkm_backward")) if train else None)
 
     clocks = clk.summary()
+    l2 = "256 MiB L2 flush write before every timed step" if flush_between else \
+        "decode steps back to back: the value table (32 GiB) exceeds L2, the sub-keys stay " \
+        "L2-resident as in a decode loop"
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded generators; no dataset)",
-        "config": dict(w.describe(), l2="256 MiB L2 flush write before every timed step",
+        "config": dict(w.describe(), l2=l2, graph=bool(graph is not None),
+                       step="forward + backward" if train else "forward",
                        parallelism=f"replicas x{world}: one token batch per GPU, tables "
                                    f"replicated, no data-path collective"),
         "roofline": roof, "phases_us": phases,
         "gather_GBps": round(achieved, 1), "clocks": clocks,
-        "gpu_launches": int(launches), "e2e": e2e,
+        "gpu_launches": int(launches), "e2e": e2e, **extra,
     }
     return res, w, inp
 
 
-def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world):
+def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world, backward=None):
     """Same metric through the public API with host buffers: every step
-    copies the step's query (and x) from pinned host memory, runs the
-    forward and copies the output back."""
+    copies the step's query (and x, and for training dy) from pinned host
+    memory, runs the step and copies the output back."""
     import sparse_key_value_b200 as skv
 
     hq = inp["query"].cpu().pin_memory()
     hx = inp["x"].cpu().pin_memory() if w.memplus else None
+    hdy = inp["dy"].cpu().pin_memory() if backward is not None else None
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     dq = torch.empty_like(inp["query"])
     dx = torch.empty_like(inp["x"]) if w.memplus else None
@@ -283,8 +370,12 @@ def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world):
         if dx is not None:
             dx.copy_(hx, non_blocking=True)
             kw2["x"] = dx
+        if hdy is not None:
+            inp["dy"].copy_(hdy, non_blocking=True)
         skv.pkm_forward(dq, inp["subkeys"], inp["values"], w.k, out=out, idx=idx, weights=wts,
                         workspace=ws, **kw2)
+        if backward is not None:
+            backward()
         hout.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -303,7 +394,7 @@ def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world):
         tot += e0.elapsed_time(e1)
     tot = max_over_ranks(tot, world)
     ms = tot / K
-    h2d = hq.numel() * hq.element_size() + (hx.numel() * hx.element_size() if hx is not None else 0)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hx, hdy) if t is not None)
     d2h = hout.numel() * hout.element_size()
     return {"value": round(world * w.T / (ms / 1e3), 1), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4)}

@@ -164,18 +164,54 @@ __global__ void __launch_bounds__(256) dq_kernel(
   const int32_t i1 = lane + 32 < k ? idx[th * k + lane + 32] : 0;
   const float g0 = lane < k ? dS[th * k + lane] : 0.f;
   const float g1 = lane + 32 < k ? dS[th * k + lane + 32] : 0.f;
+  __shared__ int32_t s_a[8][64];
+  __shared__ float s_g[8][64];
+  const int64_t N = (int64_t)n * n;
   for (int c = 0; c < 2; ++c) {
     const int hc = h * 2 + c;
     const typename Elem<DT>::T* Kc = K + (int64_t)hc * n * dh;
+    // sub-key positions of this half, each distinct one once with the sum of
+    // its dS (in slot order), compacted into the warp's list
+    const bool ok0 = lane < k && i0 >= 0 && (int64_t)i0 < N;
+    const bool ok1 = lane + 32 < k && i1 >= 0 && (int64_t)i1 < N;
+    const int32_t a0 = ok0 ? (c == 0 ? i0 / n : i0 % n) : -1;
+    const int32_t a1 = ok1 ? (c == 0 ? i1 / n : i1 % n) : -1;
+    bool lead0 = ok0, lead1 = ok1;
+    float s0 = 0.f, s1 = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int32_t aj = __shfl_sync(0xffffffffu, j < 32 ? a0 : a1, j & 31);
+      const float gj = __shfl_sync(0xffffffffu, j < 32 ? g0 : g1, j & 31);
+      if (aj == a0) {
+        if (j < lane) lead0 = false;
+        if (j >= lane) s0 += gj;
+      }
+      if (aj == a1) {
+        if (j < lane + 32) lead1 = false;
+        if (j >= lane + 32) s1 += gj;
+      }
+    }
+    const unsigned m0 = __ballot_sync(0xffffffffu, lead0);
+    const unsigned m1 = __ballot_sync(0xffffffffu, lead1);
+    const unsigned lt = (1u << lane) - 1u;
+    if (lead0) {
+      const int p = __popc(m0 & lt);
+      s_a[warp][p] = a0;
+      s_g[warp][p] = scale * s0 * rk[(int64_t)hc * n + a0];
+    }
+    if (lead1) {
+      const int p = __popc(m0) + __popc(m1 & lt);
+      s_a[warp][p] = a1;
+      s_g[warp][p] = scale * s1 * rk[(int64_t)hc * n + a1];
+    }
+    __syncwarp();
+    const int m = __popc(m0) + __popc(m1);
     float du[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) du[e] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int32_t id = __shfl_sync(0xffffffffu, j < 32 ? i0 : i1, j & 31);
-      const float g = __shfl_sync(0xffffffffu, j < 32 ? g0 : g1, j & 31);
-      if (id < 0 || (int64_t)id >= (int64_t)n * n) continue;  // reported by bag_dw
-      const int32_t a = c == 0 ? id / n : id % n;
-      const float coef = scale * g * rk[(int64_t)hc * n + a];
+#pragma unroll 4
+    for (int i = 0; i < m; ++i) {
+      const int32_t a = s_a[warp][i];
+      const float coef = s_g[warp][i];
       const typename Elem<DT>::T* row = Kc + (int64_t)a * dh + (int64_t)lane * E;
 #pragma unroll
       for (int cc = 0; cc < NC; ++cc) {
@@ -185,6 +221,7 @@ __global__ void __launch_bounds__(256) dq_kernel(
         for (int e = 0; e < V; ++e) du[cc * V + e] = fmaf(coef, f[e], du[cc * V + e]);
       }
     }
+    __syncwarp();
     const int64_t qrow = th * 2 + c;
     const float r = rq[qrow];
     float u[E];

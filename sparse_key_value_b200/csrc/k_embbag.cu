@@ -6,8 +6,10 @@
 // row ("Memory+ 블록": y ⊙ silu(x W1)).
 //
 // Layout: each thread owns one 16-byte column chunk of a bag's output and
-// walks the bag's rows with kUnroll independent 16-byte loads in flight, so
-// each gathered row is read by consecutive threads in full 128-byte lines.
+// walks the bag's rows with kUnroll = 16 independent 16-byte loads in flight
+// (64 registers, 4 CTAs of 256 threads per SM), so each gathered row is read
+// by consecutive threads in full 128-byte lines.  Measured on B200: 16 loads
+// in flight at 4 CTAs/SM beat 8 at 8 CTAs/SM by 4-5%.
 // fp32 accumulation in row order, one rounding at the store.
 #include "common.cuh"
 #include "kernels.h"
@@ -15,10 +17,10 @@
 namespace pkm {
 
 constexpr int kBagThreads = 256;
-constexpr int kUnroll = 8;
+constexpr int kUnroll = 16;  // independent 16-byte row loads in flight per thread
 
 template <pkm_dtype DT, bool GATE>
-__global__ void __launch_bounds__(kBagThreads) embbag_fwd_kernel(
+__global__ void __launch_bounds__(kBagThreads, 4) embbag_fwd_kernel(
     const typename Elem<DT>::T* __restrict__ table, int64_t n_rows, int d,
     const int32_t* __restrict__ idx, const float* __restrict__ w, int64_t n_bags, int B,
     const typename Elem<DT>::T* __restrict__ gate, typename Elem<DT>::T* __restrict__ out,

@@ -18,7 +18,7 @@ namespace pkm {
 namespace {
 constexpr int kChunk = 256;
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;
 }  // namespace
 
 size_t segsum_workspace(int64_t n, int d) {
@@ -160,56 +160,64 @@ __global__ void __launch_bounds__(kThreads) segsum_chunk_kernel(
   // the chunk's first part continues a segment from the previous chunk?
   const bool cont0 = keys[0] != mark && prev_key == keys[0];
 
+  // valid entries come first (the mark sorts last)
+  __shared__ int n_valid;
+  if (threadIdx.x == 0) n_valid = 0;
+  __syncthreads();
+  {
+    int cnt = 0;
+    for (int j = threadIdx.x; j < len; j += blockDim.x) cnt += keys[j] != mark;
+    if (cnt) atomicAdd(&n_valid, cnt);
+  }
+  __syncthreads();
+  const int lv = n_valid;
+
   for (int ch = threadIdx.x; ch < chunks_d; ch += blockDim.x) {
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
     uint32_t heads = 0;
     bool part_starts = !cont0;
-    int j = 0;
-    while (j < len && keys[j] != mark) {
-      // prefetch up to kUnroll source rows of this segment part
+    // kUnroll source rows in flight regardless of where segments end; the
+    // sums still run entry by entry in sorted order
+    for (int j0 = 0; j0 < lv; j0 += kUnroll) {
       uint4 v[kUnroll];
-      int m = 0;
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        const bool ok = j + u < len && keys[j + u] == keys[j];
-        if (ok) {
-          const typename Elem<DT>::T* row = src + (int64_t)(vals[j + u] / div) * d;
+        const int j = j0 + u;
+        if (j < lv) {
+          const typename Elem<DT>::T* row = src + (int64_t)(vals[j] / div) * d;
           v[u] = ldg_nc_16(row + (int64_t)ch * V);
-          m = u + 1;
         }
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        if (u < m) {
-          float f[V];
-          unpack16<DT>(v[u], f);
-          const float w = cf[j + u];
+        const int j = j0 + u;
+        if (j >= lv) break;
+        float f[V];
+        unpack16<DT>(v[u], f);
+        const float w = cf[j];
 #pragma unroll
-          for (int e = 0; e < V; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+        for (int e = 0; e < V; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+        const uint32_t key = keys[j];
+        if (j + 1 < len && keys[j + 1] == key) continue;  // the part goes on in this chunk
+        // the part ending at entry j is complete within the chunk
+        const bool seg_ends = keys[j + 1] != key;  // keys[len] is the next chunk's first
+        if (part_starts) ++heads;
+        const uint32_t seg = base + heads - 1;
+        if (part_starts && seg_ends) {
+          emit_final<V>(out, seg, key, d, ch, acc, status);
+        } else if (!part_starts) {
+          store_row<V>(ws.carry_first + c * d + (int64_t)ch * V, acc);
+          if (ch == threadIdx.x && threadIdx.x == 0) ws.first_end[c] = seg_ends ? 1u : 0u;
+        } else {
+          store_row<V>(ws.carry_last + c * d + (int64_t)ch * V, acc);
+          if (ch == threadIdx.x && threadIdx.x == 0) ws.last_seg[c] = seg;
         }
-      }
-      const int last = j + m - 1;
-      j += m;
-      if (j < len && keys[j] == keys[last]) continue;  // same part goes on
-      // part [.. last] is complete within the chunk
-      const uint32_t key = keys[last];
-      const bool seg_ends = keys[last + 1] != key;  // keys[len] is the next chunk's first
-      if (part_starts) ++heads;
-      const uint32_t seg = base + heads - 1;
-      if (part_starts && seg_ends) {
-        emit_final<V>(out, seg, key, d, ch, acc, status);
-      } else if (!part_starts) {
-        store_row<V>(ws.carry_first + c * d + (int64_t)ch * V, acc);
-        if (ch == threadIdx.x && threadIdx.x == 0) ws.first_end[c] = seg_ends ? 1u : 0u;
-      } else {
-        store_row<V>(ws.carry_last + c * d + (int64_t)ch * V, acc);
-        if (ch == threadIdx.x && threadIdx.x == 0) ws.last_seg[c] = seg;
-      }
 #pragma unroll
-      for (int e = 0; e < V; ++e) acc[e] = 0.f;
-      part_starts = true;
+        for (int e = 0; e < V; ++e) acc[e] = 0.f;
+        part_starts = true;
+      }
     }
   }
 }

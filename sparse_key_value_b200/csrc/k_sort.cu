@@ -3,8 +3,9 @@
 // reductions (value rows and sub-key rows are summed in sorted order, never
 // with atomics).
 //
-// Per 8-bit digit: (1) per-block digit histograms, (2) one exclusive scan
-// over [digit][block], (3) a stable scatter: each block walks its keys in
+// Per 8-bit digit: (1) per-block digit histograms, (2) an exclusive scan of
+// each digit's row of block counts (one CTA per digit) and of the digit
+// totals, (3) a stable scatter: each block walks its keys in
 // order, 256 at a time; within a warp, __match_any_sync finds the lanes with
 // the same digit and the lane's rank among them; per-warp counts are
 // prefixed in warp order, so equal digits keep their input order.
@@ -36,57 +37,108 @@ __global__ void __launch_bounds__(kThreads) radix_hist_kernel(const uint32_t* __
   hist[(int64_t)threadIdx.x * nblocks + blockIdx.x] = h[threadIdx.x];
 }
 
-// Exclusive scan of data[0..len) in place by one CTA of 1024 threads;
-// *total (optional) receives the sum.  Each thread scans a contiguous run.
+// Exclusive scan of data[0..len) in place by one CTA of 1024 threads, in
+// coalesced tiles of 4096 (four consecutive values per thread); *total /
+// *total64 (optional) receive the sum.
+__device__ __forceinline__ uint32_t block_exclusive_scan_1024(uint32_t x, uint32_t* warp_sums,
+                                                              uint32_t& block_total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t v = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    warp_sums[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  block_total = warp_sums[(blockDim.x >> 5) - 1];
+  const uint32_t before = warp > 0 ? warp_sums[warp - 1] : 0u;
+  __syncthreads();  // warp_sums is reused by the next call
+  return before + incl - x;
+}
+
 __global__ void __launch_bounds__(1024) scan_exclusive_kernel(uint32_t* __restrict__ data,
                                                               int64_t len,
                                                               uint32_t* __restrict__ total,
                                                               int64_t* __restrict__ total64) {
   __shared__ uint32_t warp_sums[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t per = (len + 1023) / 1024;
-  const int64_t b = tid * per, e = min(len, b + per);
-  uint32_t s = 0;
-  for (int64_t i = b; i < e; ++i) s += data[i];
-  // block-wide exclusive scan of the per-thread sums
-  uint32_t x = s;
+  uint32_t carry = 0;
+  for (int64_t base = 0; base < len; base += 4096) {
+    const int64_t i0 = base + (int64_t)threadIdx.x * 4;
+    uint32_t v[4];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_sums[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t w = warp_sums[lane];
+    for (int e = 0; e < 4; ++e) v[e] = i0 + e < len ? data[i0 + e] : 0u;
+    const uint32_t sum = v[0] + v[1] + v[2] + v[3];
+    uint32_t tile_total;
+    uint32_t run = carry + block_exclusive_scan_1024(sum, warp_sums, tile_total);
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
+    for (int e = 0; e < 4; ++e) {
+      if (i0 + e < len) data[i0 + e] = run;
+      run += v[e];
     }
-    warp_sums[lane] = w;
+    carry += tile_total;
+  }
+  if (threadIdx.x == 0) {
+    if (total) *total = carry;
+    if (total64) *total64 = (int64_t)carry;
+  }
+}
+
+// Per-digit scan of the block histograms hist[d][0..nblocks): CTA d replaces
+// its row by the exclusive prefix over blocks and writes the digit total.
+__global__ void __launch_bounds__(1024) radix_digit_scan_kernel(uint32_t* __restrict__ hist,
+                                                                int nblocks,
+                                                                uint32_t* __restrict__ totals) {
+  __shared__ uint32_t warp_sums[32];
+  uint32_t* row = hist + (int64_t)blockIdx.x * nblocks;
+  uint32_t carry = 0;
+  for (int base = 0; base < nblocks; base += 1024) {
+    const int i = base + threadIdx.x;
+    const uint32_t v = i < nblocks ? row[i] : 0u;
+    uint32_t tile_total;
+    const uint32_t ex = block_exclusive_scan_1024(v, warp_sums, tile_total);
+    if (i < nblocks) row[i] = carry + ex;
+    carry += tile_total;
+  }
+  if (threadIdx.x == 0) totals[blockIdx.x] = carry;
+}
+
+// Exclusive scan of the kRadix digit totals (in place).
+__global__ void __launch_bounds__(kRadix) radix_base_scan_kernel(uint32_t* __restrict__ totals) {
+  __shared__ uint32_t t[kRadix];
+  t[threadIdx.x] = totals[threadIdx.x];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t run = 0;
+    for (int d = 0; d < kRadix; ++d) {
+      const uint32_t v = t[d];
+      t[d] = run;
+      run += v;
+    }
   }
   __syncthreads();
-  uint32_t run = x - s + (warp > 0 ? warp_sums[warp - 1] : 0u);
-  for (int64_t i = b; i < e; ++i) {
-    const uint32_t v = data[i];
-    data[i] = run;
-    run += v;
-  }
-  if (tid == 1023) {
-    if (total) *total = run;
-    if (total64) *total64 = (int64_t)run;
-  }
+  totals[threadIdx.x] = t[threadIdx.x];
 }
 
 __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(
     const uint32_t* __restrict__ keys_in, const uint32_t* __restrict__ vals_in, int64_t n,
-    int shift, int nblocks, const uint32_t* __restrict__ offs, uint32_t* __restrict__ keys_out,
+    int shift, int nblocks, const uint32_t* __restrict__ offs,
+    const uint32_t* __restrict__ digit_base, uint32_t* __restrict__ keys_out,
     uint32_t* __restrict__ vals_out) {
   __shared__ uint32_t cnt[kRadix];
   __shared__ uint32_t wh[kWarps][kRadix];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  cnt[tid] = offs[(int64_t)tid * nblocks + blockIdx.x];
+  cnt[tid] = digit_base[tid] + offs[(int64_t)tid * nblocks + blockIdx.x];
   const int64_t base = (int64_t)blockIdx.x * kBlockKeys;
   const unsigned lt = (1u << lane) - 1u;
   for (int r = 0; r < kRounds; ++r) {
@@ -125,8 +177,8 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(
 
 size_t radix_sort_workspace(int64_t n) {
   const int64_t nblocks = (n + kBlockKeys - 1) / kBlockKeys;
-  // histogram/offsets + two key and two value buffers
-  return (size_t)(kRadix * nblocks + 64) * 4 + (size_t)n * 4 * 4 + 4 * 256;
+  // histogram/offsets, digit bases, two key and two value buffers
+  return (size_t)(kRadix * nblocks + 64) * 4 + 256 + kRadix * 4 + (size_t)n * 4 * 4 + 4 * 256;
 }
 
 // Sorts (keys_in, vals_in) into (keys_out, vals_out).  The inputs are not
@@ -139,6 +191,8 @@ cudaError_t launch_radix_sort(const uint32_t* keys_in, const uint32_t* vals_in, 
   char* ws = static_cast<char*>(workspace);
   uint32_t* hist = reinterpret_cast<uint32_t*>(ws);
   size_t off = ((size_t)(kRadix * nblocks + 64) * 4 + 255) / 256 * 256;
+  uint32_t* dbase = reinterpret_cast<uint32_t*>(ws + off);
+  off += (kRadix * 4 + 255) / 256 * 256;
   uint32_t* ka = reinterpret_cast<uint32_t*>(ws + off);
   uint32_t* va = ka + n;
   uint32_t* kb = va + n;
@@ -151,11 +205,11 @@ cudaError_t launch_radix_sort(const uint32_t* keys_in, const uint32_t* vals_in, 
     uint32_t* dk = last ? keys_out : ((p & 1) ? kb : ka);
     uint32_t* dv = last ? vals_out : ((p & 1) ? vb : va);
     radix_hist_kernel<<<nblocks, kThreads, 0, stream>>>(src_k, n, p * 8, nblocks, hist);
-    scan_exclusive_kernel<<<1, 1024, 0, stream>>>(hist, (int64_t)kRadix * nblocks, nullptr,
-                                                  nullptr);
+    radix_digit_scan_kernel<<<kRadix, 1024, 0, stream>>>(hist, nblocks, dbase);
+    radix_base_scan_kernel<<<1, kRadix, 0, stream>>>(dbase);
     radix_scatter_kernel<<<nblocks, kThreads, 0, stream>>>(src_k, src_v, n, p * 8, nblocks, hist,
-                                                           dk, dv);
-    note_launch(3);
+                                                           dbase, dk, dv);
+    note_launch(4);
     src_k = dk;
     src_v = dv;
   }

@@ -50,7 +50,7 @@ cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64
 cudaError_t launch_embbag_fwd(const void* table, int64_t n_rows, int d, pkm_dtype dt,
                               const int32_t* idx, const float* w, int64_t n_bags, int B,
                               const void* gate, void* out, int32_t* status, cudaStream_t stream,
-                              int ctas_per_sm = 8);
+                              int ctas_per_sm = 4);
 
 // Memory+ helpers (bf16).
 cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,
