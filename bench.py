@@ -80,11 +80,24 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Maximum of a per-rank float (timings are max over ranks)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(w, rank: int):
+    """Weak scaling: each rank draws its own token batch and holds a replica of
+    the tables (same table seed on every rank)."""
+    return w.scaled(seed=w.seed + 7919 * rank, table_seed_=w.table_seed)
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, world: int, max_ms_per_step: float) -> float:
+    """Tokens processed by all ranks per second, timed by the slowest rank."""
+    return world * tokens_per_rank / (max_ms_per_step / 1e3)
 
 
 class Clocks:
@@ -203,9 +216,7 @@ def run_ours(args, rank, world, local):
     w = WORKLOADS[args.workload]
     if args.workload == "decode":
         w = w.scaled(T=8)
-    # each rank: its own token batch, a replica of the tables
-    wr = w.scaled(seed=w.seed + 7919 * rank, table_seed_=w.table_seed)
-    inp = make_inputs(wr, "cuda")
+    inp = make_inputs(rank_workload(w, rank), "cuda")
     mp = w.memplus
     kw = dict(x=inp["x"], W1=inp["W1"], W2=inp["W2"]) if mp else {}
     T = w.T
@@ -291,7 +302,7 @@ def run_ours(args, rank, world, local):
     total_ms = max_over_ranks(sum(step_ms), world)
     assert skv.device_error() == 0
     ms_per_step = total_ms / K
-    value = world * T / (ms_per_step / 1e3)
+    value = whole_job_tokens_per_s(T, world, ms_per_step)
 
     # roofline of the dominant kernel: the bag gather (phase 4 -> 5)
     peaks, peak_kind = measured_peaks()
@@ -462,7 +473,7 @@ def run_reference(args, rank, world):
         w = w.scaled(T=8)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(w, dev)
-    per_step = 8 if w.T >= 8 else w.T
+    per_step = min(w.T, 64)  # tokens per step: the per-call set-up is amortised
     spacing = max(1, w.T // (per_step * max(1, args.steps + args.warmup)))
     times, cores = [], 1
     for i in range(args.warmup + args.steps):
