@@ -57,7 +57,8 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
     return o;
   };
   L.rq = take(T * H * 2 * sizeof(float));
-  L.rk = take(H * 2 * n * sizeof(float));
+  // padded by one chunk of columns: the scoring epilogue reads 8 at a time
+  L.rk = take((H * 2 * n + 256) * sizeof(float));
   L.hv = take((size_t)L.splits * T * H * 2 * k * sizeof(float));
   L.hi = take((size_t)L.splits * T * H * 2 * k * sizeof(int32_t));
   if (has_memplus(a)) {
