@@ -78,6 +78,22 @@ __device__ __forceinline__ uint4 ldg_nc_16(const void* p) {
   return v;
 }
 
+// L2 cache policy that keeps lines (evict last): for a small operand read
+// many times while a large stream passes through the cache.
+__device__ __forceinline__ uint64_t l2_policy_keep() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// 16-byte read-only load with an L2 cache policy (see l2_policy_keep).
+__device__ __forceinline__ uint4 ldg_nc_16_hint(const void* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -94,10 +94,12 @@ __device__ __forceinline__ void emit_final(const SegOutDev& o, uint32_t seg, uin
   if (o.grad_rows) {
     if ((int64_t)seg < o.cap) {
       if (ch == 0 && o.uniq_rows) o.uniq_rows[seg] = (int32_t)key;
+      // streaming stores: the gradient rows are written once and must not
+      // push the source rows out of L2
       float* g = o.grad_rows + (int64_t)seg * d + col;
 #pragma unroll
       for (int e = 0; e < V; e += 4)
-        *reinterpret_cast<float4*>(g + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+        __stcs(reinterpret_cast<float4*>(g + e), make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]));
     } else if (ch == 0) {
       set_status(status, PKM_ERR_DEVICE);
     }
@@ -118,7 +120,7 @@ __device__ __forceinline__ void emit_final(const SegOutDev& o, uint32_t seg, uin
     float* g = o.dense_set + (int64_t)key * d + col;
 #pragma unroll
     for (int e = 0; e < V; e += 4)
-      *reinterpret_cast<float4*>(g + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+      __stcs(reinterpret_cast<float4*>(g + e), make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]));
   }
 }
 
@@ -129,30 +131,35 @@ __device__ __forceinline__ void store_row(float* dst, const float* acc) {
     *reinterpret_cast<float4*>(dst + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
 }
 
-template <pkm_dtype DT>
+// One CTA per chunk; each thread owns NV consecutive 16-byte column vectors
+// (W elements) of the rows and walks the chunk's entries in order.
+template <pkm_dtype DT, int NV>
 __global__ void __launch_bounds__(kThreads) segsum_chunk_kernel(
     const uint32_t* __restrict__ skey, const uint32_t* __restrict__ sval, int64_t n,
     uint32_t mark, const float* __restrict__ coef, const typename Elem<DT>::T* __restrict__ src,
     int64_t div, int d, SegWs ws, SegOutDev out, int32_t* status) {
   constexpr int V = Elem<DT>::kVec;
+  constexpr int W = V * NV;
   __shared__ uint32_t keys[kChunk + 1];
-  __shared__ uint32_t vals[kChunk];
+  __shared__ uint32_t rows[kChunk];  // source row of each entry, entry / div
   __shared__ float cf[kChunk];
   const int64_t c = blockIdx.x;
   const int64_t i0 = c * kChunk;
   const int len = (int)min((int64_t)kChunk, n - i0);
+  const uint32_t div32 = (uint32_t)div;
   for (int j = threadIdx.x; j <= len; j += blockDim.x) {
     const int64_t i = i0 + j;
     keys[j] = i < n ? skey[i] : mark;
     if (j < len) {
-      vals[j] = sval[i];
-      cf[j] = keys[j] != mark ? coef[sval[i]] : 0.f;
+      const uint32_t e = sval[i];
+      rows[j] = e / div32;
+      cf[j] = keys[j] != mark ? coef[e] : 0.f;
     }
   }
   const uint32_t prev_key = i0 > 0 ? skey[i0 - 1] : mark;
   __syncthreads();
   const uint32_t base = ws.seg_base[c];
-  const int chunks_d = d / V;
+  const int groups = d / W;
   if (threadIdx.x == 0) {
     ws.first_end[c] = 1;
     ws.last_seg[c] = 0xffffffffu;
@@ -171,34 +178,46 @@ __global__ void __launch_bounds__(kThreads) segsum_chunk_kernel(
   }
   __syncthreads();
   const int lv = n_valid;
+  constexpr int kU = kUnroll / NV;  // source rows in flight per thread
+  // the source rows (dy or the queries) are re-read by many chunks: keep
+  // them in L2 while the gradient rows stream out
+  const uint64_t keep = l2_policy_keep();
 
-  for (int ch = threadIdx.x; ch < chunks_d; ch += blockDim.x) {
-    float acc[V];
+  for (int ch = threadIdx.x; ch < groups; ch += blockDim.x) {
+    float acc[W];
 #pragma unroll
-    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    for (int e = 0; e < W; ++e) acc[e] = 0.f;
     uint32_t heads = 0;
     bool part_starts = !cont0;
-    // kUnroll source rows in flight regardless of where segments end; the
-    // sums still run entry by entry in sorted order
-    for (int j0 = 0; j0 < lv; j0 += kUnroll) {
-      uint4 v[kUnroll];
+    // kU source rows in flight regardless of where segments end; the sums
+    // still run entry by entry in sorted order
+    for (int j0 = 0; j0 < lv; j0 += kU) {
+      uint4 v[kU][NV];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kU; ++u) {
         const int j = j0 + u;
         if (j < lv) {
-          const typename Elem<DT>::T* row = src + (int64_t)(vals[j] / div) * d;
-          v[u] = ldg_nc_16(row + (int64_t)ch * V);
+          const typename Elem<DT>::T* row = src + (int64_t)rows[j] * d + (int64_t)ch * W;
+#pragma unroll
+          for (int q = 0; q < NV; ++q) v[u][q] = ldg_nc_16_hint(row + q * V, keep);
         }
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kU; ++u) {
         const int j = j0 + u;
         if (j >= lv) break;
-        float f[V];
-        unpack16<DT>(v[u], f);
-        const float w = cf[j];
+        float f[W];
 #pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+        for (int q = 0; q < NV; ++q) unpack16<DT>(v[u][q], f + q * V);
+        const float2 w2 = make_float2(cf[j], cf[j]);
+        // acc += w * f, two lanes per instruction (each rounded as fmaf)
+#pragma unroll
+        for (int e = 0; e < W; e += 2) {
+          const float2 r = __ffma2_rn(w2, make_float2(f[e], f[e + 1]),
+                                      make_float2(acc[e], acc[e + 1]));
+          acc[e] = r.x;
+          acc[e + 1] = r.y;
+        }
         const uint32_t key = keys[j];
         if (j + 1 < len && keys[j + 1] == key) continue;  // the part goes on in this chunk
         // the part ending at entry j is complete within the chunk
@@ -206,16 +225,16 @@ __global__ void __launch_bounds__(kThreads) segsum_chunk_kernel(
         if (part_starts) ++heads;
         const uint32_t seg = base + heads - 1;
         if (part_starts && seg_ends) {
-          emit_final<V>(out, seg, key, d, ch, acc, status);
+          emit_final<W>(out, seg, key, d, ch, acc, status);
         } else if (!part_starts) {
-          store_row<V>(ws.carry_first + c * d + (int64_t)ch * V, acc);
+          store_row<W>(ws.carry_first + c * d + (int64_t)ch * W, acc);
           if (ch == threadIdx.x && threadIdx.x == 0) ws.first_end[c] = seg_ends ? 1u : 0u;
         } else {
-          store_row<V>(ws.carry_last + c * d + (int64_t)ch * V, acc);
+          store_row<W>(ws.carry_last + c * d + (int64_t)ch * W, acc);
           if (ch == threadIdx.x && threadIdx.x == 0) ws.last_seg[c] = seg;
         }
 #pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] = 0.f;
+        for (int e = 0; e < W; ++e) acc[e] = 0.f;
         part_starts = true;
       }
     }
@@ -274,18 +293,29 @@ cudaError_t launch_segsum(const uint32_t* skey, const uint32_t* sval, int64_t n,
   if (e != cudaSuccess) return e;
   SegOutDev out{uniq_rows, grad_rows, cap, dense_add, dense_set};
   const int V = dt == PKM_BF16 ? 8 : 4;
-  // one thread per 16-byte column chunk (whole warps, at most kThreads)
-  const int threads = min(kThreads, ((d / V) + 31) / 32 * 32);
+  // two 16-byte column vectors per thread when they divide the row
+  const int NV = (d / V) % 2 == 0 ? 2 : 1;
+  // one thread per column group (whole warps, at most kThreads)
+  const int threads = min(kThreads, ((d / V / NV) + 31) / 32 * 32);
+  const int fix_threads = min(kThreads, ((d / V) + 31) / 32 * 32);
   if (dt == PKM_BF16) {
-    segsum_chunk_kernel<PKM_BF16><<<(unsigned)chunks, threads, 0, stream>>>(
-        skey, sval, n, mark, coef, (const __nv_bfloat16*)src, div, d, ws, out, status);
-    segsum_fixup_kernel<8><<<(unsigned)chunks, threads, 0, stream>>>(skey, n, d, ws, out,
-                                                                     status);
+    if (NV == 2)
+      segsum_chunk_kernel<PKM_BF16, 2><<<(unsigned)chunks, threads, 0, stream>>>(
+          skey, sval, n, mark, coef, (const __nv_bfloat16*)src, div, d, ws, out, status);
+    else
+      segsum_chunk_kernel<PKM_BF16, 1><<<(unsigned)chunks, threads, 0, stream>>>(
+          skey, sval, n, mark, coef, (const __nv_bfloat16*)src, div, d, ws, out, status);
+    segsum_fixup_kernel<8><<<(unsigned)chunks, fix_threads, 0, stream>>>(skey, n, d, ws, out,
+                                                                         status);
   } else {
-    segsum_chunk_kernel<PKM_F32><<<(unsigned)chunks, threads, 0, stream>>>(
-        skey, sval, n, mark, coef, (const float*)src, div, d, ws, out, status);
-    segsum_fixup_kernel<4><<<(unsigned)chunks, threads, 0, stream>>>(skey, n, d, ws, out,
-                                                                     status);
+    if (NV == 2)
+      segsum_chunk_kernel<PKM_F32, 2><<<(unsigned)chunks, threads, 0, stream>>>(
+          skey, sval, n, mark, coef, (const float*)src, div, d, ws, out, status);
+    else
+      segsum_chunk_kernel<PKM_F32, 1><<<(unsigned)chunks, threads, 0, stream>>>(
+          skey, sval, n, mark, coef, (const float*)src, div, d, ws, out, status);
+    segsum_fixup_kernel<4><<<(unsigned)chunks, fix_threads, 0, stream>>>(skey, n, d, ws, out,
+                                                                         status);
   }
   note_launch(2);
   return cudaGetLastError();

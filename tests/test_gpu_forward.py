@@ -21,9 +21,11 @@ def _cuda():
     assert skv.device_error() == 0
 
 
-def run_forward(w, inp=None, sample=None):
+def run_forward(w, inp=None, sample=None, max_exempt=0.01):
     """Run the GPU forward of workload ``w`` and check it against the oracle
-    on the tokens ``sample`` (all tokens by default)."""
+    on the tokens ``sample`` (all tokens by default).  At most a fraction
+    ``max_exempt`` of the (token, head) selections may differ from the
+    oracle's, each within the tie rule."""
     import oracle
 
     if inp is None:
@@ -50,7 +52,7 @@ def run_forward(w, inp=None, sample=None):
     weights_close(wts[sd].cpu().numpy(), ref["w_ref"], W_RTOL[w.dtype])
     err = close(out[sd].float().cpu().numpy(), ref["out_ref"], RTOL[w.dtype], "out")
     n_th = len(sample) * w.H
-    assert ref["exempt"] <= max(1, 0.01 * n_th), f"{ref['exempt']} tie exemptions of {n_th}"
+    assert ref["exempt"] <= max(1, max_exempt * n_th), f"{ref['exempt']} tie exemptions of {n_th}"
     return dict(ref=ref, idx=idx_g, err=err, inp=inp)
 
 
@@ -63,6 +65,10 @@ SMALL = [
     ("tc-two-chunks", 300, 2, 128, 512, 16, 64, "bf16"),
     ("tc-k32-many-tiles", 1000, 1, 64, 1024, 32, 128, "bf16"),
     ("tc-k1", 130, 2, 64, 256, 1, 16, "bf16"),
+    # five chunks, the last one ragged: prefix pass over four, main pass over five
+    ("tc-prefix-ragged", 200, 2, 64, 1100, 32, 32, "bf16"),
+    # n % 4 != 0 takes the SIMT scoring path even with n >= 256
+    ("bf16-n-mod4", 90, 2, 64, 258, 8, 16, "bf16"),
     ("f32-k64", 70, 2, 32, 64, 64, 40, "f32"),
     ("f32-k-equals-n", 33, 1, 16, 5, 5, 24, "f32"),
 ]
@@ -73,6 +79,35 @@ def test_forward_small(case):
     name, T, H, dh, n, k, dv, dt = case
     w = WORKLOADS["pkm"].scaled(name=name, T=T, H=H, d_half=dh, n_sub=n, k=k, d_v=dv, dtype=dt,
                                 seed=sum(map(ord, name)))
+    run_forward(w)
+
+
+@pytest.mark.parametrize("sign", [1.0, -1.0], ids=["aligned", "anti-aligned"])
+def test_forward_extreme_scores(sign):
+    """Queries (anti-)aligned with every sub-key of their (head, half): the
+    scores sit around +/-6.5, so the group maxima fall outside the histogram
+    range of the prefix pass (its bound saturates at the top bin, or is empty
+    at the bottom); the selection must still be exact.  A shared direction
+    also crowds the scores, so near-ties (each still within the tie rule)
+    are more frequent than on isotropic inputs: up to 3% are allowed."""
+    w = WORKLOADS["pkm"].scaled(name="extreme", T=260, H=2, d_half=512, n_sub=512, k=32, d_v=32,
+                                seed=77)
+    inp = make_inputs(w, "cuda")
+    g = torch.Generator().manual_seed(78)
+    e = torch.randn(w.H, 2, w.d_half, generator=g)
+    e = e / e.norm(dim=-1, keepdim=True)
+    q = inp["query"].float().cpu() + sign * 10.0 * e.unsqueeze(0)
+    K = inp["subkeys"].float().cpu() + 1.0 * e.unsqueeze(2)
+    inp["query"] = q.to(torch.bfloat16).cuda()
+    inp["subkeys"] = K.to(torch.bfloat16).cuda()
+    run_forward(w, inp=inp, max_exempt=0.03)
+
+
+def test_forward_zipf_scores():
+    """Sub-keys biased towards a shared direction (the training workload's
+    Zipf popularity) at a small size: a heavy upper tail of scores."""
+    w = WORKLOADS["train"].scaled(name="zipf-small", T=400, H=2, d_half=128, n_sub=1024, k=32,
+                                  d_v=32, train=False)
     run_forward(w)
 
 
