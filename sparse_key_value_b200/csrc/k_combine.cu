@@ -188,90 +188,150 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(
 // One thread per (token, head), used when each half has a single list.  The
 // k x k grid S[i][j] = s1[i] + s2[j] decreases along rows and columns, so its
 // cells can be taken best first with a max-heap frontier: start at (0, 0);
-// taking (i, j) admits (i, j+1) and, on the first column, (i+1, 0).  Lists
-// and heap live in shared memory as [slot][thread] (conflict-free).
+// taking (i, j) admits (i, j+1) and, on the first column, (i+1, 0).
+// Heap entries are the order-preserving score bits and the cell (i, j); two
+// cells with the same score are ordered by their row ids a1[i]*n + b2[j]
+// (smaller id first), computed only on such ties.  The CTA's lists form one
+// contiguous block of hv / hi and its outputs one contiguous block of idx /
+// w: both move through shared memory with coalesced accesses.  Per-thread
+// arrays are stored [slot][thread] with a padded row (conflict-free).
 constexpr int kThreadCombine = 64;
+constexpr int kTcPad = kThreadCombine + 1;  // row stride of the [slot][thread] arrays
 
 __global__ void __launch_bounds__(kThreadCombine) combine_thread_kernel(
     const float* __restrict__ hv, const int32_t* __restrict__ hi, int64_t TH, int n, int k,
     int32_t* __restrict__ idx, float* __restrict__ wout) {
   extern __shared__ unsigned char sm[];
   const int tid = threadIdx.x;
-  constexpr int B = kThreadCombine;
-  float* s1 = reinterpret_cast<float*>(sm);          // [k][B]
-  float* s2 = s1 + k * B;                            // [k][B]
-  int32_t* a1 = reinterpret_cast<int32_t*>(s2 + k * B);
-  int32_t* b2 = a1 + k * B;
-  uint64_t* hk = reinterpret_cast<uint64_t*>(b2 + k * B);  // heap keys [k+2][B]
-  uint16_t* hc = reinterpret_cast<uint16_t*>(hk + (k + 2) * B);  // heap cells
-  float* outS = reinterpret_cast<float*>(hc + (k + 2) * B);      // [k][B]
-  const int64_t th = (int64_t)blockIdx.x * B + tid;
-  if (th >= TH) return;
-  for (int j = 0; j < k; ++j) {
-    s1[j * B + tid] = hv[(th * 2) * k + j];
-    a1[j * B + tid] = hi[(th * 2) * k + j];
-    s2[j * B + tid] = hv[(th * 2 + 1) * k + j];
-    b2[j * B + tid] = hi[(th * 2 + 1) * k + j];
-  }
-  auto key_at = [&](int i, int j) {
-    return key_of(s1[i * B + tid] + s2[j * B + tid], a1[i * B + tid] * n + b2[j * B + tid]);
-  };
-  int size = 0;
-  auto push = [&](uint64_t key, int cell) {
-    int pos = ++size;
-    while (pos > 1) {
-      const int par = pos >> 1;
-      const uint64_t pk = hk[par * B + tid];
-      if (pk >= key) break;
-      hk[pos * B + tid] = pk;
-      hc[pos * B + tid] = hc[par * B + tid];
-      pos = par;
-    }
-    hk[pos * B + tid] = key;
-    hc[pos * B + tid] = (uint16_t)cell;
-  };
-  push(key_at(0, 0), 0);
-  for (int r = 0; r < k; ++r) {
-    const uint64_t top = hk[1 * B + tid];
-    const int cell = hc[1 * B + tid];
-    // pop
-    const uint64_t lk = hk[size * B + tid];
-    const uint16_t lc = hc[size * B + tid];
-    --size;
-    int pos = 1;
-    while (true) {
-      int ch = pos * 2;
-      if (ch > size) break;
-      uint64_t ck = hk[ch * B + tid];
-      if (ch < size) {
-        const uint64_t rk2 = hk[(ch + 1) * B + tid];
-        if (rk2 > ck) {
-          ck = rk2;
-          ++ch;
-        }
+  constexpr int P = kTcPad;
+  float* s12 = reinterpret_cast<float*>(sm);                           // [2k][P]: s1, s2
+  uint32_t* hk = reinterpret_cast<uint32_t*>(s12 + 2 * k * P);         // heap scores [k+2][P]
+  float* mz = reinterpret_cast<float*>(hk + (k + 2) * P);              // [2][P]: max, 1/sum
+  uint16_t* ab = reinterpret_cast<uint16_t*>(mz + 2 * P);              // [2k][P]: a1, b2
+  uint16_t* hc = ab + 2 * k * P;                                       // heap cells [k+2][P]
+  uint16_t* rec = hc + (k + 2) * P;                                    // taken cells [k][P]
+  const int64_t th0 = (int64_t)blockIdx.x * kThreadCombine;
+  const int nth = (int)min((int64_t)kThreadCombine, TH - th0);  // (t, h) pairs of this CTA
+
+  // 1. the CTA's 2k-long list rows, element e = t_local * 2k + c * k + j
+  {
+    const int total = nth * 2 * k;
+    const float* gv = hv + th0 * 2 * k;
+    const int32_t* gi = hi + th0 * 2 * k;
+    const bool vec = ((reinterpret_cast<uintptr_t>(gv) | reinterpret_cast<uintptr_t>(gi)) & 15u) == 0;
+    const int nvec = vec ? total / 4 : 0;
+    for (int q = tid; q < nvec; q += kThreadCombine) {
+      const float4 v = reinterpret_cast<const float4*>(gv)[q];
+      const int4 w = reinterpret_cast<const int4*>(gi)[q];
+      const float vs[4] = {v.x, v.y, v.z, v.w};
+      const int32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = 4 * q + u;
+        const int tl = e / (2 * k), r = e - tl * 2 * k;
+        s12[r * P + tl] = vs[u];
+        ab[r * P + tl] = (uint16_t)ws[u];
       }
-      if (ck <= lk) break;
-      hk[pos * B + tid] = ck;
-      hc[pos * B + tid] = hc[ch * B + tid];
-      pos = ch;
     }
-    if (size > 0 || pos > 1) {
-      hk[pos * B + tid] = lk;
-      hc[pos * B + tid] = lc;
+    for (int e = nvec * 4 + tid; e < total; e += kThreadCombine) {
+      const int tl = e / (2 * k), r = e - tl * 2 * k;
+      s12[r * P + tl] = gv[e];
+      ab[r * P + tl] = (uint16_t)gi[e];
     }
-    // emit
-    idx[th * k + r] = (int32_t)(0xffffffffu - (uint32_t)top);
-    outS[r * B + tid] = unordf((uint32_t)(top >> 32));
-    const int i = cell >> 6, j = cell & 63;
-    if (j + 1 < k) push(key_at(i, j + 1), i * 64 + j + 1);
-    if (j == 0 && i + 1 < k) push(key_at(i + 1, 0), (i + 1) * 64);
   }
-  // softmax over the k kept scores (entry 0 is the maximum)
-  const float m = outS[tid];
-  float z = 0.f;
-  for (int r = 0; r < k; ++r) z += expf(outS[r * B + tid] - m);
-  const float inv = 1.0f / z;
-  for (int r = 0; r < k; ++r) wout[th * k + r] = expf(outS[r * B + tid] - m) * inv;
+  __syncthreads();
+
+  const float* s1 = s12;
+  const float* s2 = s12 + k * P;
+  const uint16_t* a1 = ab;
+  const uint16_t* b2 = ab + k * P;
+  if (tid < nth) {
+    auto id_of = [&](int cell) {
+      return (int32_t)a1[(cell >> 6) * P + tid] * n + (int32_t)b2[(cell & 63) * P + tid];
+    };
+    // is entry (s, c) ahead of entry (t, d)?
+    auto ahead = [&](uint32_t s, int c, uint32_t t, int d) {
+      return s != t ? s > t : id_of(c) < id_of(d);
+    };
+    auto score_at = [&](int i, int j) { return ordf(s1[i * P + tid] + s2[j * P + tid]); };
+    int size = 0;
+    auto push = [&](uint32_t key, int cell) {
+      int pos = ++size;
+      while (pos > 1) {
+        const int par = pos >> 1;
+        const uint32_t pk = hk[par * P + tid];
+        const int pc = hc[par * P + tid];
+        if (!ahead(key, cell, pk, pc)) break;
+        hk[pos * P + tid] = pk;
+        hc[pos * P + tid] = (uint16_t)pc;
+        pos = par;
+      }
+      hk[pos * P + tid] = key;
+      hc[pos * P + tid] = (uint16_t)cell;
+    };
+    push(score_at(0, 0), 0);
+    for (int r = 0; r < k; ++r) {
+      const int cell = hc[1 * P + tid];
+      // pop
+      const uint32_t lk = hk[size * P + tid];
+      const int lc = hc[size * P + tid];
+      --size;
+      int pos = 1;
+      while (true) {
+        int ch = pos * 2;
+        if (ch > size) break;
+        uint32_t ck = hk[ch * P + tid];
+        int cc = hc[ch * P + tid];
+        if (ch < size) {
+          const uint32_t k2 = hk[(ch + 1) * P + tid];
+          const int c2 = hc[(ch + 1) * P + tid];
+          if (ahead(k2, c2, ck, cc)) {
+            ck = k2;
+            cc = c2;
+            ++ch;
+          }
+        }
+        if (!ahead(ck, cc, lk, lc)) break;
+        hk[pos * P + tid] = ck;
+        hc[pos * P + tid] = (uint16_t)cc;
+        pos = ch;
+      }
+      if (size > 0 || pos > 1) {
+        hk[pos * P + tid] = lk;
+        hc[pos * P + tid] = (uint16_t)lc;
+      }
+      rec[r * P + tid] = (uint16_t)cell;
+      const int i = cell >> 6, j = cell & 63;
+      if (j + 1 < k) push(score_at(i, j + 1), i * 64 + j + 1);
+      if (j == 0 && i + 1 < k) push(score_at(i + 1, 0), (i + 1) * 64);
+    }
+    // softmax normaliser over the k kept scores (the first is the maximum)
+    const int c0 = rec[tid];
+    const float m = s1[(c0 >> 6) * P + tid] + s2[(c0 & 63) * P + tid];
+    float z = 0.f;
+    for (int r = 0; r < k; ++r) {
+      const int c = rec[r * P + tid];
+      z += expf(s1[(c >> 6) * P + tid] + s2[(c & 63) * P + tid] - m);
+    }
+    mz[tid] = m;
+    mz[P + tid] = 1.0f / z;
+  }
+  __syncthreads();
+
+  // 2. the CTA's outputs, element e = t_local * k + r
+  {
+    const int total = nth * k;
+    int32_t* gi = idx + th0 * k;
+    float* gw = wout + th0 * k;
+    for (int e = tid; e < total; e += kThreadCombine) {
+      const int tl = e / k, r = e - tl * k;
+      const int c = rec[r * P + tl];
+      const int i = c >> 6, j = c & 63;
+      const float sc = s1[i * P + tl] + s2[j * P + tl];
+      gi[e] = (int32_t)a1[i * P + tl] * n + (int32_t)b2[j * P + tl];
+      gw[e] = expf(sc - mz[tl]) * mz[P + tl];
+    }
+  }
 }
 
 }  // namespace
@@ -281,8 +341,9 @@ cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64
   const int64_t TH = T * H;
   if (TH <= 0) return cudaSuccess;
   if (splits == 1) {
-    const size_t smem = (size_t)kThreadCombine *
-                        ((size_t)k * 16 + (size_t)(k + 2) * 10 + (size_t)k * 4);
+    const size_t smem = (size_t)kTcPad * ((size_t)k * 8 + (size_t)(k + 2) * 4 + 8 +
+                                          (size_t)k * 4 + (size_t)(k + 2) * 2 + (size_t)k * 2);
+    if (n > 65536) return cudaErrorInvalidValue;  // sub-key ids are held as 16 bits
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(combine_thread_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)

@@ -17,36 +17,73 @@
 
 namespace pkm {
 
-// One warp per row.
-template <pkm_dtype DT>
-__global__ void row_rnorm_kernel(const typename Elem<DT>::T* __restrict__ x, int64_t rows,
-                                 int d, float* __restrict__ r) {
+// One warp per ROWS consecutive rows of at most 32 * NVL 16-byte vectors:
+// every lane issues its loads for all ROWS rows before reducing, so about
+// eight 16-byte loads per lane are in flight.
+template <pkm_dtype DT, int NVL, int ROWS>
+__global__ void __launch_bounds__(256) row_rnorm_kernel(const typename Elem<DT>::T* __restrict__ x,
+                                                        int64_t rows, int d,
+                                                        float* __restrict__ r) {
   constexpr int V = Elem<DT>::kVec;
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const typename Elem<DT>::T* p = x + row * d;
-  float ss = 0.f;
-  for (int c = lane * V; c < d; c += 32 * V) {
-    float f[V];
-    unpack16<DT>(ldg_nc_16(p + c), f);
+  const int64_t row0 = ((int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32) * ROWS;
+  if (row0 >= rows) return;
+  const int nv = d / V;  // vectors per row
+  uint4 v[ROWS][NVL];
 #pragma unroll
-    for (int e = 0; e < V; ++e) ss = fmaf(f[e], f[e], ss);
+  for (int q = 0; q < ROWS; ++q)
+#pragma unroll
+    for (int u = 0; u < NVL; ++u) {
+      const int c = lane + 32 * u;
+      if (row0 + q < rows && c < nv) v[q][u] = ldg_nc_16(x + (row0 + q) * d + (int64_t)c * V);
+    }
+#pragma unroll
+  for (int q = 0; q < ROWS; ++q) {
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < NVL; ++u) {
+      const int c = lane + 32 * u;
+      if (row0 + q < rows && c < nv) {
+        float f[V];
+        unpack16<DT>(v[q][u], f);
+#pragma unroll
+        for (int e = 0; e < V; ++e) ss = fmaf(f[e], f[e], ss);
+      }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0 && row0 + q < rows) r[row0 + q] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
   }
-  ss = warp_sum(ss);
-  if (lane == 0) r[row] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
 }
 
+template <pkm_dtype DT, int NVL>
+static void launch_rnorm_t(const void* x, int64_t rows, int d, float* r, cudaStream_t stream) {
+  constexpr int ROWS = NVL >= 8 ? 1 : 8 / NVL;
+  const int warps = 8;
+  const int64_t groups = (rows + ROWS - 1) / ROWS;
+  dim3 grid((unsigned)((groups + warps - 1) / warps));
+  row_rnorm_kernel<DT, NVL, ROWS><<<grid, warps * 32, 0, stream>>>(
+      (const typename Elem<DT>::T*)x, rows, d, r);
+}
+
+// d <= 2048 (bf16) / 1024 (fp32): the forward and backward validate d_half.
 cudaError_t launch_row_rnorm(const void* x, pkm_dtype dt, int64_t rows, int d, float* r,
                              cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  const int warps = 8;
-  dim3 grid((unsigned)((rows + warps - 1) / warps));
-  if (dt == PKM_BF16)
-    row_rnorm_kernel<PKM_BF16><<<grid, warps * 32, 0, stream>>>(
-        (const __nv_bfloat16*)x, rows, d, r);
-  else
-    row_rnorm_kernel<PKM_F32><<<grid, warps * 32, 0, stream>>>((const float*)x, rows, d, r);
+  const int V = dt == PKM_BF16 ? 8 : 4;
+  const int nvl = (d / V + 31) / 32;
+  if (nvl > 16) return cudaErrorInvalidValue;
+#define PKM_RNORM(T_)                                            \
+  if (nvl <= 1) launch_rnorm_t<T_, 1>(x, rows, d, r, stream);   \
+  else if (nvl <= 2) launch_rnorm_t<T_, 2>(x, rows, d, r, stream); \
+  else if (nvl <= 4) launch_rnorm_t<T_, 4>(x, rows, d, r, stream); \
+  else if (nvl <= 8) launch_rnorm_t<T_, 8>(x, rows, d, r, stream); \
+  else launch_rnorm_t<T_, 16>(x, rows, d, r, stream)
+  if (dt == PKM_BF16) {
+    PKM_RNORM(PKM_BF16);
+  } else {
+    PKM_RNORM(PKM_F32);
+  }
+#undef PKM_RNORM
   note_launch();
   return cudaGetLastError();
 }
