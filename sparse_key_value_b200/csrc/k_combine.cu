@@ -13,8 +13,8 @@
 // as 64-bit keys (order-preserving score bits, then the complemented row
 // id, so equal scores favour the smaller id), sorts them with a bitonic
 // network spread over its lanes, and keeps the first k.  When the per-half
-// lists come in several column splits, the warp first merges each half's
-// splits the same way.
+// lists come in several column splits (each sorted), the warp first merges
+// each half's splits pairwise in a binary tree of bitonic merges.
 #include <math.h>
 
 #include "common.cuh"
@@ -25,7 +25,6 @@ namespace pkm {
 namespace {
 
 constexpr int kCombWarps = 8;
-constexpr int kMaxSlots = 16;  // keys per lane: up to 512 candidates per warp
 
 __device__ __forceinline__ uint32_t ordf(float s) {
   uint32_t u = __float_as_uint(s);
@@ -46,7 +45,7 @@ __device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int m) {
 }
 
 // Bitonic sort, descending, of the 32*S keys held as v[s] on lane l at
-// position p = s * 32 + l.  S is a power of two <= kMaxSlots.
+// position p = s * 32 + l.  S is a power of two.
 template <int S>
 __device__ __forceinline__ void warp_sort_desc(uint64_t (&v)[S]) {
   const int lane = threadIdx.x & 31;
@@ -85,6 +84,25 @@ __device__ __forceinline__ void warp_sort_desc(uint64_t (&v)[S]) {
   }
 }
 
+// a (sorted desc, one key per lane) <- the 32 largest keys of a and b (b also
+// sorted desc, one key per lane): the lane-wise maximum of a and reversed b
+// is bitonic, and five exchange stages sort it.
+__device__ __forceinline__ uint64_t warp_merge_top32(uint64_t a, uint64_t b) {
+  const int lane = threadIdx.x & 31;
+  uint32_t lo = (uint32_t)b, hi = (uint32_t)(b >> 32);
+  lo = __shfl_sync(0xffffffffu, lo, 31 - lane);
+  hi = __shfl_sync(0xffffffffu, hi, 31 - lane);
+  const uint64_t br = ((uint64_t)hi << 32) | lo;
+  uint64_t v = a > br ? a : br;
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+    const uint64_t o = shfl_xor64(v, stride);
+    const bool lower = (lane & stride) == 0;
+    v = lower ? (v > o ? v : o) : (v > o ? o : v);
+  }
+  return v;
+}
+
 // number of candidate cells (i, j), i, j < k, with (i+1)(j+1) <= k
 __host__ __device__ __forceinline__ int pruned_cells(int k) {
   int c = 0;
@@ -92,14 +110,16 @@ __host__ __device__ __forceinline__ int pruned_cells(int k) {
   return c;
 }
 
-template <int S>
+// MS: a power of two >= the number of column splits (k <= 32 here).
+template <int MS>
 __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(
     const float* __restrict__ hv, const int32_t* __restrict__ hi, int splits, int64_t T, int H,
     int n, int k, int32_t* __restrict__ idx, float* __restrict__ wout) {
-  __shared__ float lv[kCombWarps][2][64];
-  __shared__ int32_t li[kCombWarps][2][64];
-  __shared__ uint8_t cell_i[32 * kMaxSlots];
-  __shared__ uint8_t cell_j[32 * kMaxSlots];
+  constexpr int S = 4;  // 128 sort slots: the (i+1)(j+1) <= k cells, k <= 32
+  __shared__ float lv[kCombWarps][2][32];
+  __shared__ int32_t li[kCombWarps][2][32];
+  __shared__ uint8_t cell_i[32 * S];
+  __shared__ uint8_t cell_j[32 * S];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t th = (int64_t)blockIdx.x * kCombWarps + warp;  // t * H + h
   const int64_t TH2 = T * H * 2;
@@ -118,36 +138,29 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(
   __syncthreads();
   if (th >= T * H) return;
 
-  // 1. each half's k best, merging the column splits when there are several
+  // 1. each half's k best: the splits' sorted lists (one key per lane),
+  // merged pairwise in a binary tree
   for (int c = 0; c < 2; ++c) {
     const int64_t row = th * 2 + c;
-    if (splits == 1) {
-      for (int j = lane; j < k; j += 32) {
-        lv[warp][c][j] = hv[row * k + j];
-        li[warp][c][j] = hi[row * k + j];
-      }
-    } else {
-      uint64_t v[S];
+    uint64_t v[MS];
 #pragma unroll
-      for (int s = 0; s < S; ++s) {
-        const int p = s * 32 + lane;
-        const int sp = p / k, j = p - sp * k;
-        v[s] = 0;
-        if (sp < splits) {
-          const int64_t off = ((int64_t)sp * TH2 + row) * k + j;
-          const int32_t iv = hi[off];
-          if (iv != 0x7fffffff) v[s] = key_of(hv[off], iv);
-        }
+    for (int sp = 0; sp < MS; ++sp) {
+      v[sp] = 0;
+      if (sp < splits && lane < k) {
+        const int64_t off = ((int64_t)sp * TH2 + row) * k + lane;
+        const int32_t iv = hi[off];
+        if (iv != 0x7fffffff) v[sp] = key_of(hv[off], iv);
       }
-      warp_sort_desc<S>(v);
+    }
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        const int p = s * 32 + lane;
-        if (p < k) {
-          lv[warp][c][p] = unordf((uint32_t)(v[s] >> 32));
-          li[warp][c][p] = (int32_t)(0xffffffffu - (uint32_t)v[s]);
-        }
-      }
+    for (int width = 1; width < MS; width <<= 1) {
+#pragma unroll
+      for (int a = 0; a + width < MS; a += 2 * width)
+        if (a + width < splits) v[a] = warp_merge_top32(v[a], v[a + width]);
+    }
+    if (lane < k) {
+      lv[warp][c][lane] = unordf((uint32_t)(v[0] >> 32));
+      li[warp][c][lane] = (int32_t)(0xffffffffu - (uint32_t)v[0]);
     }
   }
   __syncwarp();
@@ -169,19 +182,13 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(
 
   // 3. softmax over the k kept scores (entry 0 is the maximum)
   const float S0 = unordf((uint32_t)(v[0] >> 32));  // lane's entry `lane`
-  const float S1 = unordf((uint32_t)(v[1] >> 32));  // entry `lane + 32`
   const float m = __shfl_sync(0xffffffffu, S0, 0);
   const float e0 = lane < k ? expf(S0 - m) : 0.f;
-  const float e1 = lane + 32 < k ? expf(S1 - m) : 0.f;
-  const float z = warp_sum(e0 + e1);
+  const float z = warp_sum(e0);
   const float inv = 1.0f / z;
   if (lane < k) {
     idx[th * k + lane] = (int32_t)(0xffffffffu - (uint32_t)v[0]);
     wout[th * k + lane] = e0 * inv;
-  }
-  if (lane + 32 < k) {
-    idx[th * k + lane + 32] = (int32_t)(0xffffffffu - (uint32_t)v[1]);
-    wout[th * k + lane + 32] = e1 * inv;
   }
 }
 
@@ -353,19 +360,20 @@ cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64
     note_launch();
     return cudaGetLastError();
   }
-  const int need = max(pruned_cells(k), splits > 1 ? splits * k : 0);
+  // several column splits (tensor-core scoring, k <= 32)
+  if (k > 32 || splits > 32) return cudaErrorInvalidValue;
   dim3 grid((unsigned)((TH + kCombWarps - 1) / kCombWarps));
   const int threads = kCombWarps * 32;
-  if (need <= 64)
+  if (splits <= 2)
     combine_kernel<2><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
-  else if (need <= 128)
+  else if (splits <= 4)
     combine_kernel<4><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
-  else if (need <= 256)
+  else if (splits <= 8)
     combine_kernel<8><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
-  else if (need <= 512)
+  else if (splits <= 16)
     combine_kernel<16><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
   else
-    return cudaErrorInvalidValue;
+    combine_kernel<32><<<grid, threads, 0, stream>>>(hv, hi, splits, T, H, n, k, idx, w);
   note_launch();
   return cudaGetLastError();
 }

@@ -12,26 +12,68 @@
 
 namespace pkm {
 
-__global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src, int rows, int cols,
-                                      __nv_bfloat16* __restrict__ dst) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < rows && c < cols) tile[i][threadIdx.x] = src[(int64_t)r * cols + c];
+// dst[c][r] = src[r][c] for a rows x cols bf16 matrix.  64 x 64 tiles: rows
+// are read and written as 16-byte vectors (coalesced 128-byte segments), the
+// transpose itself happens element-wise in shared memory.
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src,
+                                                             int rows, int cols,
+                                                             __nv_bfloat16* __restrict__ dst) {
+  __shared__ uint16_t tile[64][65];
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  const int tid = threadIdx.x;
+  const uint16_t* s16 = reinterpret_cast<const uint16_t*>(src);
+  const bool vec_src = (cols % 8) == 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = (tid >> 3) + 32 * h;  // tile row: source row r0 + i
+    const int q = tid & 7;              // 16-byte vector of the row
+    const int r = r0 + i, c = c0 + 8 * q;
+    uint16_t v[8];
+    if (r < rows && vec_src && c + 8 <= cols) {
+      const uint4 u = *reinterpret_cast<const uint4*>(s16 + (int64_t)r * cols + c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = (uint16_t)(w[e] & 0xffffu);
+        v[2 * e + 1] = (uint16_t)(w[e] >> 16);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        v[e] = (r < rows && c + e < cols) ? s16[(int64_t)r * cols + c + e] : (uint16_t)0;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tile[i][8 * q + e] = v[e];
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    int c = c0 + i, r = r0 + threadIdx.x;  // dst[c][r] = src[r][c]
-    if (r < rows && c < cols) dst[(int64_t)c * rows + r] = tile[threadIdx.x][i];
+  const bool vec_dst = (rows % 8) == 0;
+  uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int j = (tid >> 3) + 32 * h;  // tile column: destination row c0 + j
+    const int q = tid & 7;
+    const int c = c0 + j, r = r0 + 8 * q;
+    if (c >= cols) continue;
+    uint16_t v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = tile[8 * q + e][j];
+    uint16_t* d = d16 + (int64_t)c * rows + r;
+    if (vec_dst && r + 8 <= rows) {
+      *reinterpret_cast<uint4*>(d) =
+          make_uint4(v[0] | ((uint32_t)v[1] << 16), v[2] | ((uint32_t)v[3] << 16),
+                     v[4] | ((uint32_t)v[5] << 16), v[6] | ((uint32_t)v[7] << 16));
+    } else {
+      for (int e = 0; e < 8 && r + e < rows; ++e) d[e] = v[e];
+    }
   }
 }
 
 cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,
                                   cudaStream_t stream) {
-  dim3 grid((cols + 31) / 32, (rows + 31) / 32), block(32, 8);
-  transpose_bf16_kernel<<<grid, block, 0, stream>>>((const __nv_bfloat16*)src, rows, cols,
-                                                    (__nv_bfloat16*)dst);
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+  transpose_bf16_kernel<<<grid, 256, 0, stream>>>((const __nv_bfloat16*)src, rows, cols,
+                                                  (__nv_bfloat16*)dst);
   note_launch();
   return cudaGetLastError();
 }

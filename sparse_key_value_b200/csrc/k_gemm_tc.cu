@@ -148,8 +148,11 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
           for (int j = 0; j < 16; ++j) {
             float a = __uint_as_float(r[2 * j]), b = __uint_as_float(r[2 * j + 1]);
             if (EPI == 1) {
-              a = a / (1.0f + expf(-a));
-              b = b / (1.0f + expf(-b));
+              // silu with the fast exponential and division intrinsics (a few
+              // ulp in fp32, far below the bf16 rounding that follows; -a
+              // large: __expf -> inf, a / inf -> -0)
+              a = __fdividef(a, 1.0f + __expf(-a));
+              b = __fdividef(b, 1.0f + __expf(-b));
             }
             packed[j] = pack_bf16x2(a, b);
           }

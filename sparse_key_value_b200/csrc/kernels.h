@@ -52,6 +52,16 @@ cudaError_t launch_embbag_fwd(const void* table, int64_t n_rows, int d, pkm_dtyp
                               const void* gate, void* out, int32_t* status, cudaStream_t stream,
                               int ctas_per_sm = 4);
 
+// The same gather for small batches (see k_embbag_split.cu): fp32 partial
+// sums of row groups in `part` (embbag_split_workspace bytes), then an
+// ordered reduction.
+constexpr int64_t kSplitGatherMaxBags = 64;
+size_t embbag_split_workspace(int64_t n_bags, int B, int d);
+cudaError_t launch_embbag_fwd_split(const void* table, int64_t n_rows, int d, pkm_dtype dt,
+                                    const int32_t* idx, const float* w, int64_t n_bags, int B,
+                                    const void* gate, void* out, float* part, int32_t* status,
+                                    cudaStream_t stream);
+
 // Memory+ helpers (bf16).
 cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,
                                   cudaStream_t stream);

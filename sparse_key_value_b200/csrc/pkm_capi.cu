@@ -37,7 +37,7 @@ static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // ------------------------------------------------------------ forward ----
 
 struct FwdLayout {
-  size_t rq, rk, hv, hi, w1t, w2t, g, z, total;
+  size_t rq, rk, hv, hi, w1t, w2t, g, z, part, total;
   int splits;
   bool tc;
 };
@@ -68,6 +68,9 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
     L.g = take(T * dv * 2);
     L.z = take(T * dv * 2);
   }
+  // small batches gather through row-group partial sums
+  if ((int64_t)T <= kSplitGatherMaxBags)
+    L.part = take(embbag_split_workspace((int64_t)T, (int)(H * k), a->d_v));
   L.total = off;
   return L;
 }
@@ -151,8 +154,13 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
     PKM_TRY(launch_gemm_bf16(a->x, w1t, T, dv, dm, /*silu*/ 1, g, status, st));
   }
   mark(a, 4, st);
-  PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g,
-                            mp ? z : a->out, status, st));
+  if (T <= kSplitGatherMaxBags)
+    PKM_TRY(launch_embbag_fwd_split(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g,
+                                    mp ? z : a->out, reinterpret_cast<float*>(ws + L.part),
+                                    status, st));
+  else
+    PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g,
+                              mp ? z : a->out, status, st));
   mark(a, 5, st);
   if (mp) PKM_TRY(launch_gemm_bf16(z, w2t, T, dm, dv, /*none*/ 0, a->out, status, st));
   mark(a, 6, st);
