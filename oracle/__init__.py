@@ -69,10 +69,14 @@ def _load():
         lib.orc_pkm_backward.argtypes = [I64, I, I, I, I, I, P, I, P, I, P, I, I64,
                                          P, P, P, P, I, P, P, P, P, P]
         lib.orc_value_grad_rows.argtypes = [I64, I, I, I, P, P, P, I, P, I64, P]
+        lib.orc_memplus_backward.argtypes = [I64, I, I, P, P, I, P, I, P, I, P, I, P, P, P, P]
+        lib.orc_qproj.argtypes = [I64, I, I, P, I, P, I, P]
+        lib.orc_qproj_backward.argtypes = [I64, I, I, P, I, P, I, P, P, P]
         lib.orc_num_threads.argtypes = []
         for f in ("orc_half_scores", "orc_topk", "orc_pkm_select",
                   "orc_bruteforce_select", "orc_softmax", "orc_bag", "orc_memplus",
-                  "orc_pkm_backward", "orc_num_threads", "orc_value_grad_rows"):
+                  "orc_pkm_backward", "orc_num_threads", "orc_value_grad_rows",
+                  "orc_memplus_backward", "orc_qproj", "orc_qproj_backward"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -200,6 +204,54 @@ def memplus(y, x, W1, W2):
     _check(_load().orc_memplus(T, dm, dv, _p(y), _p(xa), xt, _p(w1), w1t, _p(w2), w2t,
                                _p(out)), "memplus")
     return out
+
+
+def memplus_backward(y, x, W1, W2, dout):
+    """Backward of out = (y ⊙ silu(x W1)) W2 ("Memory+ 블록").
+
+    Returns dict(dy [T,dv] (the gradient into the bag output), dx [T,dm],
+    dW1 [dm,dv], dW2 [dv,dm]).
+    """
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    xa, xt = _input(x)
+    w1, w1t = _input(W1)
+    w2, w2t = _input(W2)
+    da, dt = _input(dout)
+    T, dm = xa.shape
+    dv = w1.shape[1]
+    dy = np.empty((T, dv))
+    dx = np.empty((T, dm))
+    dW1 = np.empty((dm, dv))
+    dW2 = np.empty((dv, dm))
+    _check(_load().orc_memplus_backward(T, dm, dv, _p(y), _p(xa), xt, _p(w1), w1t, _p(w2), w2t,
+                                        _p(da), dt, _p(dy), _p(dx), _p(dW1), _p(dW2)),
+           "memplus_backward")
+    return dict(dy=dy, dx=dx, dW1=dW1, dW2=dW2)
+
+
+def qproj(x, Wq):
+    """q = x Wq: every head's and half's query from the layer input."""
+    xa, xt = _input(x)
+    wa, wt = _input(Wq)
+    T, dm = xa.shape
+    dq = wa.shape[1]
+    q = np.empty((T, dq))
+    _check(_load().orc_qproj(T, dm, dq, _p(xa), xt, _p(wa), wt, _p(q)), "qproj")
+    return q
+
+
+def qproj_backward(x, Wq, dq):
+    """Backward of q = x Wq: dict(dWq [dm,dq], dx [T,dm])."""
+    xa, xt = _input(x)
+    wa, wt = _input(Wq)
+    dq = np.ascontiguousarray(dq, dtype=np.float64)
+    T, dm = xa.shape
+    d_q = wa.shape[1]
+    dWq = np.empty((dm, d_q))
+    dx = np.empty((T, dm))
+    _check(_load().orc_qproj_backward(T, dm, d_q, _p(xa), xt, _p(wa), wt, _p(dq), _p(dWq),
+                                      _p(dx)), "qproj_backward")
+    return dict(dWq=dWq, dx=dx)
 
 
 def pkm_backward(q, K, table, idx, vrow, w, dy, want_dv: bool = True):

@@ -532,3 +532,109 @@ int orc_value_grad_rows(int64_t T, int H, int k, int dv, const int64_t *idx, con
     }
     return err;
 }
+
+/* ------------------------------------------------------------------ */
+/* Memory+ backward and the query projection                           */
+/* ------------------------------------------------------------------ */
+
+/*
+ * "Memory Layers at Scale" digest, "Memory+ 블록": out = (y ⊙ silu(x W1)) W2,
+ * in row-vector form per token t (a = x W1, g = silu(a), z = y ⊙ g).  Given
+ * the gradient dout of out:
+ *   dz      = dout W2^T
+ *   dy      = dz ⊙ g                      (into the lookup's backward)
+ *   da      = dz ⊙ y ⊙ silu'(a),  silu'(a) = s(a) (1 + a (1 - s(a))),  s = sigmoid
+ *   dx      = da W1^T
+ *   dW1     = sum_t x_t^T da_t,   dW2 = sum_t z_t^T dout_t
+ * y is given in double (the bag output); x, W1, W2, dout are decoded exactly.
+ */
+int orc_memplus_backward(int64_t T, int dm, int dv, const double *y, const void *x,
+                         int x_dtype, const void *W1, int w1_dtype, const void *W2,
+                         int w2_dtype, const void *dout, int dout_dtype, double *dy_out,
+                         double *dx_out, double *dW1_out, double *dW2_out) {
+    if (T < 0 || dm < 1 || dv < 1) return -2;
+    double *z = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * dv);
+    double *da = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * dv);
+    if (!z || !da) {
+        free(z);
+        free(da);
+        return -1;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; t++) {
+        for (int v = 0; v < dv; v++) {
+            double a = 0.0, dz = 0.0;
+            for (int m = 0; m < dm; m++) {
+                a += ld(x, x_dtype, t * dm + m) * ld(W1, w1_dtype, (int64_t)m * dv + v);
+                dz += ld(dout, dout_dtype, t * dm + m) * ld(W2, w2_dtype, (int64_t)v * dm + m);
+            }
+            const double s = 1.0 / (1.0 + exp(-a));
+            const double yv = y[t * dv + v];
+            z[t * dv + v] = yv * a * s;
+            dy_out[t * dv + v] = dz * a * s;
+            da[t * dv + v] = dz * yv * s * (1.0 + a * (1.0 - s));
+        }
+        for (int m = 0; m < dm; m++) {
+            double acc = 0.0;
+            for (int v = 0; v < dv; v++)
+                acc += da[t * dv + v] * ld(W1, w1_dtype, (int64_t)m * dv + v);
+            dx_out[t * dm + m] = acc;
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < dm; m++)
+        for (int v = 0; v < dv; v++) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; t++) acc += ld(x, x_dtype, t * dm + m) * da[t * dv + v];
+            dW1_out[(int64_t)m * dv + v] = acc;
+        }
+#pragma omp parallel for schedule(static)
+    for (int v = 0; v < dv; v++)
+        for (int m = 0; m < dm; m++) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; t++)
+                acc += z[t * dv + v] * ld(dout, dout_dtype, t * dm + m);
+            dW2_out[(int64_t)v * dm + m] = acc;
+        }
+    free(z);
+    free(da);
+    return 0;
+}
+
+/* q = x Wq ([T, dm] x [dm, dq]): the query of every head and half from the
+   layer input */
+int orc_qproj(int64_t T, int dm, int dq, const void *x, int x_dtype, const void *Wq,
+              int wq_dtype, double *q_out) {
+    if (T < 0 || dm < 1 || dq < 1) return -2;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; t++)
+        for (int j = 0; j < dq; j++) {
+            double acc = 0.0;
+            for (int m = 0; m < dm; m++)
+                acc += ld(x, x_dtype, t * dm + m) * ld(Wq, wq_dtype, (int64_t)m * dq + j);
+            q_out[t * dq + j] = acc;
+        }
+    return 0;
+}
+
+/* backward of q = x Wq: dWq = sum_t x_t^T dq_t, dx_t = dq_t Wq^T */
+int orc_qproj_backward(int64_t T, int dm, int dq, const void *x, int x_dtype, const void *Wq,
+                       int wq_dtype, const double *dqv, double *dWq_out, double *dx_out) {
+    if (T < 0 || dm < 1 || dq < 1) return -2;
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < dm; m++)
+        for (int j = 0; j < dq; j++) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; t++) acc += ld(x, x_dtype, t * dm + m) * dqv[t * dq + j];
+            dWq_out[(int64_t)m * dq + j] = acc;
+        }
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; t++)
+        for (int m = 0; m < dm; m++) {
+            double acc = 0.0;
+            for (int j = 0; j < dq; j++)
+                acc += dqv[t * dq + j] * ld(Wq, wq_dtype, (int64_t)m * dq + j);
+            dx_out[t * dm + m] = acc;
+        }
+    return 0;
+}

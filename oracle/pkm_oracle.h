@@ -62,6 +62,21 @@ int orc_pkm_backward(int64_t T, int H, int dh, int n, int k, int dv,
                      double *dq_out, double *dK_out, double *dv_out);
 
 /* dV rows for the requested row ids only: out [n_rows, dv] */
+/* Memory+ backward: given y [T,dv] (double), x [T,dm], W1 [dm,dv],
+   W2 [dv,dm] and dout [T,dm]: dy [T,dv], dx [T,dm], dW1 [dm,dv], dW2 [dv,dm] */
+int orc_memplus_backward(int64_t T, int dm, int dv, const double *y, const void *x,
+                         int x_dtype, const void *W1, int w1_dtype, const void *W2,
+                         int w2_dtype, const void *dout, int dout_dtype, double *dy_out,
+                         double *dx_out, double *dW1_out, double *dW2_out);
+
+/* query projection q = x Wq, x [T,dm], Wq [dm,dq], q [T,dq] */
+int orc_qproj(int64_t T, int dm, int dq, const void *x, int x_dtype, const void *Wq,
+              int wq_dtype, double *q_out);
+
+/* its backward: dWq [dm,dq] = x^T dq, dx [T,dm] = dq Wq^T (dq double) */
+int orc_qproj_backward(int64_t T, int dm, int dq, const void *x, int x_dtype, const void *Wq,
+                       int wq_dtype, const double *dqv, double *dWq_out, double *dx_out);
+
 int orc_value_grad_rows(int64_t T, int H, int k, int dv, const int64_t *idx, const double *w,
                         const void *dy, int dy_dtype, const int64_t *rows, int64_t n_rows,
                         double *out);

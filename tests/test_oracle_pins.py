@@ -350,3 +350,74 @@ def test_value_grad_rows_matches_backward(orc):
     rows = np.array(sorted(set(idx.ravel().tolist()))[::2] + [n * n - 1])
     got = orc.value_grad_rows(idx, w, dy, rows)
     np.testing.assert_allclose(got, full["dV"][rows], rtol=1e-13, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# Memory+ backward and the query projection
+# --------------------------------------------------------------------------
+
+def _memplus_inputs(seed, T=6, dm=5, dv=7):
+    rng = np.random.default_rng(seed)
+    return (rng.normal(size=(T, dv)), rng.normal(size=(T, dm)), rng.normal(size=(dm, dv)),
+            rng.normal(size=(dv, dm)), rng.normal(size=(T, dm)))
+
+
+def test_memplus_backward_matches_autograd(orc):
+    """dy, dx, dW1, dW2 equal torch autograd (fp64) of <dout, (y ⊙ silu(x W1)) W2>;
+    x, W1 and W2 travel as bf16 (exact decoding)."""
+    y, x, W1, W2, dout = _memplus_inputs(21)
+    xb, W1b, W2b = (torch.from_numpy(a).to(torch.bfloat16) for a in (x, W1, W2))
+    r = orc.memplus_backward(y, xb, W1b, W2b, dout)
+    yt = torch.tensor(y, requires_grad=True)
+    xt, W1t, W2t = (a.double().requires_grad_(True) for a in (xb, W1b, W2b))
+    out = (yt * torch.nn.functional.silu(xt @ W1t)) @ W2t
+    (out * torch.from_numpy(dout)).sum().backward()
+    for key, t in (("dy", yt), ("dx", xt), ("dW1", W1t), ("dW2", W2t)):
+        np.testing.assert_allclose(r[key], t.grad.numpy(), rtol=1e-12, atol=1e-12, err_msg=key)
+
+
+def test_memplus_backward_finite_differences(orc):
+    """Central differences of <dout, memplus(y, x, W1, W2)> (the oracle's own
+    forward, pinned above) on every entry of small inputs."""
+    y, x, W1, W2, dout = _memplus_inputs(22, T=3, dm=4, dv=3)
+    r = orc.memplus_backward(y, x, W1, W2, dout)
+    h = 1e-6
+
+    def f(y_, x_, W1_, W2_):
+        return float(np.sum(orc.memplus(y_, x_, W1_, W2_) * dout))
+
+    args = [y, x, W1, W2]
+    for pos, key in ((0, "dy"), (1, "dx"), (2, "dW1"), (3, "dW2")):
+        num = np.empty_like(args[pos])
+        for i in np.ndindex(args[pos].shape):
+            up = [a.copy() for a in args]
+            dn = [a.copy() for a in args]
+            up[pos][i] += h
+            dn[pos][i] -= h
+            num[i] = (f(*up) - f(*dn)) / (2 * h)
+        np.testing.assert_allclose(r[key], num, rtol=1e-6, atol=1e-7, err_msg=key)
+
+
+def test_memplus_backward_zero_gate(orc):
+    """W1 = 0: a = 0, silu(0) = 0, silu'(0) = 1/2, so dy = 0, dW2 = 0 and
+    da = (dout W2^T) ⊙ y / 2 (dW1 = x^T da, dx = da W1^T = 0)."""
+    y, x, _, W2, dout = _memplus_inputs(23)
+    W1 = np.zeros((x.shape[1], y.shape[1]))
+    r = orc.memplus_backward(y, x, W1, W2, dout)
+    assert np.all(r["dy"] == 0.0) and np.all(r["dW2"] == 0.0) and np.all(r["dx"] == 0.0)
+    da = (dout @ W2.T) * y * 0.5
+    np.testing.assert_allclose(r["dW1"], x.T @ da, rtol=1e-13, atol=1e-14)
+
+
+def test_qproj_and_backward(orc):
+    """q = x Wq is numpy's matmul; its backward equals autograd (bf16 inputs)."""
+    rng = np.random.default_rng(24)
+    x, Wq, dq = rng.normal(size=(5, 6)), rng.normal(size=(6, 8)), rng.normal(size=(5, 8))
+    xb, Wqb = torch.from_numpy(x).to(torch.bfloat16), torch.from_numpy(Wq).to(torch.bfloat16)
+    q = orc.qproj(xb, Wqb)
+    np.testing.assert_allclose(q, xb.double().numpy() @ Wqb.double().numpy(), rtol=1e-13)
+    xt, Wt = xb.double().requires_grad_(True), Wqb.double().requires_grad_(True)
+    ((xt @ Wt) * torch.from_numpy(dq)).sum().backward()
+    r = orc.qproj_backward(xb, Wqb, dq)
+    np.testing.assert_allclose(r["dWq"], Wt.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(r["dx"], xt.grad.numpy(), rtol=1e-12, atol=1e-13)
