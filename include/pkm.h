@@ -110,6 +110,11 @@ typedef struct {
        Memory+ gate GEMM), [5] after the bag gather, [6] end (after the
        Memory+ output GEMM). */
     void **phase_events;
+    /* Optional, Memory+ only: NULL, or [T, d_v] (dtype) receiving the bag
+       output y before the gate, as pkm_memplus_backward needs it.  With it
+       the gate product is applied in a separate pass (y rounded to the
+       dtype first), otherwise fused into the gather. */
+    void *y_out;
 } pkm_fwd_args;
 
 #define PKM_FWD_N_EVENTS 7
@@ -224,6 +229,71 @@ PKM_API int32_t pkm_version(void);
 /* Instrumentation: number of kernels this process has launched through the
    library so far (host-side counter, all devices). */
 PKM_API uint64_t pkm_launch_count(void);
+
+/*
+ * Memory+ backward ("Memory Layers at Scale" digest, "Memory+ 블록": out =
+ * (y ⊙ silu(x W1)) W2).  Row-vector form per token, a = x W1, g = silu(a):
+ *   dz  = dout W2^T,          dy  = dz ⊙ g   (the lookup's upstream gradient)
+ *   da  = dz ⊙ y ⊙ silu'(a),  dx  = da W1^T
+ *   dW1 = x^T da,             dW2 = (y ⊙ g)^T dout
+ * No counterpart in the sources beyond the forward they give; the formulas
+ * are its derivatives.  All of x, W1, W2, y, dout are bf16.
+ *
+ *   x [T, d_model], W1 [d_model, d_v], W2 [d_v, d_model]  the forward's inputs
+ *   y    [T, d_v]      the bag output (pkm_fwd_args.y_out of the forward)
+ *   dout [T, d_model]  gradient of out
+ *   dy   [T, d_v]      out (bf16): gradient of y, the dy of pkm_backward
+ *   dx   [T, d_model]  out (fp32), overwritten
+ *   dW1  [d_model, d_v], dW2 [d_v, d_model]  out (fp32)
+ * Limits: d_model, d_v multiples of 8.  T = 0 is a valid empty call (the
+ * weight gradients are then zero).
+ */
+typedef struct {
+    int64_t T;
+    int32_t d_model, d_v;
+    const void *x;
+    const void *W1;
+    const void *W2;
+    const void *y;
+    const void *dout;
+    void *dy;
+    float *dx;
+    float *dW1;
+    float *dW2;
+    void *workspace; /* device scratch of pkm_memplus_backward_workspace_size bytes */
+    size_t workspace_bytes;
+} pkm_memplus_bwd_args;
+
+PKM_API size_t pkm_memplus_backward_workspace_size(const pkm_memplus_bwd_args *args);
+PKM_API pkm_status pkm_memplus_backward(const pkm_memplus_bwd_args *args, pkm_stream_t stream);
+
+/*
+ * Query projection q = x Wq that feeds the lookup from the layer input
+ * (the query of every head and half, d_q = H * 2 * d_half), and its
+ * backward.  bf16 x [T, d_model], Wq [d_model, d_q].
+ *   pkm_qproj_forward:  q [T, d_q] (bf16) out.
+ *   pkm_qproj_backward: dq [T, d_q] (fp32, pkm_bwd_args.dquery) in;
+ *                       dWq [d_model, d_q] (fp32) out; dx [T, d_model]
+ *                       (fp32) += dq Wq^T (accumulates onto, e.g., the dx of
+ *                       pkm_memplus_backward).
+ * Limits: d_model, d_q multiples of 8.
+ */
+typedef struct {
+    int64_t T;
+    int32_t d_model, d_q;
+    const void *x;
+    const void *Wq;
+    void *q;
+    const float *dq;
+    float *dWq;
+    float *dx;
+    void *workspace; /* device scratch of pkm_qproj_workspace_size bytes */
+    size_t workspace_bytes;
+} pkm_qproj_args;
+
+PKM_API size_t pkm_qproj_workspace_size(const pkm_qproj_args *args);
+PKM_API pkm_status pkm_qproj_forward(const pkm_qproj_args *args, pkm_stream_t stream);
+PKM_API pkm_status pkm_qproj_backward(const pkm_qproj_args *args, pkm_stream_t stream);
 
 #ifdef __cplusplus
 }

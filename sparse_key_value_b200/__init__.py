@@ -66,13 +66,15 @@ def forward_workspace_size(T, H, d_half, n_sub, k, d_v, dtype=PKM_BF16, memplus=
 
 
 def pkm_forward(query, subkeys, values, k: int, x=None, W1=None, W2=None, out=None, idx=None,
-                weights=None, workspace=None, stream=None, phase_events=None):
+                weights=None, workspace=None, stream=None, phase_events=None, y_out=None):
     """Forward of one memory layer (see pkm_forward in include/pkm.h).
 
     query [T,H,2,d_half], subkeys [H,2,n_sub,d_half], values [n_sub^2, d_v];
     optional Memory+ gate x [T,d_model], W1 [d_model,d_v], W2 [d_v,d_model].
     ``phase_events``: optional list of 7 torch.cuda.Event recorded at the
     phase boundaries (see pkm_fwd_args.phase_events).
+    ``y_out``: Memory+ only, a [T, d_v] tensor receiving the bag output
+    before the gate (what memplus_backward needs).
     Returns (out, idx, weights)."""
     _need_cuda(query, subkeys, values, x, W1, W2)
     T, H, two, dh = query.shape
@@ -95,6 +97,7 @@ def pkm_forward(query, subkeys, values, k: int, x=None, W1=None, W2=None, out=No
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     a.workspace, a.workspace_bytes = _p(workspace), workspace.numel()
+    a.y_out = _p(y_out)
     if phase_events is not None:
         if len(phase_events) != 7 or any(e.cuda_event == 0 for e in phase_events):
             raise ValueError("phase_events: 7 events, each recorded once before use")
@@ -206,3 +209,66 @@ def device_error(stream=None, device=None) -> int:
     check(load().pkm_get_device_error(_stream(dev, stream), ctypes.byref(code)),
           "pkm_get_device_error")
     return int(code.value)
+
+
+def memplus_backward(x, W1, W2, y, dout, workspace=None, stream=None):
+    """Backward of the Memory+ block (see pkm_memplus_backward in include/pkm.h).
+
+    x [T,d_model], W1 [d_model,d_v], W2 [d_v,d_model], y [T,d_v] (the
+    forward's y_out), dout [T,d_model], all bf16.  Returns dict(dy (bf16,
+    the dy of pkm_backward), dx, dW1, dW2 (fp32))."""
+    _need_cuda(x, W1, W2, y, dout)
+    T, dm = x.shape
+    dv = W1.shape[1]
+    dev = x.device
+    dy = torch.empty(T, dv, dtype=x.dtype, device=dev)
+    dx = torch.empty(T, dm, dtype=torch.float32, device=dev)
+    dW1 = torch.empty(dm, dv, dtype=torch.float32, device=dev)
+    dW2 = torch.empty(dv, dm, dtype=torch.float32, device=dev)
+    a = _lib.MemplusBwdArgs(T, dm, dv, _p(x), _p(W1), _p(W2), _p(y), _p(dout), _p(dy), _p(dx),
+                            _p(dW1), _p(dW2), None, 0)
+    lib = load()
+    need = int(lib.pkm_memplus_backward_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    a.workspace, a.workspace_bytes = _p(workspace), workspace.numel()
+    check(lib.pkm_memplus_backward(ctypes.byref(a), _stream(dev, stream)), "pkm_memplus_backward")
+    return dict(dy=dy, dx=dx, dW1=dW1, dW2=dW2)
+
+
+def _qproj_args(x, Wq, q=None, dq=None, dWq=None, dx=None) -> "_lib.QprojArgs":
+    T, dm = x.shape
+    return _lib.QprojArgs(T, dm, Wq.shape[1], _p(x), _p(Wq), _p(q), _p(dq), _p(dWq), _p(dx),
+                          None, 0)
+
+
+def _qproj_call(fn: str, a, dev, workspace, stream):
+    lib = load()
+    need = int(lib.pkm_qproj_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    a.workspace, a.workspace_bytes = _p(workspace), workspace.numel()
+    check(getattr(lib, fn)(ctypes.byref(a), _stream(dev, stream)), fn)
+
+
+def qproj_forward(x, Wq, out=None, workspace=None, stream=None):
+    """q = x Wq (bf16 [T, d_q]; see pkm_qproj_forward in include/pkm.h)."""
+    _need_cuda(x, Wq)
+    if out is None:
+        out = torch.empty(x.shape[0], Wq.shape[1], dtype=x.dtype, device=x.device)
+    _qproj_call("pkm_qproj_forward", _qproj_args(x, Wq, q=out), x.device, workspace, stream)
+    return out
+
+
+def qproj_backward(x, Wq, dq, dx=None, workspace=None, stream=None):
+    """dWq = x^T dq and dx += dq Wq^T (dq fp32 [T, d_q]; dx fp32 [T, d_model],
+    zero-initialised when not given).  Returns dict(dWq, dx)."""
+    _need_cuda(x, Wq, dq)
+    dev = x.device
+    if dx is None:
+        dx = torch.zeros(x.shape[0], x.shape[1], dtype=torch.float32, device=dev)
+    dWq = torch.empty(x.shape[1], Wq.shape[1], dtype=torch.float32, device=dev)
+    dq = dq.reshape(x.shape[0], Wq.shape[1]).contiguous()
+    _qproj_call("pkm_qproj_backward", _qproj_args(x, Wq, dq=dq, dWq=dWq, dx=dx), dev, workspace,
+                stream)
+    return dict(dWq=dWq, dx=dx)

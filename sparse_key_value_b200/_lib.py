@@ -33,7 +33,7 @@ class FwdArgs(ctypes.Structure):
                 ("d_v", I32), ("dtype", ctypes.c_int), ("query", P), ("subkeys", P),
                 ("values", P), ("x", P), ("W1", P), ("W2", P), ("d_model", I32), ("out", P),
                 ("idx", P), ("weights", P), ("workspace", P), ("workspace_bytes", SZ),
-                ("phase_events", P)]
+                ("phase_events", P), ("y_out", P)]
 
 
 FWD_N_EVENTS = 7
@@ -48,10 +48,23 @@ class BwdArgs(ctypes.Structure):
                 ("workspace_bytes", SZ)]
 
 
+class MemplusBwdArgs(ctypes.Structure):
+    _fields_ = [("T", I64), ("d_model", I32), ("d_v", I32), ("x", P), ("W1", P), ("W2", P),
+                ("y", P), ("dout", P), ("dy", P), ("dx", P), ("dW1", P), ("dW2", P),
+                ("workspace", P), ("workspace_bytes", SZ)]
+
+
+class QprojArgs(ctypes.Structure):
+    _fields_ = [("T", I64), ("d_model", I32), ("d_q", I32), ("x", P), ("Wq", P), ("q", P),
+                ("dq", P), ("dWq", P), ("dx", P), ("workspace", P), ("workspace_bytes", SZ)]
+
+
 EXPORTS = ("pkm_forward_workspace_size", "pkm_forward", "pkm_backward_workspace_size",
            "pkm_backward", "embbag_forward", "embbag_backward_workspace_size",
            "embbag_backward", "pkm_get_device_error", "pkm_status_string", "pkm_version",
-           "pkm_launch_count", "pkm_forward_noalloc")
+           "pkm_launch_count", "pkm_forward_noalloc", "pkm_memplus_backward_workspace_size",
+           "pkm_memplus_backward", "pkm_qproj_workspace_size", "pkm_qproj_forward",
+           "pkm_qproj_backward")
 
 _lib = None
 
@@ -90,6 +103,17 @@ def load(path: str = LIB_PATH):
     lib.pkm_forward_noalloc.restype = ctypes.c_int
     lib.pkm_launch_count.argtypes = []
     lib.pkm_launch_count.restype = ctypes.c_uint64
+    MA, QA = ctypes.POINTER(MemplusBwdArgs), ctypes.POINTER(QprojArgs)
+    lib.pkm_memplus_backward_workspace_size.argtypes = [MA]
+    lib.pkm_memplus_backward_workspace_size.restype = SZ
+    lib.pkm_memplus_backward.argtypes = [MA, P]
+    lib.pkm_memplus_backward.restype = ctypes.c_int
+    lib.pkm_qproj_workspace_size.argtypes = [QA]
+    lib.pkm_qproj_workspace_size.restype = SZ
+    lib.pkm_qproj_forward.argtypes = [QA, P]
+    lib.pkm_qproj_forward.restype = ctypes.c_int
+    lib.pkm_qproj_backward.argtypes = [QA, P]
+    lib.pkm_qproj_backward.restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
     return lib

@@ -12,12 +12,14 @@
 
 namespace pkm {
 
-// dst[c][r] = src[r][c] for a rows x cols bf16 matrix.  64 x 64 tiles: rows
+// dst[c][r] = src[r][c] for a rows x cols bf16 matrix, dst rows ld long
+// (ld >= rows; entries rows..ld-1 are written as zeros).  64 x 64 tiles: rows
 // are read and written as 16-byte vectors (coalesced 128-byte segments), the
 // transpose itself happens element-wise in shared memory.
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src,
                                                              int rows, int cols,
-                                                             __nv_bfloat16* __restrict__ dst) {
+                                                             __nv_bfloat16* __restrict__ dst,
+                                                             int ld) {
   __shared__ uint16_t tile[64][65];
   const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
   const int tid = threadIdx.x;
@@ -46,7 +48,7 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16
     for (int e = 0; e < 8; ++e) tile[i][8 * q + e] = v[e];
   }
   __syncthreads();
-  const bool vec_dst = (rows % 8) == 0;
+  const bool vec_dst = (ld % 8) == 0;
   uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -57,23 +59,25 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16
     uint16_t v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) v[e] = tile[8 * q + e][j];
-    uint16_t* d = d16 + (int64_t)c * rows + r;
-    if (vec_dst && r + 8 <= rows) {
+    uint16_t* d = d16 + (int64_t)c * ld + r;
+    if (vec_dst && r + 8 <= ld) {
       *reinterpret_cast<uint4*>(d) =
           make_uint4(v[0] | ((uint32_t)v[1] << 16), v[2] | ((uint32_t)v[3] << 16),
                      v[4] | ((uint32_t)v[5] << 16), v[6] | ((uint32_t)v[7] << 16));
     } else {
-      for (int e = 0; e < 8 && r + e < rows; ++e) d[e] = v[e];
+      for (int e = 0; e < 8 && r + e < ld; ++e) d[e] = v[e];
     }
   }
 }
 
 cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,
-                                  cudaStream_t stream) {
-  if (rows <= 0 || cols <= 0) return cudaSuccess;
-  dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+                                  cudaStream_t stream, int ld) {
+  if (ld <= 0) ld = rows;
+  if (rows <= 0 || cols <= 0 || ld < rows) return rows <= 0 || cols <= 0 ? cudaSuccess
+                                                                          : cudaErrorInvalidValue;
+  dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((ld + 63) / 64));
   transpose_bf16_kernel<<<grid, 256, 0, stream>>>((const __nv_bfloat16*)src, rows, cols,
-                                                  (__nv_bfloat16*)dst);
+                                                  (__nv_bfloat16*)dst, ld);
   note_launch();
   return cudaGetLastError();
 }
@@ -81,10 +85,11 @@ cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
 // C[M,N] = epi(sum_k A[m,k] B[n,k]); 64x64 tile, 256 threads, 4x4 each.
+// out_mode: 0 bf16 (epi applied), 1 fp32, 2 fp32 accumulate.
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const __nv_bfloat16* __restrict__ A,
                                                         const __nv_bfloat16* __restrict__ B,
                                                         int64_t M, int N, int K, int epi,
-                                                        __nv_bfloat16* __restrict__ C) {
+                                                        int out_mode, void* __restrict__ Cv) {
   __shared__ float As[16][64 + 1];
   __shared__ float Bs[16][64 + 1];
   const int64_t m0 = (int64_t)blockIdx.y * 64;
@@ -123,29 +128,43 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const __nv_bfloat16* __r
       int nn = n0 + tx * 4 + j;
       if (nn >= N) continue;
       float v = acc[i][j];
-      if (epi == 1) v = silu_f(v);
-      C[m * N + nn] = __float2bfloat16_rn(v);
+      if (out_mode == 0) {
+        if (epi == 1) v = silu_f(v);
+        static_cast<__nv_bfloat16*>(Cv)[m * N + nn] = __float2bfloat16_rn(v);
+      } else {
+        float* c = static_cast<float*>(Cv) + m * N + nn;
+        *c = out_mode == 2 ? *c + v : v;
+      }
     }
   }
 }
 
 cudaError_t launch_gemm_simt(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                             void* C, cudaStream_t stream) {
+                             int out_mode, void* C, cudaStream_t stream) {
   dim3 grid((N + 63) / 64, (unsigned)((M + 63) / 64));
   gemm_simt_kernel<<<grid, 256, 0, stream>>>((const __nv_bfloat16*)A, (const __nv_bfloat16*)B,
-                                             M, N, K, epi, (__nv_bfloat16*)C);
+                                             M, N, K, epi, out_mode, C);
   note_launch();
   return cudaGetLastError();
 }
-
 cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                           void* C, int32_t* status, cudaStream_t stream);
+                           int out_mode, void* C, int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
                              void* C, int32_t* status, cudaStream_t stream) {
   if (M <= 0) return cudaSuccess;
-  if (gemm_tc_supported(M, N, K)) return launch_gemm_tc(A, B, M, N, K, epi, C, status, stream);
-  return launch_gemm_simt(A, B, M, N, K, epi, C, stream);
+  if (gemm_tc_supported(M, N, K))
+    return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream);
+  return launch_gemm_simt(A, B, M, N, K, epi, 0, C, stream);
+}
+
+cudaError_t launch_gemm_f32(const void* A, const void* B, int64_t M, int N, int K,
+                            bool accumulate, float* C, int32_t* status, cudaStream_t stream) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  const int mode = accumulate ? 2 : 1;
+  if (gemm_tc_supported(M, N, K))
+    return launch_gemm_tc(A, B, M, N, K, 0, mode, C, status, stream);
+  return launch_gemm_simt(A, B, M, N, K, 0, mode, C, stream);
 }
 
 }  // namespace pkm

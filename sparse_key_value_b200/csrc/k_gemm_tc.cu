@@ -1,8 +1,9 @@
 // k_gemm_tc.cu -- the dense GEMMs of the Memory+ block on the tensor cores
 // ("Memory Layers at Scale" digest, "Memory+ 블록": out = (y ⊙ silu(x W1)) W2).
 //
-//   C[M, N] = epi(A[M, K] * B[N, K]^T),  A, B bf16 K-major, C bf16 row-major,
-//   epi = silu (gate) or identity (output projection), fp32 accumulation.
+//   C[M, N] = epi(A[M, K] * B[N, K]^T),  A, B bf16 K-major, C row-major,
+//   epi = silu (gate) or identity, fp32 accumulation; C is bf16 (rounded to
+//   nearest even), fp32, or fp32 accumulated into (C += A B^T).
 //
 // One CTA per 128 x 256 output tile:
 //   warp 0     TMA producer: 64-wide k-blocks of A [128 x 64] and B [256 x 64]
@@ -49,10 +50,11 @@ __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, GemmCt
   return false;
 }
 
-template <int EPI>
+// OUT: 0 bf16 store, 1 fp32 store, 2 fp32 accumulate (C += result)
+template <int EPI, int OUT>
 __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t M,
-    int N, int K, __nv_bfloat16* __restrict__ C, int32_t* status) {
+    int N, int K, void* __restrict__ Cv, int32_t* status) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* stages = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -142,7 +144,25 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + g * 32, r);
         tmem_ld_wait();
-        if (m < M) {
+        if (m < M && OUT != 0) {
+          float* dst = static_cast<float*>(Cv) + m * N + col0;
+          const int nq = col0 + 32 <= N ? 8 : (N - col0) / 4;  // N % 8 == 0
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (j < nq) {
+              float4 v = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                     __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+              if (OUT == 2) {
+                const float4 o = reinterpret_cast<const float4*>(dst)[j];
+                v.x += o.x;
+                v.y += o.y;
+                v.z += o.z;
+                v.w += o.w;
+              }
+              reinterpret_cast<float4*>(dst)[j] = v;
+            }
+          }
+        } else if (m < M) {
           uint32_t packed[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -156,7 +176,7 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
             }
             packed[j] = pack_bf16x2(a, b);
           }
-          __nv_bfloat16* dst = C + m * N + col0;
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(Cv) + m * N + col0;
           if (col0 + 32 <= N) {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -183,8 +203,9 @@ bool gemm_tc_supported(int64_t M, int N, int K) {
   return M >= 1 && N >= 16 && K >= gm::kKB && N % 8 == 0 && K % 8 == 0;
 }
 
+// out_mode: 0 bf16 (epi applied), 1 fp32, 2 fp32 accumulate; epi only with bf16 output.
 cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                           void* C, int32_t* status, cudaStream_t stream) {
+                           int out_mode, void* C, int32_t* status, cudaStream_t stream) {
   if (M <= 0) return cudaSuccess;
   CUtensorMap tmA, tmB;
   {
@@ -201,19 +222,22 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K
   }
   dim3 grid((unsigned)((M + gm::kM - 1) / gm::kM), (unsigned)((N + gm::kN - 1) / gm::kN));
   cudaError_t e;
-  if (epi == 1) {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)gm::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    gemm_tc_kernel<1><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(
-        tmA, tmB, M, N, K, (__nv_bfloat16*)C, status);
+#define PKM_GEMM_TC(E_, O_)                                                                  \
+  e = cudaFuncSetAttribute(gemm_tc_kernel<E_, O_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           (int)gm::kSmemBytes);                                             \
+  if (e != cudaSuccess) return e;                                                            \
+  gemm_tc_kernel<E_, O_><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(tmA, tmB, M, N, K, C, \
+                                                                        status)
+  if (out_mode == 1) {
+    PKM_GEMM_TC(0, 1);
+  } else if (out_mode == 2) {
+    PKM_GEMM_TC(0, 2);
+  } else if (epi == 1) {
+    PKM_GEMM_TC(1, 0);
   } else {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)gm::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    gemm_tc_kernel<0><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(
-        tmA, tmB, M, N, K, (__nv_bfloat16*)C, status);
+    PKM_GEMM_TC(0, 0);
   }
+#undef PKM_GEMM_TC
   note_launch();
   return cudaGetLastError();
 }

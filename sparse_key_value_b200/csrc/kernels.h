@@ -63,13 +63,20 @@ cudaError_t launch_embbag_fwd_split(const void* table, int64_t n_rows, int d, pk
                                     cudaStream_t stream);
 
 // Memory+ helpers (bf16).
+// z = y ⊙ g elementwise (bf16, one rounding)
+cudaError_t launch_gate_mul_bf16(const void* y, const void* g, int64_t n, void* z,
+                                 cudaStream_t stream);
+// dst[c][r] = src[r][c]; dst rows are ld >= rows long, zero past rows (ld <= 0: ld = rows).
 cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, int ld = 0);
 // C[M,N] = epi(A[M,K] * B[N,K]^T), A/B bf16 K-major; epi: 0 none, 1 silu.
 // Optional `mul` [M,N] bf16 multiplies the result after the epilogue.
 bool gemm_tc_supported(int64_t M, int N, int K);
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
                              void* C, int32_t* status, cudaStream_t stream);
+// C[M,N] (fp32) = A[M,K] B[N,K]^T, or C += it when accumulate.
+cudaError_t launch_gemm_f32(const void* A, const void* B, int64_t M, int N, int K,
+                            bool accumulate, float* C, int32_t* status, cudaStream_t stream);
 
 // ---------------------------------------------------------------- backward
 // dw[t,j] = <dy[t], table[idx[t,j]]>; with H>0 also dS = w (dw - sum w dw)

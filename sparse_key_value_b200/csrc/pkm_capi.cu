@@ -88,6 +88,7 @@ static pkm_status validate_fwd(const pkm_fwd_args* a) {
   const void* need[] = {a->query, a->subkeys, a->values, a->out, a->idx, a->weights};
   for (const void* p : need)
     if (!p || !aligned16(p)) return PKM_ERR_INVALID_ARG;
+  if (a->y_out && (!has_memplus(a) || !aligned16(a->y_out))) return PKM_ERR_INVALID_ARG;
   if (has_memplus(a)) {
     if (!a->x || !a->W1 || !a->W2) return PKM_ERR_INVALID_ARG;
     if (!aligned16(a->x) || !aligned16(a->W1) || !aligned16(a->W2)) return PKM_ERR_INVALID_ARG;
@@ -154,13 +155,17 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
     PKM_TRY(launch_gemm_bf16(a->x, w1t, T, dv, dm, /*silu*/ 1, g, status, st));
   }
   mark(a, 4, st);
+  // with y_out the bag output is kept and the gate applied in a second pass
+  const void* gate = a->y_out ? nullptr : g;
+  void* bag_out = a->y_out ? a->y_out : (mp ? z : a->out);
   if (T <= kSplitGatherMaxBags)
-    PKM_TRY(launch_embbag_fwd_split(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g,
-                                    mp ? z : a->out, reinterpret_cast<float*>(ws + L.part),
+    PKM_TRY(launch_embbag_fwd_split(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k,
+                                    gate, bag_out, reinterpret_cast<float*>(ws + L.part),
                                     status, st));
   else
-    PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, g,
-                              mp ? z : a->out, status, st));
+    PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, gate,
+                              bag_out, status, st));
+  if (a->y_out) PKM_TRY(launch_gate_mul_bf16(a->y_out, g, T * dv, z, st));
   mark(a, 5, st);
   if (mp) PKM_TRY(launch_gemm_bf16(z, w2t, T, dm, dv, /*none*/ 0, a->out, status, st));
   mark(a, 6, st);

@@ -115,3 +115,47 @@ def test_embbag_rejects_bad_args(lib):
     assert lib.embbag_forward(f, 10, 16, 1, f, f, 4, 0, None, f, None) == 1   # B = 0
     assert lib.embbag_forward(None, 10, 16, 1, f, f, 4, 3, None, f, None) == 1
     assert lib.embbag_forward(f, 10, 16, 1, f, f, 0, 3, None, f, None) == 0   # no bags
+
+
+def test_y_out_requires_memplus_and_alignment(lib):
+    a = _fwd()
+    a.workspace_bytes = 1 << 40
+    a.y_out = ctypes.c_void_p(1 << 20)
+    assert lib.pkm_forward(ctypes.byref(a), None) == 1  # plain lookup: no gate, no y_out
+
+
+def _mp(**kw):
+    from sparse_key_value_b200 import _lib
+    fake = ctypes.c_void_p(1 << 20)
+    base = dict(T=64, d_model=64, d_v=32)
+    base.update(kw)
+    return _lib.MemplusBwdArgs(base["T"], base["d_model"], base["d_v"], fake, fake, fake, fake,
+                               fake, fake, fake, fake, fake, fake, 1 << 40)
+
+
+def test_memplus_backward_validation(lib):
+    assert lib.pkm_memplus_backward(ctypes.byref(_mp(d_model=60)), None) == 1
+    assert lib.pkm_memplus_backward(ctypes.byref(_mp(d_v=0)), None) == 1
+    a = _mp()
+    a.dout = None
+    assert lib.pkm_memplus_backward(ctypes.byref(a), None) == 1
+    a = _mp()
+    a.dW1 = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.pkm_memplus_backward(ctypes.byref(a), None) == 1
+    a = _mp()
+    need = lib.pkm_memplus_backward_workspace_size(ctypes.byref(a))
+    a.workspace_bytes = need - 1
+    assert lib.pkm_memplus_backward(ctypes.byref(a), None) == 6
+
+
+def test_qproj_validation(lib):
+    from sparse_key_value_b200 import _lib
+    fake = ctypes.c_void_p(1 << 20)
+    a = _lib.QprojArgs(64, 64, 12, fake, fake, fake, fake, fake, fake, fake, 1 << 40)
+    assert lib.pkm_qproj_forward(ctypes.byref(a), None) == 1  # d_q % 8 != 0
+    a = _lib.QprojArgs(64, 64, 16, fake, fake, None, fake, fake, fake, fake, 1 << 40)
+    assert lib.pkm_qproj_forward(ctypes.byref(a), None) == 1  # no q
+    a = _lib.QprojArgs(64, 64, 16, fake, fake, fake, None, fake, fake, fake, 1 << 40)
+    assert lib.pkm_qproj_backward(ctypes.byref(a), None) == 1  # no dq
+    a = _lib.QprojArgs(64, 64, 16, fake, fake, fake, fake, fake, fake, fake, 16)
+    assert lib.pkm_qproj_forward(ctypes.byref(a), None) == 6
