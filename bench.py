@@ -44,7 +44,7 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default="pkm",
-                   choices=["pkm", "memplus", "tiny", "decode", "train"])
+                   choices=["pkm", "memplus", "tiny", "decode", "train", "memplus_train"])
     p.add_argument("--graph", action="store_true",
                    help="capture one step in a CUDA graph and replay it (default for decode)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -231,6 +231,23 @@ def run_ours(args, rank, world, local):
     lib = skv.load()
 
     train = w.train
+    mp_train = train and mp
+    if mp_train:
+        # Memory+ training: the forward keeps the bag output y; the Memory+
+        # backward turns the layer-output gradient into the lookup's dy
+        yb = torch.empty(T, w.d_v, dtype=w.torch_dtype, device="cuda")
+        dyv = torch.empty(T, w.d_v, dtype=w.torch_dtype, device="cuda")
+        mdx = torch.empty(T, w.d_model, dtype=torch.float32, device="cuda")
+        mdW1 = torch.empty(w.d_model, w.d_v, dtype=torch.float32, device="cuda")
+        mdW2 = torch.empty(w.d_v, w.d_model, dtype=torch.float32, device="cuda")
+        margs = skv._lib.MemplusBwdArgs(T, w.d_model, w.d_v, skv._p(inp["x"]), skv._p(inp["W1"]),
+                                        skv._p(inp["W2"]), skv._p(yb), skv._p(inp["dy"]),
+                                        skv._p(dyv), skv._p(mdx), skv._p(mdW1), skv._p(mdW2),
+                                        None, 0)
+        mws = torch.empty(max(16, lib.pkm_memplus_backward_workspace_size(
+            skv.ctypes.byref(margs))), dtype=torch.uint8, device="cuda")
+        margs.workspace, margs.workspace_bytes = skv._p(mws), mws.numel()
+        kw["y_out"] = yb
     if train:
         R = T * w.H * w.k
         dq = torch.empty(T, w.H, 2, w.d_half, dtype=torch.float32, device="cuda")
@@ -238,7 +255,8 @@ def run_ours(args, rank, world, local):
         uniq = torch.empty(R, dtype=torch.int32, device="cuda")
         grad = torch.empty(R, w.d_v, dtype=torch.float32, device="cuda")
         n_uniq = torch.zeros(1, dtype=torch.int64, device="cuda")
-        bargs = skv._bwd_args(inp["query"], inp["subkeys"], inp["values"], idx, wts, inp["dy"],
+        bargs = skv._bwd_args(inp["query"], inp["subkeys"], inp["values"], idx, wts,
+                              dyv if mp_train else inp["dy"],
                               dquery=skv._p(dq), dsubkeys=skv._p(dK), uniq_rows=skv._p(uniq),
                               grad_rows=skv._p(grad), n_uniq=skv._p(n_uniq), uniq_cap=R)
         bws = torch.empty(max(16, lib.pkm_backward_workspace_size(skv.ctypes.byref(bargs))),
@@ -252,6 +270,11 @@ def run_ours(args, rank, world, local):
         if train:
             if bev is not None:
                 bev[0].record()
+            if mp_train:
+                skv.check(lib.pkm_memplus_backward(skv.ctypes.byref(margs), sptr),
+                          "pkm_memplus_backward")
+            if bev is not None:
+                bev[2].record()
             skv.check(lib.pkm_backward(skv.ctypes.byref(bargs), sptr), "pkm_backward")
             if bev is not None:
                 bev[1].record()
@@ -274,7 +297,7 @@ def run_ours(args, rank, world, local):
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
-    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     for e in sum(ev, []) + sum(bev, []):
         e.record()  # creates the event handles the library records into
     barrier(world)
@@ -328,19 +351,33 @@ def run_ours(args, rank, world, local):
         phases = None
     extra = {}
     if train:
-        bwd_ms = statistics.mean([b[0].elapsed_time(b[1]) for b in bev])
+        # the lookup's backward (after the Memory+ part, if any) against HBM
+        bwd_ms = statistics.mean([b[2].elapsed_time(b[1]) for b in bev])
         U = int(n_uniq.item())
         bbytes = backward_bytes(w, U)
         extra["backward"] = {"us": round(bwd_ms * 1e3, 1), "distinct_rows": U,
                              "algorithmic_bytes": bbytes,
                              "GBps": round(bbytes / (bwd_ms / 1e3) / 1e9, 1),
                              "frac": round(bbytes / (bwd_ms / 1e3) / 1e9 / peak, 4)}
+        if mp_train:
+            # five GEMMs of 2*T*d_model*d_v FLOPs: a, dz, dx, dW1, dW2
+            mp_ms = statistics.mean([b[0].elapsed_time(b[2]) for b in bev])
+            flops = 5 * 2 * T * w.d_model * w.d_v
+            tf = flops / (mp_ms / 1e3) / 1e12
+            pk = float(peaks["bf16_tflops"])
+            extra["memplus_backward"] = {"us": round(mp_ms * 1e3, 1), "flops": flops,
+                                         "TFLOPs": round(tf, 1), "peak": pk,
+                                         "frac": round(tf / pk, 4),
+                                         "peak_source": f"{peak_kind} bf16_tflops"}
 
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world,
-                      backward=(lambda: skv.check(lib.pkm_backward(skv.ctypes.byref(bargs), sptr),
-                                                  "pkm_backward")) if train else None)
+                      backward=(lambda: (
+                          skv.check(lib.pkm_memplus_backward(skv.ctypes.byref(margs), sptr),
+                                    "pkm_memplus_backward") if mp_train else None,
+                          skv.check(lib.pkm_backward(skv.ctypes.byref(bargs), sptr),
+                                    "pkm_backward"))) if train else None)
 
     clocks = clk.summary()
     l2 = "256 MiB L2 flush write before every timed step" if flush_between else \

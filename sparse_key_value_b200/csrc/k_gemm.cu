@@ -148,13 +148,14 @@ cudaError_t launch_gemm_simt(const void* A, const void* B, int64_t M, int N, int
   return cudaGetLastError();
 }
 cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                           int out_mode, void* C, int32_t* status, cudaStream_t stream);
+                           int out_mode, void* C, int32_t* status, cudaStream_t stream,
+                           int splits, int64_t c_split);
 
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
                              void* C, int32_t* status, cudaStream_t stream) {
   if (M <= 0) return cudaSuccess;
   if (gemm_tc_supported(M, N, K))
-    return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream);
+    return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream, 1, 0);
   return launch_gemm_simt(A, B, M, N, K, epi, 0, C, stream);
 }
 
@@ -163,8 +164,49 @@ cudaError_t launch_gemm_f32(const void* A, const void* B, int64_t M, int N, int 
   if (M <= 0 || N <= 0) return cudaSuccess;
   const int mode = accumulate ? 2 : 1;
   if (gemm_tc_supported(M, N, K))
-    return launch_gemm_tc(A, B, M, N, K, 0, mode, C, status, stream);
+    return launch_gemm_tc(A, B, M, N, K, 0, mode, C, status, stream, 1, 0);
   return launch_gemm_simt(A, B, M, N, K, 0, mode, C, stream);
+}
+
+// C = sum over s of part[s] (fixed order)
+__global__ void sum_slices_kernel(const float* __restrict__ part, int S, int64_t n,
+                                  float* __restrict__ C) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) acc += part[(int64_t)s * n + i];
+    C[i] = acc;
+  }
+}
+
+int gemm_splitk_slices(int64_t M, int N, int K) {
+  if (!gemm_tc_supported(M, N, K)) return 1;
+  const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
+  const int KB = (K + 63) / 64;
+  int s = 1;
+  while (s < 8 && tiles * s * 2 <= 148 && KB >= 4 * s * 2) s *= 2;
+  return s;
+}
+
+size_t gemm_splitk_workspace(int64_t M, int N, int K) {
+  const int s = gemm_splitk_slices(M, N, K);
+  return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
+}
+
+cudaError_t launch_gemm_f32_splitk(const void* A, const void* B, int64_t M, int N, int K,
+                                   float* C, float* part, int32_t* status, cudaStream_t stream) {
+  const int S = gemm_splitk_slices(M, N, K);
+  if (S <= 1 || !part) return launch_gemm_f32(A, B, M, N, K, false, C, status, stream);
+  cudaError_t e = launch_gemm_tc(A, B, M, N, K, 0, 1, part, status, stream, S, M * N);
+  if (e != cudaSuccess) return e;
+  // the GEMM launcher makes ceil(KB / ceil(KB / S)) slices; with KB >= 8 S this is S
+  const int KB = (K + 63) / 64, kbps = (KB + S - 1) / S, nz = (KB + kbps - 1) / kbps;
+  const int64_t n = M * N;
+  const int64_t blocks = (n + 255) / 256;
+  sum_slices_kernel<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, stream>>>(
+      part, nz, n, C);
+  note_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace pkm

@@ -54,7 +54,8 @@ __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, GemmCt
 template <int EPI, int OUT>
 __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t M,
-    int N, int K, void* __restrict__ Cv, int32_t* status) {
+    int N, int K, void* __restrict__ Cv, int kb_per_split, int64_t c_split,
+    int32_t* status) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* stages = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -62,7 +63,12 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t m0 = (int64_t)blockIdx.x * gm::kM;
   const int n0 = blockIdx.y * gm::kN;
-  const int KB = (K + gm::kKB - 1) / gm::kKB;
+  // split-K (grid.z): this CTA adds k-blocks [kb0, kb0 + KB) into the
+  // output slice blockIdx.z (c_split elements apart)
+  const int KB_all = (K + gm::kKB - 1) / gm::kKB;
+  const int kb0 = kb_per_split > 0 ? (int)blockIdx.z * kb_per_split : 0;
+  const int KB = kb_per_split > 0 ? min(kb_per_split, KB_all - kb0) : KB_all;
+  Cv = static_cast<char*>(Cv) + (int64_t)blockIdx.z * c_split * (OUT != 0 ? 4 : 2);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < gm::kStages; ++s) {
@@ -97,8 +103,8 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
         if (!gemm_wait(&ctl->empty[stage], phase ^ 1, ctl, status)) { ok = false; break; }
         unsigned char* sa = stages + stage * gm::kStageBytes;
         mbar_arrive_expect_tx(&ctl->full[stage], gm::kStageBytes);
-        tma_load_2d(sa, &tmA, &ctl->full[stage], kb * gm::kKB, (int32_t)m0);
-        tma_load_2d(sa + gm::kABytes, &tmB, &ctl->full[stage], kb * gm::kKB, n0);
+        tma_load_2d(sa, &tmA, &ctl->full[stage], (kb0 + kb) * gm::kKB, (int32_t)m0);
+        tma_load_2d(sa + gm::kABytes, &tmB, &ctl->full[stage], (kb0 + kb) * gm::kKB, n0);
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
       }
@@ -204,8 +210,10 @@ bool gemm_tc_supported(int64_t M, int N, int K) {
 }
 
 // out_mode: 0 bf16 (epi applied), 1 fp32, 2 fp32 accumulate; epi only with bf16 output.
+// splits > 1: split-K into `splits` slices of C, c_split elements apart.
 cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                           int out_mode, void* C, int32_t* status, cudaStream_t stream) {
+                           int out_mode, void* C, int32_t* status, cudaStream_t stream,
+                           int splits, int64_t c_split) {
   if (M <= 0) return cudaSuccess;
   CUtensorMap tmA, tmB;
   {
@@ -220,14 +228,21 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K
     const uint32_t box[2] = {(uint32_t)gm::kKB, (uint32_t)gm::kN};
     if (!make_tmap_bf16(&tmB, B, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  dim3 grid((unsigned)((M + gm::kM - 1) / gm::kM), (unsigned)((N + gm::kN - 1) / gm::kN));
+  const int KB = (K + gm::kKB - 1) / gm::kKB;
+  int kbps = 0, nz = 1;
+  if (splits > 1) {  // every slice gets at least one k-block
+    kbps = (KB + splits - 1) / splits;
+    nz = (KB + kbps - 1) / kbps;
+  }
+  dim3 grid((unsigned)((M + gm::kM - 1) / gm::kM), (unsigned)((N + gm::kN - 1) / gm::kN),
+            (unsigned)nz);
   cudaError_t e;
 #define PKM_GEMM_TC(E_, O_)                                                                  \
   e = cudaFuncSetAttribute(gemm_tc_kernel<E_, O_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                            (int)gm::kSmemBytes);                                             \
   if (e != cudaSuccess) return e;                                                            \
   gemm_tc_kernel<E_, O_><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(tmA, tmB, M, N, K, C, \
-                                                                        status)
+                                                                        kbps, c_split, status)
   if (out_mode == 1) {
     PKM_GEMM_TC(0, 1);
   } else if (out_mode == 2) {

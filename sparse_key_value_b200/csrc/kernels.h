@@ -77,6 +77,12 @@ cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int
 // C[M,N] (fp32) = A[M,K] B[N,K]^T, or C += it when accumulate.
 cudaError_t launch_gemm_f32(const void* A, const void* B, int64_t M, int N, int K,
                             bool accumulate, float* C, int32_t* status, cudaStream_t stream);
+// The same (C overwritten) split over K into slices when the output has few
+// tiles (weight gradients contracting over tokens): partial products in
+// `part` (gemm_splitk_workspace bytes), summed in slice order.
+size_t gemm_splitk_workspace(int64_t M, int N, int K);
+cudaError_t launch_gemm_f32_splitk(const void* A, const void* B, int64_t M, int N, int K,
+                                   float* C, float* part, int32_t* status, cudaStream_t stream);
 
 // ---------------------------------------------------------------- backward
 // dw[t,j] = <dy[t], table[idx[t,j]]>; with H>0 also dS = w (dw - sum w dw)

@@ -57,7 +57,7 @@ unsigned elem_grid(int64_t n) {
 }
 
 struct MpLayout {
-  size_t w1t, a, dz, da, z, xt, dat, zt, dot, total;
+  size_t w1t, a, dz, da, z, xt, dat, zt, dot, part, total;
 };
 
 MpLayout mp_layout(const pkm_memplus_bwd_args* g) {
@@ -79,6 +79,9 @@ MpLayout mp_layout(const pkm_memplus_bwd_args* g) {
   L.dat = take(dv * Tp * 2);
   L.zt = take(dv * Tp * 2);
   L.dot = take(dm * Tp * 2);
+  const size_t p1 = gemm_splitk_workspace((int64_t)dm, (int)dv, (int)Tp);
+  const size_t p2 = gemm_splitk_workspace((int64_t)dv, (int)dm, (int)Tp);
+  L.part = take(p1 > p2 ? p1 : p2);
   L.total = off;
   return L;
 }
@@ -101,7 +104,7 @@ pkm_status mp_validate(const pkm_memplus_bwd_args* g) {
 }
 
 struct QpLayout {
-  size_t wqt, dqb, dqt, xt, total;
+  size_t wqt, dqb, dqt, xt, part, total;
 };
 
 QpLayout qp_layout(const pkm_qproj_args* g) {
@@ -118,6 +121,7 @@ QpLayout qp_layout(const pkm_qproj_args* g) {
   L.dqb = take(T * dq * 2);
   L.dqt = take(dq * Tp * 2);
   L.xt = take(dm * Tp * 2);
+  L.part = take(gemm_splitk_workspace((int64_t)dm, (int)dq, (int)Tp));
   L.total = off;
   return L;
 }
@@ -194,8 +198,11 @@ pkm_status memplus_backward_impl(const pkm_memplus_bwd_args* g, cudaStream_t st)
   PKM_TRY(launch_transpose_bf16(da, (int)T, dv, ws + L.dat, st, (int)Tp));
   PKM_TRY(launch_transpose_bf16(z, (int)T, dv, ws + L.zt, st, (int)Tp));
   PKM_TRY(launch_transpose_bf16(g->dout, (int)T, dm, ws + L.dot, st, (int)Tp));
-  PKM_TRY(launch_gemm_f32(ws + L.xt, ws + L.dat, dm, dv, (int)Tp, false, g->dW1, status, st));
-  PKM_TRY(launch_gemm_f32(ws + L.zt, ws + L.dot, dv, dm, (int)Tp, false, g->dW2, status, st));
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  PKM_TRY(launch_gemm_f32_splitk(ws + L.xt, ws + L.dat, dm, dv, (int)Tp, g->dW1, part, status,
+                                 st));
+  PKM_TRY(launch_gemm_f32_splitk(ws + L.zt, ws + L.dot, dv, dm, (int)Tp, g->dW2, part, status,
+                                 st));
   return PKM_OK;
 }
 
@@ -256,7 +263,8 @@ PKM_API pkm_status pkm_qproj_backward(const pkm_qproj_args* g, pkm_stream_t stre
   PKM_TRY(launch_gemm_f32(dqb, g->Wq, T, dm, dq, true, g->dx, status, st));
   PKM_TRY(launch_transpose_bf16(g->x, (int)T, dm, ws + L.xt, st, (int)Tp));
   PKM_TRY(launch_transpose_bf16(dqb, (int)T, dq, ws + L.dqt, st, (int)Tp));
-  PKM_TRY(launch_gemm_f32(ws + L.xt, ws + L.dqt, dm, dq, (int)Tp, false, g->dWq, status, st));
+  PKM_TRY(launch_gemm_f32_splitk(ws + L.xt, ws + L.dqt, dm, dq, (int)Tp, g->dWq,
+                                 reinterpret_cast<float*>(ws + L.part), status, st));
   return PKM_OK;
 }
 

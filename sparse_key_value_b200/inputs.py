@@ -19,6 +19,8 @@ measured on; all data is synthetic, no dataset is involved):
                calibrated so that a least-squares fit of log(count) against
                log(rank) over ranks 1..10^4 of the selected rows gives an
                exponent of 1.10 (about 1.3e5 distinct rows of 2^20 slots).
+* ``memplus_train``  the ``memplus`` shapes and tables plus an upstream
+               gradient of the layer output (the Memory+ training step).
 * ``decode``   8 tokens per step x 256 steps against the ``memplus`` tables.
 
 Distributions: queries N(0,1); sub-keys N(0, std 1/sqrt(d_half)); values
@@ -105,6 +107,9 @@ WORKLOADS = {
     "train": Workload("train", T=8192, H=4, d_half=512, n_sub=1024, k=32, d_v=2048,
                       dtype="bf16", seed=1004, train=True,
                       zipf_alpha=0.5, zipf_beta=4.0, zipf_gamma=4.9),
+    "memplus_train": Workload("memplus_train", T=16384, H=4, d_half=512, n_sub=4096, k=32,
+                              d_v=1024, dtype="bf16", seed=1006, memplus=True, d_model=1024,
+                              train=True, table_seed_=1003),
     "decode": Workload("decode", T=8, H=4, d_half=512, n_sub=4096, k=32, d_v=1024,
                        dtype="bf16", seed=1005, memplus=True, d_model=1024,
                        decode_steps=256, table_seed_=1003),
@@ -177,7 +182,7 @@ def make_inputs(w: Workload, device="cpu", with_values: bool = True) -> dict:
         out["W1"] = _randn((w.d_model, w.d_v), s, gw).to(dt).to(device)
         out["W2"] = _randn((w.d_v, w.d_model), s, gw).to(dt).to(device)
     if w.train:
-        out["dy"] = _randn((w.T, w.d_v), 1.0, _cpu_gen(w.seed + 4)).to(dt).to(device)
+        out["dy"] = _randn((w.T, w.d_out), 1.0, _cpu_gen(w.seed + 4)).to(dt).to(device)
     if with_values:
         out["values"] = value_table(w, device)
     return out

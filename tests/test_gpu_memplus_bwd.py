@@ -45,8 +45,9 @@ def _memplus_case(seed, T, dm, dv):
 
 
 # (T, d_model, d_v): tensor-core GEMMs with a ragged token count; d_model = 32
-# puts the K = d_model products on the SIMT GEMM; T < 64 pads the token axis
-SHAPES = [(300, 256, 128), (130, 32, 48), (40, 64, 64), (1, 16, 8)]
+# puts the K = d_model products on the SIMT GEMM; T < 64 pads the token axis;
+# T = 4096 splits the token-contracting weight-gradient GEMMs over K
+SHAPES = [(300, 256, 128), (130, 32, 48), (40, 64, 64), (1, 16, 8), (4096, 256, 256)]
 
 
 @pytest.mark.parametrize("T,dm,dv", SHAPES, ids=[f"T{s[0]}-dm{s[1]}-dv{s[2]}" for s in SHAPES])
