@@ -307,3 +307,33 @@ def value_grad_rows(idx, w, dy, rows):
     _check(_load().orc_value_grad_rows(T, H, k, dv, _p(idx), _p(w), _p(da), dt, _p(rows),
                                        rows.shape[0], _p(out)), "value_grad_rows")
     return out
+
+
+def sparse_sgd(table, rows, grads, lr):
+    """table[r] -= lr * grad for the touched rows only ("모델 안의 메모리":
+    a fact lives in a few slots, so only those slots are updated).  fp64,
+    returns the updated table (a copy)."""
+    t = np.array(table, dtype=np.float64, copy=True)
+    rows = np.asarray(rows, dtype=np.int64)
+    g = np.asarray(grads, dtype=np.float64)
+    for i, r in enumerate(rows):
+        t[r] -= lr * g[i]
+    return t
+
+
+def sparse_adam(table, m, v, rows, grads, lr, beta1, beta2, eps, step):
+    """Adam restricted to the touched rows (moments of untouched rows are
+    left as they are, not decayed), with the bias corrections of the global
+    1-based step.  fp64; returns (table, m, v) updated copies."""
+    t = np.array(table, dtype=np.float64, copy=True)
+    m = np.array(m, dtype=np.float64, copy=True)
+    v = np.array(v, dtype=np.float64, copy=True)
+    rows = np.asarray(rows, dtype=np.int64)
+    g = np.asarray(grads, dtype=np.float64)
+    c1 = 1.0 - beta1 ** step
+    c2 = 1.0 - beta2 ** step
+    for i, r in enumerate(rows):
+        m[r] = beta1 * m[r] + (1.0 - beta1) * g[i]
+        v[r] = beta2 * v[r] + (1.0 - beta2) * g[i] * g[i]
+        t[r] -= lr * (m[r] / c1) / (np.sqrt(v[r] / c2) + eps)
+    return t, m, v

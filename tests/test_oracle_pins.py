@@ -421,3 +421,58 @@ def test_qproj_and_backward(orc):
     r = orc.qproj_backward(xb, Wqb, dq)
     np.testing.assert_allclose(r["dWq"], Wt.grad.numpy(), rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(r["dx"], xt.grad.numpy(), rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# sparse optimiser step on the touched rows
+# --------------------------------------------------------------------------
+
+def test_sparse_sgd_equals_dense_sgd_with_zero_rows(orc):
+    """Sparse SGD equals torch's dense SGD step whose gradient is zero on the
+    untouched rows."""
+    rng = np.random.default_rng(31)
+    table, rows = rng.normal(size=(20, 6)), np.array([3, 7, 11, 19])
+    grads = rng.normal(size=(4, 6))
+    p = torch.tensor(table, requires_grad=True)
+    dense = np.zeros_like(table)
+    dense[rows] = grads
+    p.grad = torch.from_numpy(dense)
+    torch.optim.SGD([p], lr=0.05).step()
+    np.testing.assert_allclose(orc.sparse_sgd(table, rows, grads, 0.05), p.detach().numpy(),
+                               rtol=0, atol=1e-15)
+
+
+def test_sparse_adam_equals_torch_sparse_adam(orc):
+    """Three steps of the touched-rows Adam equal torch.optim.SparseAdam fed
+    the same sparse gradients (different rows each step).  torch applies eps
+    after folding the bias corrections into the step size (eps scaled by
+    sqrt(1 - beta2^t) relative to the oracle's m_hat / (sqrt(v_hat) + eps));
+    a negligible eps makes the two forms coincide."""
+    rng = np.random.default_rng(32)
+    table = rng.normal(size=(16, 5))
+    p = torch.nn.Parameter(torch.tensor(table))
+    opt = torch.optim.SparseAdam([p], lr=0.01, betas=(0.9, 0.99), eps=1e-30)
+    t, m, v = table, np.zeros_like(table), np.zeros_like(table)
+    for step, rows in enumerate(([1, 4, 9], [4, 5], [0, 9, 15]), start=1):
+        rows = np.array(rows)
+        grads = rng.normal(size=(len(rows), 5))
+        p.grad = torch.sparse_coo_tensor(torch.from_numpy(rows)[None], torch.from_numpy(grads),
+                                         (16, 5))
+        opt.step()
+        t, m, v = orc.sparse_adam(t, m, v, rows, grads, 0.01, 0.9, 0.99, 1e-30, step)
+        np.testing.assert_allclose(t, p.detach().numpy(), rtol=1e-12, atol=1e-14)
+    untouched = np.setdiff1d(np.arange(16), [0, 1, 4, 5, 9, 15])
+    np.testing.assert_array_equal(t[untouched], table[untouched])
+
+
+def test_sparse_adam_first_step_closed_form(orc):
+    """Step 1 from zero moments: m_hat = g and v_hat = g^2, so the update is
+    lr * g / (|g| + eps) on the touched rows."""
+    rng = np.random.default_rng(33)
+    table, rows = rng.normal(size=(10, 4)), np.array([2, 6])
+    g = rng.normal(size=(2, 4))
+    t, m, v = orc.sparse_adam(table, np.zeros_like(table), np.zeros_like(table), rows, g,
+                              0.1, 0.9, 0.999, 0.5, 1)
+    ref = table.copy()
+    ref[rows] -= 0.1 * g / (np.abs(g) + 0.5)
+    np.testing.assert_allclose(t, ref, rtol=1e-13, atol=1e-15)
