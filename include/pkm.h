@@ -295,6 +295,41 @@ PKM_API size_t pkm_qproj_workspace_size(const pkm_qproj_args *args);
 PKM_API pkm_status pkm_qproj_forward(const pkm_qproj_args *args, pkm_stream_t stream);
 PKM_API pkm_status pkm_qproj_backward(const pkm_qproj_args *args, pkm_stream_t stream);
 
+/*
+ * Optimiser step on the touched value rows only ("모델 안의 메모리", "잊지 않고
+ * 배우기": a fact occupies a few memory slots, so only those are updated).
+ * The rows and gradients are pkm_backward's sparse value gradient
+ * (uniq_rows, grad_rows, n_uniq); each row is updated in place by one CTA:
+ *   PKM_OPT_SGD   p -= lr * g
+ *   PKM_OPT_ADAM  m = beta1 m + (1-beta1) g;  v = beta2 v + (1-beta2) g^2;
+ *                 p -= lr * (m / c1) / (sqrt(v / c2) + eps),  c = 1 - beta^step;
+ *                 the moments of untouched rows are left as they are.
+ * bf16 tables are updated in fp32 and rounded once (nearest even).
+ *   table [n_rows, d] (dtype), rows [cap] distinct ids, grads [cap, d] fp32,
+ *   count device int64 (entries used: min(*count, cap); more sets
+ *   PKM_ERR_DEVICE), m, v [n_rows, d] fp32 (Adam only).
+ * Limits: d a multiple of 8; Adam: 0 <= beta < 1, eps >= 0, step >= 1.
+ */
+typedef enum { PKM_OPT_SGD = 0, PKM_OPT_ADAM = 1 } pkm_opt_kind;
+
+typedef struct {
+    pkm_opt_kind kind;
+    float lr, beta1, beta2, eps;
+    int64_t step;
+    int64_t n_rows;
+    int32_t d;
+    pkm_dtype dtype;
+    void *table;
+    const int32_t *rows;
+    const float *grads;
+    const int64_t *count;
+    int64_t cap;
+    float *m;
+    float *v;
+} pkm_sparse_opt_args;
+
+PKM_API pkm_status pkm_sparse_optimizer_step(const pkm_sparse_opt_args *args, pkm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

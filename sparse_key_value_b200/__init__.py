@@ -272,3 +272,23 @@ def qproj_backward(x, Wq, dq, dx=None, workspace=None, stream=None):
     _qproj_call("pkm_qproj_backward", _qproj_args(x, Wq, dq=dq, dWq=dWq, dx=dx), dev, workspace,
                 stream)
     return dict(dWq=dWq, dx=dx)
+
+
+def sparse_optimizer_step(table, rows, grads, count, lr: float, kind: str = "sgd", m=None,
+                          v=None, betas=(0.9, 0.999), eps: float = 1e-8, step: int = 1,
+                          stream=None):
+    """In-place SGD or touched-rows Adam on the rows of a sparse value
+    gradient (see pkm_sparse_optimizer_step in include/pkm.h): table
+    [n_rows, d], rows int32 [cap], grads fp32 [cap, d], count device int64
+    [1] (pkm_backward's uniq_rows, grad_rows, n_uniq); m, v fp32 [n_rows, d]
+    for Adam."""
+    _need_cuda(table, rows, grads, count, m, v)
+    adam = kind == "adam"
+    if adam and (m is None or v is None):
+        raise ValueError("adam needs the moment tensors m and v")
+    a = _lib.SparseOptArgs(1 if adam else 0, lr, betas[0], betas[1], eps, step, table.shape[0],
+                           table.shape[1], _dt(table), _p(table), _p(rows), _p(grads), _p(count),
+                           rows.shape[0], _p(m), _p(v))
+    check(load().pkm_sparse_optimizer_step(ctypes.byref(a), _stream(table.device, stream)),
+          "pkm_sparse_optimizer_step")
+    return table

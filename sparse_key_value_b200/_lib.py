@@ -59,12 +59,19 @@ class QprojArgs(ctypes.Structure):
                 ("dq", P), ("dWq", P), ("dx", P), ("workspace", P), ("workspace_bytes", SZ)]
 
 
+class SparseOptArgs(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("lr", ctypes.c_float), ("beta1", ctypes.c_float),
+                ("beta2", ctypes.c_float), ("eps", ctypes.c_float), ("step", I64),
+                ("n_rows", I64), ("d", I32), ("dtype", ctypes.c_int), ("table", P), ("rows", P),
+                ("grads", P), ("count", P), ("cap", I64), ("m", P), ("v", P)]
+
+
 EXPORTS = ("pkm_forward_workspace_size", "pkm_forward", "pkm_backward_workspace_size",
            "pkm_backward", "embbag_forward", "embbag_backward_workspace_size",
            "embbag_backward", "pkm_get_device_error", "pkm_status_string", "pkm_version",
            "pkm_launch_count", "pkm_forward_noalloc", "pkm_memplus_backward_workspace_size",
            "pkm_memplus_backward", "pkm_qproj_workspace_size", "pkm_qproj_forward",
-           "pkm_qproj_backward")
+           "pkm_qproj_backward", "pkm_sparse_optimizer_step")
 
 _lib = None
 
@@ -114,6 +121,8 @@ def load(path: str = LIB_PATH):
     lib.pkm_qproj_forward.restype = ctypes.c_int
     lib.pkm_qproj_backward.argtypes = [QA, P]
     lib.pkm_qproj_backward.restype = ctypes.c_int
+    lib.pkm_sparse_optimizer_step.argtypes = [ctypes.POINTER(SparseOptArgs), P]
+    lib.pkm_sparse_optimizer_step.restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
     return lib

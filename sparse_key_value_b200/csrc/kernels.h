@@ -84,6 +84,14 @@ size_t gemm_splitk_workspace(int64_t M, int N, int K);
 cudaError_t launch_gemm_f32_splitk(const void* A, const void* B, int64_t M, int N, int K,
                                    float* C, float* part, int32_t* status, cudaStream_t stream);
 
+// In-place SGD / touched-rows Adam on the rows of a sparse value gradient
+// (see k_sparse_opt.cu); m, v are [n_rows, d] fp32 Adam moments.
+cudaError_t launch_sparse_opt(void* table, pkm_dtype dt, int64_t n_rows, int d,
+                              const int32_t* rows, const float* grads, const int64_t* count,
+                              int64_t cap, bool adam, float* m, float* v, float lr, float b1,
+                              float b2, float eps, int64_t step, int32_t* status,
+                              cudaStream_t stream);
+
 // ---------------------------------------------------------------- backward
 // dw[t,j] = <dy[t], table[idx[t,j]]>; with H>0 also dS = w (dw - sum w dw)
 // per (t, h) group of k.

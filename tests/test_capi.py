@@ -159,3 +159,25 @@ def test_qproj_validation(lib):
     assert lib.pkm_qproj_backward(ctypes.byref(a), None) == 1  # no dq
     a = _lib.QprojArgs(64, 64, 16, fake, fake, fake, fake, fake, fake, fake, 16)
     assert lib.pkm_qproj_forward(ctypes.byref(a), None) == 6
+
+
+def test_sparse_optimizer_validation(lib):
+    from sparse_key_value_b200 import _lib
+    fake = ctypes.c_void_p(1 << 20)
+
+    def args(**kw):
+        base = dict(kind=0, lr=0.1, beta1=0.9, beta2=0.999, eps=1e-8, step=1, n_rows=100, d=64,
+                    dtype=1, cap=10)
+        base.update(kw)
+        return _lib.SparseOptArgs(base["kind"], base["lr"], base["beta1"], base["beta2"],
+                                  base["eps"], base["step"], base["n_rows"], base["d"],
+                                  base["dtype"], fake, fake, fake, fake, base["cap"], fake, fake)
+
+    assert lib.pkm_sparse_optimizer_step(ctypes.byref(args(d=60)), None) == 1
+    assert lib.pkm_sparse_optimizer_step(ctypes.byref(args(kind=2)), None) == 1
+    assert lib.pkm_sparse_optimizer_step(ctypes.byref(args(kind=1, beta1=1.0)), None) == 1
+    assert lib.pkm_sparse_optimizer_step(ctypes.byref(args(kind=1, step=0)), None) == 1
+    assert lib.pkm_sparse_optimizer_step(ctypes.byref(args(lr=float("nan"))), None) == 1
+    a = args(kind=1)
+    a.m = None
+    assert lib.pkm_sparse_optimizer_step(ctypes.byref(a), None) == 1
