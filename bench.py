@@ -371,6 +371,19 @@ def run_ours(args, rank, world, local):
                                          "peak_source": f"{peak_kind} bf16_tflops"}
 
     if train:
+        # the step's dominant work is the lookup backward, so the roofline
+        # reports it; the gather's figure over-counts there, since Zipf-skewed
+        # rows repeat and the repeats hit L2
+        b = extra["backward"]
+        extra["gather"] = dict(roof, note="Zipf-skewed rows repeat across tokens; repeated "
+                                          "rows are L2 hits, so algorithmic bytes over-count DRAM")
+        roof = {"kernel": "pkm_backward (sort, segmented value-gradient sum, dw/dS, dq, dK)",
+                "bound": "hbm", "achieved": b["GBps"], "peak": peak, "unit": "GB/s",
+                "frac": b["frac"], "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": b["algorithmic_bytes"], "traffic": None,
+                "backward_us": b["us"]}
+
+    if train:
         # optimiser step on the touched rows (not part of the timed training
         # step): touched-rows Adam with fp32 moments on the backward's sparse
         # gradient, applied to the table in place after everything else

@@ -6,6 +6,8 @@ import numpy as np
 import pytest
 import torch
 
+from parity import RTOL, close
+
 pytestmark = pytest.mark.gpu
 
 skv = pytest.importorskip("sparse_key_value_b200")
@@ -105,3 +107,42 @@ def test_step_on_backward_output():
     mask = torch.ones(table.shape[0], dtype=torch.bool, device="cuda")
     mask[rows] = False
     assert torch.equal(table[mask], before[mask])
+
+
+def test_shared_pool_gradient_in_one_reduction():
+    """"Memory Layers at Scale" digest, "공유 메모리 풀": several layers read one
+    value pool.  Each layer's forward writes its selection into its slice of
+    one layer-major buffer; the pool's sparse value gradient is then one
+    sorted segmented sum over all layers' slots (embbag_backward), equal to
+    the oracle's sum over the layers and to per-layer gradients added
+    densely."""
+    import oracle
+
+    L = 3
+    w = WORKLOADS["train"].scaled(T=128, H=2, d_half=256, n_sub=64, k=8, d_v=64)
+    pool = make_inputs(w, "cuda")["values"]
+    T, B = w.T, w.H * w.k
+    idx = torch.empty(L * T, B, dtype=torch.int32, device="cuda")
+    wts = torch.empty(L * T, B, dtype=torch.float32, device="cuda")
+    g = torch.Generator().manual_seed(41)
+    dy = torch.randn(L * T, w.d_v, generator=g).to(torch.bfloat16).cuda()
+    for layer in range(L):
+        lw = w.scaled(seed=w.seed + 100 * (layer + 1), table_seed_=w.seed + 200 * (layer + 1))
+        li = make_inputs(lw, "cuda", with_values=False)
+        s = slice(layer * T, (layer + 1) * T)
+        skv.pkm_forward(li["query"], li["subkeys"], pool, w.k, idx=idx[s].view(T, w.H, w.k),
+                        weights=wts[s].view(T, w.H, w.k))
+    res = skv.embbag_backward(dy, idx, wts, n_rows=pool.shape[0])
+    dense = torch.zeros(pool.shape[0], w.d_v, dtype=torch.float32, device="cuda")
+    for layer in range(L):
+        s = slice(layer * T, (layer + 1) * T)
+        skv.embbag_backward(dy[s], idx[s], wts[s], n_rows=pool.shape[0], sparse=False,
+                            dense=dense)
+    torch.cuda.synchronize()
+    rows = np.unique(idx.cpu().numpy().astype(np.int64))
+    np.testing.assert_array_equal(res["uniq_rows"].cpu().numpy(), rows)
+    ref = oracle.value_grad_rows(idx.cpu().numpy().astype(np.int64).reshape(L * T, 1, B),
+                                 wts.double().cpu().numpy().reshape(L * T, 1, B), dy.cpu(), rows)
+    close(res["grad_rows"].cpu().numpy(), ref, RTOL["f32"], "pool grad_rows")
+    close(dense[torch.from_numpy(rows).cuda()].cpu().numpy(), ref, RTOL["f32"],
+          "per-layer dense sum")
