@@ -101,18 +101,61 @@ def whole_job_tokens_per_s(tokens_per_rank: int, world: int, max_ms_per_step: fl
 
 
 class Clocks:
-    """nvidia-smi samples (200 ms) of this GPU during the timed region."""
+    """SM clock and throttle-reason samples of this GPU during the timed region.
+
+    NVML (read-only queries) from a thread every 5 ms, so that even a short
+    timed region is covered; the first sample is taken before the region
+    starts counting.  Falls back to `nvidia-smi -lms 200` when NVML is not
+    importable."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
+        self.nvml = None
+        self.samples = []  # (sm MHz, max MHz, reason names)
         self.path = os.path.join("/tmp", f"pkm_clocks_{os.getpid()}.csv")
 
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+        return pynvml, h
+
+    def _sample_nvml(self):
+        nv, h = self.nvml
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while True:
+            sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.samples.append((sm, smax, [n for n, b in bits.items() if r & b]))
+            self.started.set()
+            if self.stop.wait(0.005):
+                return
+
     def __enter__(self):
+        import threading
+        try:
+            self.nvml = self._nvml_handle()
+            self.stop, self.started = threading.Event(), threading.Event()
+            self.thread = threading.Thread(target=self._sample_nvml, daemon=True)
+            self.thread.start()
+            self.started.wait(2.0)
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -124,6 +167,10 @@ class Clocks:
         return self
 
     def __exit__(self, *exc):
+        if self.nvml is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            return
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -133,26 +180,30 @@ class Clocks:
             self.f.close()
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        os.remove(self.path)
-        loaded = [s for s in sm if smax and s > 0.5 * smax] or sm
+        source = "nvml 5 ms"
+        if self.nvml is None:
+            source = "nvidia-smi 200 ms"
+            if self.proc is None or not os.path.exists(self.path):
+                return {"sm_mhz": None, "sm_max_mhz": None,
+                        "reasons": ["nvidia-smi unavailable"]}
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm_v, smax_v = float(f[1]), float(f[2])
+                except ValueError:
+                    continue
+                self.samples.append((sm_v, smax_v,
+                                     [n for n, v in zip(self.NAMES, f[5:9])
+                                      if v.lower() == "active"]))
+            os.remove(self.path)
+        sm = [x[0] for x in self.samples]
+        smax = self.samples[-1][1] if self.samples else None
+        reasons = sorted({n for x in self.samples for n in x[2]})
+        loaded = [v for v in sm if smax and v > 0.5 * smax] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": len(sm), "source": source, "reasons": reasons}
 
 
 def measured_peaks():
