@@ -158,7 +158,9 @@ def test_forward_deterministic():
 # ------------------------------------------------------------ bag gather --
 
 BAGS = [(1, 1, 8, "bf16"), (513, 128, 2048, "bf16"), (77, 33, 1024, "bf16"),
-        (50, 7, 24, "f32"), (31, 128, 4096, "bf16"), (200, 5, 8, "f32")]
+        (50, 7, 24, "f32"), (31, 128, 4096, "bf16"), (200, 5, 8, "f32"),
+        (301, 16, 512, "bf16"), (64, 9, 256, "f32"), (40, 3, 1024, "f32"),
+        (5, 2, 8192, "bf16"), (1, 130, 512, "bf16")]
 
 
 @pytest.mark.parametrize("n_bags,B,d,dt", BAGS)
@@ -188,6 +190,38 @@ def test_embbag_bad_index_sets_status():
     assert skv.device_error() == 0  # cleared on read
     ref = 0.5 * (table[0].float() + table[1].float())
     torch.testing.assert_close(out[0].float(), ref, rtol=2e-2, atol=1e-2)
+
+
+def test_embbag_bad_index_wide_rows():
+    """Bad row ids among many good ones in rows of 1 KiB: each bad id is
+    skipped and reported; the other rows of its bag still sum."""
+    g = torch.Generator().manual_seed(5)
+    table = torch.randn(50, 512, generator=g).to(torch.bfloat16).cuda()
+    idx = torch.tensor([[0, 1, 50], [2, -7, 3], [4, 5, 6]], dtype=torch.int32, device="cuda")
+    w = torch.full((3, 3), 0.5, device="cuda")
+    out = skv.embbag_forward(table, idx, w)
+    assert skv.device_error() == 4  # PKM_ERR_DEVICE
+    ref = 0.5 * torch.stack([table[0].float() + table[1].float(),
+                             table[2].float() + table[3].float(),
+                             table[4].float() + table[5].float() + table[6].float()])
+    torch.testing.assert_close(out.float(), ref, rtol=2e-2, atol=1e-2)
+
+
+def test_embbag_row_order_sum():
+    """The gather sums each bag's rows in order j = 0 .. B-1 in fp32 and
+    rounds once: against a sequential fp32 sum done here (fused and separate
+    multiply-adds differ by at most one rounding per row)."""
+    g = torch.Generator().manual_seed(6)
+    n_bags, B, d = 9, 40, 1024
+    table = torch.randn(300, d, generator=g).to(torch.bfloat16)
+    idx, w = random_bags(n_bags, B, 300, seed=7)
+    out = skv.embbag_forward(table.cuda(), idx.cuda(), w.cuda())
+    ref = torch.zeros(n_bags, d)
+    tf = table.float()
+    for j in range(B):
+        ref = ref + w[:, j:j + 1] * tf[idx[:, j].long()]
+    torch.testing.assert_close(out.float().cpu(), ref.to(torch.bfloat16).float(), rtol=1e-2,
+                               atol=1e-3)
 
 
 # ------------------------------------------------- full-size workloads --
