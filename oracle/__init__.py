@@ -15,6 +15,8 @@ Each function states which passage of the pages it follows:
 * "Memory Layers at Scale" digest, "병렬 EmbeddingBag 구현": the weighted bag.
 * "모델 안의 메모리", "작동 방식" and figure D: halves scored against the
   half-keys, best of each combined, weighted average of the values read.
+* "Conditional Memory via Scalable Lookup" review (Engram), "희소 검색" and
+  "핵심 수식": multi-head hashed n-gram rows, the context gate.
 
 Parity pins (tests/test_oracle_pins.py) tie every function to something other
 than itself: brute force over all N keys, closed forms, numpy/torch library
@@ -72,11 +74,15 @@ def _load():
         lib.orc_memplus_backward.argtypes = [I64, I, I, P, P, I, P, I, P, I, P, I, P, P, P, P]
         lib.orc_qproj.argtypes = [I64, I, I, P, I, P, I, P]
         lib.orc_qproj_backward.argtypes = [I64, I, I, P, I, P, I, P, P, P]
+        lib.orc_engram_rows.argtypes = [I64, I, P, I, P, I, P, P, P]
+        lib.orc_engram_gate.argtypes = [I64, I, I, P, P, I, I64, P, I, ctypes.c_double, P, P,
+                                        P]
         lib.orc_num_threads.argtypes = []
         for f in ("orc_half_scores", "orc_topk", "orc_pkm_select",
                   "orc_bruteforce_select", "orc_softmax", "orc_bag", "orc_memplus",
                   "orc_pkm_backward", "orc_num_threads", "orc_value_grad_rows",
-                  "orc_memplus_backward", "orc_qproj", "orc_qproj_backward"):
+                  "orc_memplus_backward", "orc_qproj", "orc_qproj_backward",
+                  "orc_engram_rows", "orc_engram_gate"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -337,3 +343,47 @@ def sparse_adam(table, m, v, rows, grads, lr, beta1, beta2, eps, step):
         v[r] = beta2 * v[r] + (1.0 - beta2) * g[i] * g[i]
         t[r] -= lr * (m[r] / c1) / (np.sqrt(v[r] / c2) + eps)
     return t, m, v
+
+
+ENGRAM_PAD = 0xFFFFFFFF
+ENGRAM_EPS = 1e-6
+
+
+def engram_rows(tokens, orders, K: int, seeds, M):
+    """Engram multi-head hashing ("Conditional Memory via Scalable Lookup"
+    review, "다중 헤드 해싱"; "핵심 수식" 1: e = E_{n,k}[phi_{n,k}(g_{t,n})]).
+
+    tokens [n_seq, L] ids >= 0; orders: the n-gram orders; K hashes per
+    order; seeds / M: per head j = o*K + k (uint64 seed, rows of its
+    table).  Returns rows int64 [n_seq*L, len(orders)*K] of the stacked
+    table (head j's rows follow those of the heads before it).  The hash is
+    the one the C source defines (the page names none)."""
+    tok = np.ascontiguousarray(tokens, dtype=np.int32)
+    n_seq, L = tok.shape
+    od = np.ascontiguousarray(orders, dtype=np.int32)
+    sd = np.ascontiguousarray(seeds, dtype=np.uint64)
+    Ma = np.ascontiguousarray(M, dtype=np.int64)
+    HK = len(od) * K
+    assert sd.shape == (HK,) and Ma.shape == (HK,)
+    rows = np.empty((n_seq * L, HK), dtype=np.int64)
+    _check(_load().orc_engram_rows(n_seq, L, _p(tok), len(od), _p(od), K, _p(sd), _p(Ma),
+                                   _p(rows)), "engram_rows")
+    return rows
+
+
+def engram_gate(rows, E, h, eps: float = ENGRAM_EPS):
+    """e_t = sum of the heads' rows; the context gate ("핵심 수식" 2)
+    alpha_t = sigmoid(<RMSNorm(h_t), RMSNorm(e_t)> / sqrt(d)) with the
+    parameter-free RMSNorm; v_t = alpha_t e_t.  fp64.  Returns dict(e,
+    alpha, v)."""
+    r = np.ascontiguousarray(rows, dtype=np.int64)
+    T, HK = r.shape
+    ea, et = _input(E)
+    ha, ht = _input(h)
+    d = ea.shape[1]
+    e = np.empty((T, d))
+    a = np.empty(T)
+    v = np.empty((T, d))
+    _check(_load().orc_engram_gate(T, HK, d, _p(r), _p(ea), et, ea.shape[0], _p(ha), ht, eps,
+                                   _p(e), _p(a), _p(v)), "engram_gate")
+    return dict(e=e, alpha=a, v=v)

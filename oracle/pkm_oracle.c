@@ -638,3 +638,91 @@ int orc_qproj_backward(int64_t T, int dm, int dq, const void *x, int x_dtype, co
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Engram hashed n-gram lookup ["Conditional Memory via Scalable      */
+/* Lookup" review, "희소 검색": multi-head hashing; "핵심 수식" 1 and 2] */
+/* ------------------------------------------------------------------ */
+
+/* phi_{n,k}(g): the page names independent hash functions per n-gram order
+   and head but not the functions themselves.  This oracle's definition
+   (shared with the CUDA path only through this statement, not code):
+   h = seed; for each token id x of g, oldest first, taken as 32 unsigned
+   bits: h ^= x; h *= 0x9E3779B97F4A7C15 (mod 2^64); h ^= h >> 32.
+   The row inside the head's table is h mod M. */
+static uint64_t engram_hash(const int32_t *seq, int64_t p, int n, uint64_t seed) {
+    uint64_t h = seed;
+    for (int i = n - 1; i >= 0; i--) {
+        const int64_t q = p - i;
+        const uint32_t x = q >= 0 ? (uint32_t)seq[q] : ORC_ENGRAM_PAD;
+        h ^= (uint64_t)x;
+        h *= 0x9E3779B97F4A7C15ull;
+        h ^= h >> 32;
+    }
+    return h;
+}
+
+int orc_engram_rows(int64_t n_seq, int L, const int32_t *tokens, int n_orders,
+                    const int *orders, int K, const uint64_t *seeds, const int64_t *M,
+                    int64_t *rows_out) {
+    if (n_seq < 0 || L < 1 || n_orders < 1 || K < 1) return -2;
+    const int HK = n_orders * K;
+    int64_t *offset = malloc(sizeof(int64_t) * HK);
+    if (!offset) return -1;
+    int64_t off = 0;
+    for (int j = 0; j < HK; j++) {
+        if (M[j] < 1 || orders[j / K] < 1) {
+            free(offset);
+            return -2;
+        }
+        offset[j] = off;  /* head j's table starts after the heads before it */
+        off += M[j];
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t s = 0; s < n_seq; s++)
+        for (int p = 0; p < L; p++)
+            for (int o = 0; o < n_orders; o++)
+                for (int k = 0; k < K; k++) {
+                    const int j = o * K + k;
+                    const uint64_t h = engram_hash(tokens + s * L, p, orders[o], seeds[j]);
+                    rows_out[(s * L + p) * HK + j] = offset[j] + (int64_t)(h % (uint64_t)M[j]);
+                }
+    free(offset);
+    return 0;
+}
+
+/* e_t = sum over the HK heads of E[row]; the context gate
+   alpha_t = sigmoid(<RMSNorm(h_t), RMSNorm(e_t)> / sqrt(d)) with the
+   parameter-free RMSNorm x / sqrt(mean(x^2) + eps); v_t = alpha_t e_t. */
+int orc_engram_gate(int64_t T, int HK, int d, const int64_t *rows, const void *E, int e_dtype,
+                    int64_t n_rows, const void *h, int h_dtype, double eps, double *e_out,
+                    double *alpha_out, double *v_out) {
+    if (T < 0 || HK < 1 || d < 1) return -2;
+    int err = 0;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; t++) {
+        double *e = e_out + t * d;
+        for (int i = 0; i < d; i++) e[i] = 0.0;
+        for (int j = 0; j < HK; j++) {
+            const int64_t r = rows[t * HK + j];
+            if (r < 0 || r >= n_rows) {
+                err = -3;
+                continue;
+            }
+            for (int i = 0; i < d; i++) e[i] += ld(E, e_dtype, r * d + i);
+        }
+        double hh = 0.0, ee = 0.0, he = 0.0;
+        for (int i = 0; i < d; i++) {
+            const double hv = ld(h, h_dtype, t * d + i);
+            hh += hv * hv;
+            ee += e[i] * e[i];
+            he += hv * e[i];
+        }
+        const double rh = sqrt(hh / d + eps), re = sqrt(ee / d + eps);
+        const double logit = he / (rh * re) / sqrt((double)d);
+        const double a = 1.0 / (1.0 + exp(-logit));
+        alpha_out[t] = a;
+        for (int i = 0; i < d; i++) v_out[t * d + i] = a * e[i];
+    }
+    return err;
+}

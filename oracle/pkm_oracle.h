@@ -18,6 +18,7 @@
 #define ORC_F32 1
 #define ORC_BF16 2
 #define ORC_NORM_EPS 1e-12
+#define ORC_ENGRAM_PAD 0xFFFFFFFFu /* token id read before a sequence's start */
 
 #ifdef __cplusplus
 extern "C" {
@@ -80,6 +81,21 @@ int orc_qproj_backward(int64_t T, int dm, int dq, const void *x, int x_dtype, co
 int orc_value_grad_rows(int64_t T, int H, int k, int dv, const int64_t *idx, const double *w,
                         const void *dy, int dy_dtype, const int64_t *rows, int64_t n_rows,
                         double *out);
+
+/* Engram ("Conditional Memory via Scalable Lookup" review): hashed n-gram
+   rows.  tokens [n_seq, L] (ids >= 0); orders [n_orders]; seeds and M
+   [n_orders * K] (head j = o*K + k); rows_out [n_seq*L, n_orders*K] are
+   global rows of the stacked table (head j's rows after those of heads < j).
+   Positions before a sequence's start read the pad id ORC_ENGRAM_PAD. */
+int orc_engram_rows(int64_t n_seq, int L, const int32_t *tokens, int n_orders,
+                    const int *orders, int K, const uint64_t *seeds, const int64_t *M,
+                    int64_t *rows_out);
+
+/* e = sum of the HK rows, alpha = sigmoid(<rms(h), rms(e)>/sqrt(d)), v = alpha e;
+   E [n_rows, d], h [T, d]; e_out, v_out [T, d], alpha_out [T] */
+int orc_engram_gate(int64_t T, int HK, int d, const int64_t *rows, const void *E, int e_dtype,
+                    int64_t n_rows, const void *h, int h_dtype, double eps, double *e_out,
+                    double *alpha_out, double *v_out);
 
 int orc_num_threads(void);
 

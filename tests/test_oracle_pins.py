@@ -476,3 +476,137 @@ def test_sparse_adam_first_step_closed_form(orc):
     ref = table.copy()
     ref[rows] -= 0.1 * g / (np.abs(g) + 0.5)
     np.testing.assert_allclose(t, ref, rtol=1e-13, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# Engram ("Conditional Memory via Scalable Lookup" review): hashed n-gram
+# rows and the context gate.  The page names independent hash functions per
+# order and head but not the functions, so the hash is pinned by what the
+# page does fix: each head reads its own table, a row depends on its n-gram
+# window alone, equal n-grams give equal rows, and the heads are independent.
+# --------------------------------------------------------------------------
+
+_ORDERS, _K = [2, 3], 2
+_SEEDS = [0x1234, 0xBEEF, 0x51ED, 0xC0DE]
+_M = [1009, 1013, 997, 1019]
+
+
+def test_engram_rows_stay_in_their_heads_table(orc):
+    tok = np.random.default_rng(40).integers(0, 50000, (3, 200))
+    rows = orc.engram_rows(tok, _ORDERS, _K, _SEEDS, _M)
+    off = np.concatenate([[0], np.cumsum(_M)[:-1]])
+    assert rows.shape == (600, 4)
+    assert np.all(rows >= off) and np.all(rows < off + np.array(_M))
+
+
+def test_engram_row_depends_only_on_its_window(orc):
+    """Changing a token outside positions p-n+1..p leaves the order-n rows
+    at p alone; changing one inside moves them (up to a 1/M collision)."""
+    rng = np.random.default_rng(41)
+    tok = rng.integers(0, 50000, (1, 64))
+    base = orc.engram_rows(tok, _ORDERS, _K, _SEEDS, _M)
+    p = 40
+    moved = 0
+    for o, n in enumerate(_ORDERS):
+        cols = slice(o * _K, (o + 1) * _K)
+        for q in (p - n, p + 1):  # just outside the window
+            t2 = tok.copy()
+            t2[0, q] += 1
+            np.testing.assert_array_equal(orc.engram_rows(t2, _ORDERS, _K, _SEEDS, _M)[p, cols],
+                                          base[p, cols])
+        for q in range(p - n + 1, p + 1):  # inside it
+            t2 = tok.copy()
+            t2[0, q] += 1
+            moved += int(np.any(orc.engram_rows(t2, _ORDERS, _K, _SEEDS, _M)[p, cols]
+                                != base[p, cols]))
+    assert moved == sum(_ORDERS)
+
+
+def test_engram_equal_ngrams_equal_rows(orc):
+    """The same n-gram planted at other positions and in another sequence
+    reads the same rows; a bigram that agrees only in its last token does
+    not."""
+    rng = np.random.default_rng(42)
+    tok = rng.integers(0, 50000, (2, 50))
+    tok[0, 10:13] = tok[1, 30:33] = [7, 8, 9]
+    rows = orc.engram_rows(tok, _ORDERS, _K, _SEEDS, _M).reshape(2, 50, -1)
+    np.testing.assert_array_equal(rows[0, 12], rows[1, 32])      # 2- and 3-gram (7,8,9)
+    np.testing.assert_array_equal(rows[0, 11, :_K], rows[1, 31, :_K])  # bigram (7,8)
+    tok[1, 31] = 6                                                # (6,9) vs (8,9)
+    rows2 = orc.engram_rows(tok, _ORDERS, _K, _SEEDS, _M).reshape(2, 50, -1)
+    assert np.any(rows2[1, 32, :_K] != rows[0, 12, :_K])
+
+
+def test_engram_sequence_start_reads_the_pad_id(orc):
+    """Before a sequence's first token the n-gram reads the pad id: position
+    0 of a sequence equals position 1 of the same sequence with the pad id
+    (-1 as a 32-bit token) put in front, for every order whose window ends
+    there -- and sequences do not leak into each other."""
+    rng = np.random.default_rng(43)
+    s = rng.integers(0, 50000, 30)
+    a = orc.engram_rows(s[None], _ORDERS, _K, _SEEDS, _M)
+    padded = np.concatenate([[-1, -1], s])[None]
+    b = orc.engram_rows(padded, _ORDERS, _K, _SEEDS, _M)
+    np.testing.assert_array_equal(a, b[2:])
+    two = orc.engram_rows(np.stack([s, s]), _ORDERS, _K, _SEEDS, _M)
+    np.testing.assert_array_equal(two[:30], two[30:])
+
+
+def test_engram_rows_fill_the_table_evenly(orc):
+    """Distinct bigrams spread over a head's M rows like uniform draws
+    (chi-square statistic within 6 standard deviations of its mean)."""
+    M = 1009
+    tok = np.random.default_rng(44).integers(0, 2 ** 31 - 1, (1, 200000))
+    rows = orc.engram_rows(tok, [2], 1, [99], [M])[1:, 0]
+    cnt = np.bincount(rows, minlength=M)
+    exp = len(rows) / M
+    chi2 = float(((cnt - exp) ** 2 / exp).sum())
+    assert abs(chi2 - (M - 1)) < 6 * math.sqrt(2 * (M - 1))
+
+
+def test_engram_heads_hash_independently(orc):
+    """Two heads with the same table size: the same bigrams land in the same
+    row of both about 1/M of the time, as independent hashes would."""
+    M = 1009
+    tok = np.random.default_rng(45).integers(0, 50000, (1, 100000))
+    rows = orc.engram_rows(tok, [2], 2, [5, 6], [M, M])
+    same = np.mean(rows[:, 0] == rows[:, 1] - M)
+    assert abs(same - 1 / M) < 6 * math.sqrt(1 / M / len(rows))
+
+
+def test_engram_gate_closed_forms(orc):
+    """h along e: <RMSNorm(h), RMSNorm(e)> = d, so alpha = sigmoid(sqrt(d));
+    h against e: sigmoid(-sqrt(d)); h orthogonal to e: 1/2.  Large values
+    make the eps of the norm negligible."""
+    d = 64
+    E = np.zeros((3, d))
+    E[0, :] = 300.0
+    E[1, : d // 2] = 500.0
+    E[2, d // 2:] = 500.0
+    rows = np.array([[0], [0], [1]])
+    h = np.stack([np.full(d, 100.0), np.full(d, -100.0), np.r_[np.zeros(d // 2),
+                                                              np.full(d // 2, 100.0)]])
+    r = orc.engram_gate(rows, E, h)
+    sig = lambda z: 1 / (1 + math.exp(-z))
+    np.testing.assert_allclose(r["alpha"], [sig(math.sqrt(d)), sig(-math.sqrt(d)), 0.5],
+                               rtol=1e-9)
+    np.testing.assert_allclose(r["v"], r["alpha"][:, None] * r["e"], rtol=1e-15)
+
+
+def test_engram_gate_matches_library(orc):
+    """torch's embedding_bag (sum) and rms_norm in fp64 on random rows."""
+    rng = np.random.default_rng(46)
+    T, HK, d, n_rows = 20, 6, 48, 300
+    E = rng.normal(size=(n_rows, d))
+    rows = rng.integers(0, n_rows, (T, HK))
+    h = rng.normal(size=(T, d))
+    r = orc.engram_gate(rows, E, h)
+    Et = torch.tensor(E)
+    e = torch.nn.functional.embedding_bag(torch.tensor(rows), Et, mode="sum")
+    ht = torch.tensor(h)
+    nh = torch.nn.functional.rms_norm(ht, (d,), eps=orc.ENGRAM_EPS)
+    ne = torch.nn.functional.rms_norm(e, (d,), eps=orc.ENGRAM_EPS)
+    alpha = torch.sigmoid((nh * ne).sum(-1) / math.sqrt(d))
+    np.testing.assert_allclose(r["e"], e.numpy(), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(r["alpha"], alpha.numpy(), rtol=1e-12)
+    np.testing.assert_allclose(r["v"], (alpha[:, None] * e).numpy(), rtol=1e-12, atol=1e-13)
