@@ -44,7 +44,8 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default="pkm",
-                   choices=["pkm", "memplus", "tiny", "decode", "train", "memplus_train"])
+                   choices=["pkm", "memplus", "tiny", "decode", "train", "memplus_train",
+                            "engram"])
     p.add_argument("--graph", action="store_true",
                    help="capture one step in a CUDA graph and replay it (default for decode)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -547,6 +548,166 @@ def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world, backward=None):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4)}
 
 
+# ---------------------------------------------------------- Engram lookup --
+
+def engram_bytes_per_token(w) -> int:
+    """Algorithmic bytes of the Engram lookup per token: one row per head,
+    the hidden-state row, the output row, the gate value and the token id."""
+    b = w.elem_bytes
+    return w.heads * w.d * b + 2 * w.d * b + 4 + 4
+
+
+def run_engram(args, rank, world, local):
+    """The Engram lookup (hash, gather of one row per head, context gate) on
+    the engram workload: one kernel per step, timed with CUDA events."""
+    import sparse_key_value_b200 as skv
+    from sparse_key_value_b200.inputs import ENGRAM, make_engram_inputs
+
+    lib = skv.load()
+    w = ENGRAM.scaled(seed=ENGRAM.seed + 7919 * rank)  # own tokens per rank, same tables
+    inp = make_engram_inputs(w, "cuda")
+    T, d = w.T, w.d
+    v = torch.empty(T, d, dtype=w.torch_dtype, device="cuda")
+    alpha = torch.empty(T, dtype=torch.float32, device="cuda")
+    od = (skv.ctypes.c_int32 * len(w.orders))(*w.orders)
+    sd = (skv.ctypes.c_uint64 * w.heads)(*w.seeds)
+    md = (skv.ctypes.c_int64 * w.heads)(*w.rows_per_head)
+    cp = lambda a: skv.ctypes.cast(a, skv.ctypes.c_void_p)  # noqa: E731
+    eargs = skv._lib.EngramArgs(w.n_seq, w.L, len(w.orders), w.K, cp(od), cp(sd), cp(md), d,
+                                1 if w.dtype == "bf16" else 0, skv._p(inp["tokens"]),
+                                skv._p(inp["table"]), skv._p(inp["h"]), skv._p(v),
+                                skv._p(alpha), None, None)
+    stream = torch.cuda.current_stream()
+    sptr = skv.ctypes.c_void_p(stream.cuda_stream)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step():
+        skv.check(lib.pkm_engram_forward(skv.ctypes.byref(eargs), sptr), "pkm_engram_forward")
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert skv.device_error() == 0
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = lib.pkm_launch_count()
+    with Clocks(local) as clk:
+        for e0, e1 in ev:
+            flush.zero_()  # L2 flush between timed steps (outside the events)
+            e0.record()
+            step()
+            e1.record()
+        torch.cuda.synchronize()
+    launches = lib.pkm_launch_count() - launches0
+    barrier(world)
+    ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    total_ms = max_over_ranks(sum(ms), world)
+    ms_per_step = total_ms / K
+    value = whole_job_tokens_per_s(T, world, ms_per_step)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    per_launch = engram_bytes_per_token(w) * T
+    kern_ms = statistics.mean(ms)  # one launch per step: the step is the kernel
+    achieved = per_launch / (kern_ms / 1e3) / 1e9
+    roof = {"kernel": "engram_kernel (hash + gather + context gate)", "bound": "hbm",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_bytes_per_launch": per_launch, "traffic": None,
+            "kernel_us": round(kern_ms * 1e3, 2)}
+
+    e2e = None
+    if not args.no_e2e:
+        htok = inp["tokens"].cpu().pin_memory()
+        hh = inp["h"].cpu().pin_memory()
+        hv = torch.empty(v.shape, dtype=v.dtype).pin_memory()
+        ha = torch.empty(alpha.shape, dtype=alpha.dtype).pin_memory()
+        tok_d, h_d = torch.empty_like(inp["tokens"]), torch.empty_like(inp["h"])
+
+        def e2e_step():
+            tok_d.copy_(htok, non_blocking=True)
+            h_d.copy_(hh, non_blocking=True)
+            r = skv.engram_forward(tok_d, inp["table"], h_d, w.orders, w.K, w.seeds,
+                                   w.rows_per_head, out=v)
+            hv.copy_(r["v"], non_blocking=True)
+            ha.copy_(r["alpha"], non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        tot = 0.0
+        barrier(world)
+        for _ in range(K):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            e2e_step()
+            e1.record()
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        tot = max_over_ranks(tot, world)
+        e2e = {"value": round(world * T / (tot / K / 1e3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": htok.numel() * 4 + hh.numel() * hh.element_size(),
+               "d2h_bytes_per_step": hv.numel() * hv.element_size() + ha.numel() * 4,
+               "ms_per_step": round(tot / K, 4)}
+    assert skv.device_error() == 0
+    res = {
+        "metric": "engram lookup tokens/s", "value": round(value, 1), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded generators; no dataset)",
+        "config": dict(w.describe(), l2="256 MiB L2 flush write before every timed step",
+                       step="forward", parallelism=f"replicas x{world}: one token batch per "
+                                                   f"GPU, tables replicated"),
+        "roofline": roof, "clocks": clk.summary(), "gpu_launches": int(launches), "e2e": e2e,
+    }
+    return res, w, inp
+
+
+def engram_oracle_seconds(w, inp, tokens, min_seconds: float = 0.0):
+    """Seconds of oracle work per pass over ``tokens`` for the Engram
+    lookup: the hashed rows of the whole batch (scaled to the sample) plus
+    the gate of the sampled tokens, repeated until ``min_seconds`` of work
+    have been timed.  Table rows are fetched from the device once, before
+    the timing.  Returns (seconds per pass, threads)."""
+    import numpy as np
+
+    import oracle
+
+    tok = inp["tokens"].cpu().numpy()
+    rows = oracle.engram_rows(tok, w.orders, w.K, w.seeds, w.rows_per_head)
+    sel = rows[np.asarray(tokens)]
+    uniq, inv = np.unique(sel, return_inverse=True)
+    E = inp["table"][torch.from_numpy(uniq).to(inp["table"].device)].cpu()
+    h = inp["h"][torch.as_tensor(tokens).to(inp["h"].device)].cpu()
+    inv = inv.reshape(sel.shape)
+    passes, secs = 0, 0.0
+    while passes == 0 or secs < min_seconds:
+        t0 = time.perf_counter()
+        oracle.engram_rows(tok, w.orders, w.K, w.seeds, w.rows_per_head)
+        t_rows = (time.perf_counter() - t0) * len(tokens) / w.T
+        t0 = time.perf_counter()
+        oracle.engram_gate(inv, E, h)
+        secs += t_rows + time.perf_counter() - t0
+        passes += 1
+    return secs / passes, oracle.num_threads()
+
+
+def engram_cpu_baseline(args, w, inp):
+    import oracle
+
+    oracle.build()
+    tokens = list(range(w.T))
+    target = args.cpu_seconds / 2
+    per_pass, cores = engram_oracle_seconds(w, inp, tokens, min_seconds=target)
+    return {"value": round(w.T / per_pass, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"all {w.T} tokens of the engram workload, passes repeated for about "
+                      f"{target:.0f} s; fp64 hash + gather + gate ({per_pass:.3f} s per pass)"}
+
+
 # --------------------------------------------------------- oracle timing --
 
 def oracle_tokens_per_s(w, inp, tokens, values_dev):
@@ -604,6 +765,8 @@ def run_reference(args, rank, world):
     from sparse_key_value_b200.inputs import WORKLOADS, make_inputs
 
     oracle.build()
+    if args.workload == "engram":
+        return engram_reference(args, world)
     w = WORKLOADS[args.workload]
     if args.workload == "decode":
         w = w.scaled(T=8)
@@ -633,12 +796,47 @@ def run_reference(args, rank, world):
     }
 
 
+def engram_reference(args, world):
+    """The Engram oracle on the host cores, 256 tokens per step."""
+    from sparse_key_value_b200.inputs import ENGRAM, make_engram_inputs
+
+    w = ENGRAM
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_engram_inputs(w, dev)
+    per_step = 256
+    times, cores = [], 1
+    n = args.warmup + args.steps
+    for i in range(n):
+        tokens = [(j * n + i) * (w.T // (per_step * n)) % w.T for j in range(per_step)]
+        s, cores = engram_oracle_seconds(w, inp, tokens)
+        if i >= args.warmup:
+            times.append(s)
+    sec = sum(times) / len(times)
+    value = per_step / sec
+    return {
+        "impl": "reference", "metric": "engram lookup tokens/s", "value": round(value, 2),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generators; no dataset)",
+        "config": dict(w.describe(), parallelism="host cores of rank 0"),
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cores,
+                         "kind": "oracle", "sample": f"{per_step} tokens per step of the "
+                                                      f"engram workload"},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def main():
     args = parse()
     rank, world, local = dist_setup(args)
     try:
         if args.impl == "reference":
             res = run_reference(args, rank, world)
+        elif args.workload == "engram":
+            res, w, inp = run_engram(args, rank, world, local)
+            res["cpu_baseline"] = engram_cpu_baseline(args, w, inp) \
+                if rank == 0 and world == 1 and not args.no_cpu_baseline else None
         else:
             res, w, inp = run_ours(args, rank, world, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -330,6 +330,55 @@ typedef struct {
 
 PKM_API pkm_status pkm_sparse_optimizer_step(const pkm_sparse_opt_args *args, pkm_stream_t stream);
 
+/*
+ * Engram lookup ("Conditional Memory via Scalable Lookup" review, "희소 검색"
+ * and "핵심 수식" 1-2): hashed n-gram rows, their sum and the context gate.
+ * For token t = s*L + p of sequence s and head j = o*K + k (n = orders[o]):
+ *   g      = tokens[s, p-n+1 .. p], positions before 0 read the pad id
+ *            0xFFFFFFFF; ids are taken as 32 unsigned bits
+ *   hash   h = seeds[j]; for each id x of g, oldest first:
+ *            h ^= x; h *= 0x9E3779B97F4A7C15 (mod 2^64); h ^= h >> 32
+ *   row    = offset_j + h mod rows_per_head[j], offset_j the sum of
+ *            rows_per_head of the heads before j (the heads' tables are
+ *            stacked in one table)
+ *   e_t    = sum over the heads of table[row]          (fp32, head order)
+ *   alpha_t = sigmoid(<RMSNorm(h_t), RMSNorm(e_t)> / sqrt(d)),
+ *            RMSNorm(x) = x / sqrt(mean(x^2) + 1e-6)  (no learned scale)
+ *   v_t    = alpha_t e_t                                (one rounding)
+ * The page names independent hash functions per order and head but not
+ * the functions; the one above is this library's definition.
+ *   tokens [n_seq, L] int32 (device), table [sum rows_per_head, d], h and v
+ *   [T, d] (dtype, device); optional outputs (NULL to skip): alpha [T] fp32,
+ *   rows [T, heads] int32, e [T, d] (dtype).  orders, seeds and
+ *   rows_per_head are HOST arrays read during the call.
+ * Limits: 1 <= n_orders <= 8, orders in 1..8, heads = n_orders*K <= 64,
+ * rows_per_head >= 1 with their sum < 2^31, d a multiple of 8 with
+ * d <= 8192 (bf16) or 4096 (fp32).  Nothing is allocated; no workspace.
+ */
+#define PKM_ENGRAM_MAX_ORDERS 8
+#define PKM_ENGRAM_MAX_HEADS 64
+
+typedef struct {
+    int64_t n_seq;
+    int32_t L;
+    int32_t n_orders;
+    int32_t K;
+    const int32_t *orders;        /* host [n_orders] */
+    const uint64_t *seeds;        /* host [n_orders * K] */
+    const int64_t *rows_per_head; /* host [n_orders * K] */
+    int32_t d;
+    pkm_dtype dtype;
+    const int32_t *tokens;
+    const void *table;
+    const void *h;
+    void *v;
+    float *alpha;
+    int32_t *rows;
+    void *e;
+} pkm_engram_args;
+
+PKM_API pkm_status pkm_engram_forward(const pkm_engram_args *args, pkm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

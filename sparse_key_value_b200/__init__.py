@@ -292,3 +292,37 @@ def sparse_optimizer_step(table, rows, grads, count, lr: float, kind: str = "sgd
     check(load().pkm_sparse_optimizer_step(ctypes.byref(a), _stream(table.device, stream)),
           "pkm_sparse_optimizer_step")
     return table
+
+
+def engram_forward(tokens, table, h, orders, K: int, seeds, rows_per_head, alpha=True,
+                   rows=False, e=False, out=None, stream=None):
+    """Engram lookup (see pkm_engram_forward in include/pkm.h): hashed
+    n-gram rows of the stacked table, their sum e and the context gate.
+
+    tokens [n_seq, L] int32, table [sum(rows_per_head), d], h [T, d] CUDA
+    tensors (T = n_seq * L); orders, seeds and rows_per_head host sequences
+    (head j = o*K + k).  Returns dict(v, alpha, rows, e), the optional ones
+    None unless asked for."""
+    _need_cuda(tokens, table, h, out)
+    if tokens.dtype != torch.int32:
+        raise TypeError("tokens must be int32")
+    n_seq, L = tokens.shape
+    T, d = h.shape
+    if T != n_seq * L or table.shape[1] != d or table.dtype != h.dtype:
+        raise ValueError("shapes: tokens [n_seq, L], h [n_seq*L, d], table [rows, d], one dtype")
+    dev = h.device
+    heads = len(orders) * K
+    od = (ctypes.c_int32 * len(orders))(*orders)
+    sd = (ctypes.c_uint64 * heads)(*[int(x) & (2 ** 64 - 1) for x in seeds])
+    md = (ctypes.c_int64 * heads)(*rows_per_head)
+    v = torch.empty(T, d, dtype=h.dtype, device=dev) if out is None else out
+    a_t = torch.empty(T, dtype=torch.float32, device=dev) if alpha else None
+    r_t = torch.empty(T, heads, dtype=torch.int32, device=dev) if rows else None
+    e_t = torch.empty(T, d, dtype=h.dtype, device=dev) if e else None
+    args = _lib.EngramArgs(n_seq, L, len(orders), K, ctypes.cast(od, ctypes.c_void_p),
+                           ctypes.cast(sd, ctypes.c_void_p), ctypes.cast(md, ctypes.c_void_p),
+                           d, _dt(h), _p(tokens), _p(table), _p(h), _p(v), _p(a_t), _p(r_t),
+                           _p(e_t))
+    check(load().pkm_engram_forward(ctypes.byref(args), _stream(dev, stream)),
+          "pkm_engram_forward")
+    return dict(v=v, alpha=a_t, rows=r_t, e=e_t)

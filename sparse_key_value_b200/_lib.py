@@ -66,12 +66,19 @@ class SparseOptArgs(ctypes.Structure):
                 ("grads", P), ("count", P), ("cap", I64), ("m", P), ("v", P)]
 
 
+class EngramArgs(ctypes.Structure):
+    _fields_ = [("n_seq", I64), ("L", I32), ("n_orders", I32), ("K", I32), ("orders", P),
+                ("seeds", P), ("rows_per_head", P), ("d", I32), ("dtype", ctypes.c_int),
+                ("tokens", P), ("table", P), ("h", P), ("v", P), ("alpha", P), ("rows", P),
+                ("e", P)]
+
+
 EXPORTS = ("pkm_forward_workspace_size", "pkm_forward", "pkm_backward_workspace_size",
            "pkm_backward", "embbag_forward", "embbag_backward_workspace_size",
            "embbag_backward", "pkm_get_device_error", "pkm_status_string", "pkm_version",
            "pkm_launch_count", "pkm_forward_noalloc", "pkm_memplus_backward_workspace_size",
            "pkm_memplus_backward", "pkm_qproj_workspace_size", "pkm_qproj_forward",
-           "pkm_qproj_backward", "pkm_sparse_optimizer_step")
+           "pkm_qproj_backward", "pkm_sparse_optimizer_step", "pkm_engram_forward")
 
 _lib = None
 
@@ -121,6 +128,8 @@ def load(path: str = LIB_PATH):
     lib.pkm_qproj_forward.restype = ctypes.c_int
     lib.pkm_qproj_backward.argtypes = [QA, P]
     lib.pkm_qproj_backward.restype = ctypes.c_int
+    lib.pkm_engram_forward.argtypes = [ctypes.POINTER(EngramArgs), P]
+    lib.pkm_engram_forward.restype = ctypes.c_int
     lib.pkm_sparse_optimizer_step.argtypes = [ctypes.POINTER(SparseOptArgs), P]
     lib.pkm_sparse_optimizer_step.restype = ctypes.c_int
     if path == LIB_PATH:

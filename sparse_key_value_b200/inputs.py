@@ -22,6 +22,12 @@ measured on; all data is synthetic, no dataset is involved):
 * ``memplus_train``  the ``memplus`` shapes and tables plus an upstream
                gradient of the layer output (the Memory+ training step).
 * ``decode``   8 tokens per step x 256 steps against the ``memplus`` tables.
+* ``engram``   (``EngramWorkload``) the hashed n-gram lookup: 8 sequences x
+               2048 tokens, 2- and 3-grams with 4 hash heads each, one table
+               per head of 1,048,573 .. 1,048,433 rows (the eight largest
+               primes below 2^20; 8.4 M rows x 1024 bf16 = 17 GB stacked),
+               token ids uniform over 2^17 (so rows are spread over the
+               tables; text would repeat n-grams), hidden state N(0,1).
 
 Distributions: queries N(0,1); sub-keys N(0, std 1/sqrt(d_half)); values
 N(0, std 0.02); x N(0,1); W1, W2 N(0, std 1/sqrt(1024)); upstream gradient
@@ -213,3 +219,81 @@ def random_bags(n_bags: int, B: int, n_rows: int, seed: int,
     wt = torch.rand(n_bags, B, generator=g, dtype=torch.float32) + 0.05
     wt = wt / wt.sum(dim=1, keepdim=True)
     return idx.to(torch.int32), wt
+
+
+# ------------------------------------------------------------ Engram --
+
+@dataclasses.dataclass(frozen=True)
+class EngramWorkload:
+    name: str
+    n_seq: int
+    L: int
+    orders: tuple
+    K: int
+    rows_per_head: tuple
+    d: int
+    dtype: str = "bf16"
+    vocab: int = 1 << 17
+    seed: int = 2001        # tokens and hidden state
+    table_seed: int = 2003  # the stacked table and the hash seeds
+
+    @property
+    def T(self) -> int:
+        return self.n_seq * self.L
+
+    @property
+    def heads(self) -> int:
+        return len(self.orders) * self.K
+
+    @property
+    def n_rows(self) -> int:
+        return int(sum(self.rows_per_head))
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    @property
+    def elem_bytes(self) -> int:
+        return 2 if self.dtype == "bf16" else 4
+
+    @property
+    def seeds(self) -> tuple:
+        """One 64-bit hash seed per head, drawn from the workload seed."""
+        g = _cpu_gen(self.table_seed + 1)
+        return tuple(int(x) for x in torch.randint(0, 2 ** 62, (self.heads,), generator=g))
+
+    def scaled(self, **kw) -> "EngramWorkload":
+        return dataclasses.replace(self, **kw)
+
+    def describe(self) -> dict:
+        return dict(workload=self.name, n_seq=self.n_seq, L=self.L, tokens=self.T,
+                    orders=list(self.orders), hashes_per_order=self.K, d=self.d,
+                    table_rows=self.n_rows, dtype=self.dtype)
+
+
+ENGRAM = EngramWorkload("engram", n_seq=8, L=2048, orders=(2, 3), K=4,
+                        rows_per_head=(1048573, 1048571, 1048559, 1048549, 1048517, 1048507,
+                                       1048447, 1048433), d=1024)
+
+
+def make_engram_inputs(w: EngramWorkload, device="cpu") -> dict:
+    """tokens int32 [n_seq, L] uniform over the vocabulary, the stacked
+    table [n_rows, d] N(0, 0.02) and the hidden state h [T, d] N(0, 1)."""
+    device = torch.device(device)
+    tok = torch.randint(0, w.vocab, (w.n_seq, w.L), generator=_cpu_gen(w.seed),
+                        dtype=torch.int64).to(torch.int32)
+    h = _randn((w.T, w.d), 1.0, _cpu_gen(w.seed + 1)).to(w.torch_dtype)
+    table = torch.empty(w.n_rows, w.d, dtype=w.torch_dtype, device=device)
+    if device.type == "cpu" or w.n_rows * w.d * w.elem_bytes <= _DEVICE_GEN_BYTES:
+        table.copy_(_randn((w.n_rows, w.d), 0.02, _cpu_gen(w.table_seed + 7)))
+    else:
+        g = torch.Generator(device=device)
+        g.manual_seed(w.table_seed + 7)
+        chunk = max(1, (32 << 20) // w.d)
+        for r0 in range(0, w.n_rows, chunk):
+            r1 = min(w.n_rows, r0 + chunk)
+            tmp = torch.randn(r1 - r0, w.d, generator=g, device=device, dtype=torch.float32)
+            table[r0:r1].copy_(tmp.mul_(0.02))
+            del tmp
+    return dict(tokens=tok.to(device), table=table, h=h.to(device))

@@ -181,3 +181,48 @@ def test_sparse_optimizer_validation(lib):
     a = args(kind=1)
     a.m = None
     assert lib.pkm_sparse_optimizer_step(ctypes.byref(a), None) == 1
+
+
+def _engram(**kw):
+    from sparse_key_value_b200 import _lib
+    orders = (ctypes.c_int32 * 2)(2, 3)
+    seeds = (ctypes.c_uint64 * 4)(1, 2, 3, 4)
+    M = (ctypes.c_int64 * 4)(7, 11, 13, 17)
+    fake = ctypes.c_void_p(1 << 20)
+    base = dict(n_seq=2, L=8, n_orders=2, K=2, orders=ctypes.cast(orders, ctypes.c_void_p),
+                seeds=ctypes.cast(seeds, ctypes.c_void_p), rows_per_head=ctypes.cast(M, ctypes.c_void_p),
+                d=64, dtype=1, tokens=fake, table=fake, h=fake, v=fake, alpha=None, rows=None,
+                e=None)
+    base.update(kw)
+    a = _lib.EngramArgs(**base)
+    a._keep = (orders, seeds, M)
+    return a
+
+
+@pytest.mark.parametrize("bad", [dict(n_orders=0), dict(n_orders=9), dict(K=0), dict(K=65),
+                                 dict(L=0), dict(n_seq=-1), dict(d=12), dict(d=8200),
+                                 dict(dtype=5), dict(orders=None), dict(seeds=None),
+                                 dict(rows_per_head=None), dict(table=None), dict(h=None),
+                                 dict(v=None), dict(tokens=ctypes.c_void_p((1 << 20) + 2)),
+                                 dict(table=ctypes.c_void_p((1 << 20) + 8)),
+                                 dict(alpha=ctypes.c_void_p((1 << 20) + 2))])
+def test_engram_rejects_bad_args(lib, bad):
+    a = _engram(**bad)
+    assert lib.pkm_engram_forward(ctypes.byref(a), None) == 1
+
+
+def test_engram_rejects_bad_head_config(lib):
+    orders = (ctypes.c_int32 * 2)(2, 9)  # order 9 > 8
+    a = _engram(orders=ctypes.cast(orders, ctypes.c_void_p))
+    assert lib.pkm_engram_forward(ctypes.byref(a), None) == 1
+    M = (ctypes.c_int64 * 4)(7, 0, 13, 17)  # an empty head table
+    a = _engram(rows_per_head=ctypes.cast(M, ctypes.c_void_p))
+    assert lib.pkm_engram_forward(ctypes.byref(a), None) == 1
+    M = (ctypes.c_int64 * 4)(1 << 30, 1 << 30, 13, 17)  # 2^31 rows in total
+    a = _engram(rows_per_head=ctypes.cast(M, ctypes.c_void_p))
+    assert lib.pkm_engram_forward(ctypes.byref(a), None) == 1
+
+
+def test_engram_empty_batch_is_ok_without_gpu(lib):
+    a = _engram(n_seq=0)
+    assert lib.pkm_engram_forward(ctypes.byref(a), None) == 0
