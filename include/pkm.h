@@ -145,6 +145,18 @@ PKM_API size_t pkm_forward_workspace_size(const pkm_fwd_args *args);
 PKM_API pkm_status pkm_forward(const pkm_fwd_args *args, pkm_stream_t stream);
 
 /*
+ * The selection alone (norms, sub-key scores, per-half top-k, k x k combine,
+ * softmax): writes idx and weights as pkm_forward does; values, out, x, W1,
+ * W2, y_out and d_model are ignored (d_v is only validated).  The workspace
+ * is that of pkm_forward for the same arguments.  It is the first step of a
+ * lookup whose value table is sharded by rows across GPUs: every rank
+ * selects for its own tokens with the replicated sub-keys, the selections
+ * are exchanged and each rank gathers the rows it holds
+ * (embbag_forward_range).
+ */
+PKM_API pkm_status pkm_select(const pkm_fwd_args *args, pkm_stream_t stream);
+
+/*
  * Backward of the plain lookup (out = y), selection held fixed (top-k is
  * piecewise constant).  With w = softmax(S):
  *   dw_j      = <dy_t, values[idx_j]>
@@ -188,6 +200,24 @@ typedef struct {
 
 PKM_API size_t pkm_backward_workspace_size(const pkm_bwd_args *args);
 PKM_API pkm_status pkm_backward(const pkm_bwd_args *args, pkm_stream_t stream);
+
+/*
+ * Partial bags over one shard of a table sharded by rows ("Memory Layers at
+ * Scale" digest: memories of 64B and 128B parameters exceed one GPU): the
+ * shard holds rows [row_lo, row_lo + n_local) of the full table as its own
+ * [n_local, d] table.
+ *   out[t] = sum over j with row_lo <= idx[t,j] < row_lo + n_local of
+ *            w[t,j] * table[idx[t,j] - row_lo]
+ *   idx int32 / w fp32 [n_bags, B] (full-table ids), out fp32 [n_bags, d].
+ * Ids outside the shard contribute nothing and are not an error (another
+ * shard holds them).  fp32 accumulation in j order, no rounding, so the
+ * shards' partials sum (in shard order) to the full bag up to the order of
+ * fp32 additions.
+ */
+PKM_API pkm_status embbag_forward_range(const void *table, int64_t row_lo, int64_t n_local,
+                                        int32_t d, pkm_dtype dtype, const int32_t *idx,
+                                        const float *w, int64_t n_bags, int32_t B, float *out,
+                                        pkm_stream_t stream);
 
 /*
  * Generic weighted bags ("병렬 EmbeddingBag 구현"):

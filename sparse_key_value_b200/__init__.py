@@ -326,3 +326,43 @@ def engram_forward(tokens, table, h, orders, K: int, seeds, rows_per_head, alpha
     check(load().pkm_engram_forward(ctypes.byref(args), _stream(dev, stream)),
           "pkm_engram_forward")
     return dict(v=v, alpha=a_t, rows=r_t, e=e_t)
+
+
+def pkm_select(query, subkeys, k: int, d_v: int = 8, idx=None, weights=None, workspace=None,
+               stream=None):
+    """The selection alone (see pkm_select in include/pkm.h): returns (idx,
+    weights) [T, H, k] as pkm_forward would."""
+    _need_cuda(query, subkeys)
+    T, H, two, dh = query.shape
+    n = subkeys.shape[2]
+    dev = query.device
+    if idx is None:
+        idx = torch.empty(T, H, k, dtype=torch.int32, device=dev)
+    if weights is None:
+        weights = torch.empty(T, H, k, dtype=torch.float32, device=dev)
+    a = fwd_args(T, H, dh, n, k, d_v, _dt(query), 0, False, query=_p(query),
+                 subkeys=_p(subkeys), idx=_p(idx), weights=_p(weights))
+    lib = load()
+    need = int(lib.pkm_forward_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    a.workspace, a.workspace_bytes = _p(workspace), workspace.numel()
+    check(lib.pkm_select(ctypes.byref(a), _stream(dev, stream)), "pkm_select")
+    return idx, weights
+
+
+def embbag_forward_range(table_shard, row_lo: int, idx, w, out=None, stream=None):
+    """Partial bags over one row shard (see embbag_forward_range in
+    include/pkm.h): table_shard holds rows [row_lo, row_lo + len) of the full
+    table; idx int32 / w fp32 [n_bags, B] hold full-table ids; returns fp32
+    [n_bags, d]."""
+    _need_cuda(table_shard, idx, w, out)
+    n_bags, B = idx.shape
+    d = table_shard.shape[1]
+    if out is None:
+        out = torch.empty(n_bags, d, dtype=torch.float32, device=table_shard.device)
+    check(load().embbag_forward_range(_p(table_shard), row_lo, table_shard.shape[0], d,
+                                      _dt(table_shard), _p(idx), _p(w), n_bags, B, _p(out),
+                                      _stream(table_shard.device, stream)),
+          "embbag_forward_range")
+    return out

@@ -78,7 +78,8 @@ EXPORTS = ("pkm_forward_workspace_size", "pkm_forward", "pkm_backward_workspace_
            "embbag_backward", "pkm_get_device_error", "pkm_status_string", "pkm_version",
            "pkm_launch_count", "pkm_forward_noalloc", "pkm_memplus_backward_workspace_size",
            "pkm_memplus_backward", "pkm_qproj_workspace_size", "pkm_qproj_forward",
-           "pkm_qproj_backward", "pkm_sparse_optimizer_step", "pkm_engram_forward")
+           "pkm_qproj_backward", "pkm_sparse_optimizer_step", "pkm_engram_forward",
+           "pkm_select", "embbag_forward_range")
 
 _lib = None
 
@@ -94,6 +95,10 @@ def load(path: str = LIB_PATH):
     FA, BA = ctypes.POINTER(FwdArgs), ctypes.POINTER(BwdArgs)
     lib.pkm_forward_workspace_size.argtypes = [FA]
     lib.pkm_forward_workspace_size.restype = SZ
+    lib.pkm_select.argtypes = [FA, P]
+    lib.pkm_select.restype = ctypes.c_int
+    lib.embbag_forward_range.argtypes = [P, I64, I64, I32, ctypes.c_int, P, P, I64, I32, P, P]
+    lib.embbag_forward_range.restype = ctypes.c_int
     lib.pkm_forward.argtypes = [FA, P]
     lib.pkm_forward.restype = ctypes.c_int
     lib.pkm_backward_workspace_size.argtypes = [BA]

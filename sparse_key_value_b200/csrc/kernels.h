@@ -55,6 +55,12 @@ cudaError_t launch_embbag_fwd(const void* table, int64_t n_rows, int d, pkm_dtyp
 // The same gather for small batches (see k_embbag_split.cu): fp32 partial
 // sums of row groups in `part` (embbag_split_workspace bytes), then an
 // ordered reduction.
+// Partial bags of one shard of a row-sharded table: fp32 out [n_bags, d];
+// only ids in [row_lo, row_lo + n_local) contribute (read at id - row_lo).
+cudaError_t launch_embbag_range(const void* table, int64_t row_lo, int64_t n_local, int d,
+                                pkm_dtype dt, const int32_t* idx, const float* w, int64_t n_bags,
+                                int B, float* out, cudaStream_t stream);
+
 constexpr int64_t kSplitGatherMaxBags = 64;
 size_t embbag_split_workspace(int64_t n_bags, int B, int d);
 cudaError_t launch_embbag_fwd_split(const void* table, int64_t n_rows, int d, pkm_dtype dt,

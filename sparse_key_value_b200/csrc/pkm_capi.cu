@@ -112,7 +112,8 @@ static void mark(const pkm_fwd_args* a, int i, cudaStream_t st) {
     cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), st);
 }
 
-static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
+static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
+                               bool select_only = false) {
   int32_t* status = status_ptr();
   if (!status) return PKM_ERR_CUDA;
   const FwdLayout L = fwd_layout(a);
@@ -148,6 +149,7 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   // a4 + a5: k x k combine, top-k, softmax
   PKM_TRY(launch_combine(hv, hi, L.splits, T, H, n, k, a->idx, a->weights, st));
   mark(a, 3, st);
+  if (select_only) return PKM_OK;
   // (a7) gate GEMM, a6 bag gather over the H*k selected rows of each token
   if (mp) {
     PKM_TRY(launch_transpose_bf16(a->W1, dm, dv, w1t, st));  // [dv, dm]
@@ -169,6 +171,33 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st) {
   mark(a, 5, st);
   if (mp) PKM_TRY(launch_gemm_bf16(z, w2t, T, dm, dv, /*none*/ 0, a->out, status, st));
   mark(a, 6, st);
+  return PKM_OK;
+}
+
+// Arguments of a selection-only call: the forward's, without the value table,
+// the output and Memory+ (those fields are ignored).
+static pkm_fwd_args select_args(const pkm_fwd_args* a) {
+  pkm_fwd_args b = *a;
+  b.x = b.W1 = b.W2 = nullptr;
+  b.y_out = nullptr;
+  b.d_model = 0;
+  return b;
+}
+
+static pkm_status validate_select(const pkm_fwd_args* b) {
+  if (b->T < 0 || b->H < 1 || b->n_sub < 1 || b->k < 1 || b->k > 64 || b->k > b->n_sub)
+    return PKM_ERR_INVALID_ARG;
+  if (b->d_half < 8 || b->d_half % 8 || b->d_v < 8 || b->d_v % 8) return PKM_ERR_INVALID_ARG;
+  if ((int64_t)b->n_sub * b->n_sub >= (int64_t(1) << 31)) return PKM_ERR_INVALID_ARG;
+  if (b->dtype != PKM_F32 && b->dtype != PKM_BF16) return PKM_ERR_INVALID_ARG;
+  if (b->H * b->k > 4096) return PKM_ERR_INVALID_ARG;
+  if (b->d_half > 2048) return PKM_ERR_UNSUPPORTED;
+  if (b->T == 0) return PKM_OK;
+  const void* need[] = {b->query, b->subkeys, b->idx, b->weights};
+  for (const void* p : need)
+    if (!p || !aligned16(p)) return PKM_ERR_INVALID_ARG;
+  if (!b->workspace || !aligned16(b->workspace) || b->workspace_bytes < fwd_layout(b).total)
+    return PKM_ERR_WORKSPACE;
   return PKM_OK;
 }
 
@@ -198,6 +227,14 @@ size_t pkm_forward_workspace_size(const pkm_fwd_args* args) {
   return fwd_layout(args).total;
 }
 
+pkm_status pkm_select(const pkm_fwd_args* args, pkm_stream_t stream) {
+  if (!args) return PKM_ERR_INVALID_ARG;
+  const pkm_fwd_args b = select_args(args);
+  pkm_status s = validate_select(&b);
+  if (s != PKM_OK || b.T == 0) return s;
+  return forward_impl(&b, reinterpret_cast<cudaStream_t>(stream), /*select_only*/ true);
+}
+
 pkm_status pkm_forward(const pkm_fwd_args* args, pkm_stream_t stream) {
   pkm_status s = validate_fwd(args);
   if (s != PKM_OK || args->T == 0) return s;
@@ -219,6 +256,21 @@ pkm_status embbag_forward(const void* table, int64_t n_rows, int32_t d, pkm_dtyp
   cudaError_t e = launch_embbag_fwd(table, n_rows, d, dtype, idx, w, n_bags, B, gate, out,
                                     status, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
+}
+
+pkm_status embbag_forward_range(const void* table, int64_t row_lo, int64_t n_local, int32_t d,
+                                pkm_dtype dtype, const int32_t* idx, const float* w,
+                                int64_t n_bags, int32_t B, float* out, pkm_stream_t stream) {
+  if (n_bags < 0 || row_lo < 0 || n_local < 1 || d < 8 || d % 8 || B < 1 || B > 4096)
+    return PKM_ERR_INVALID_ARG;
+  if (dtype != PKM_F32 && dtype != PKM_BF16) return PKM_ERR_INVALID_ARG;
+  if (n_bags == 0) return PKM_OK;
+  if (!table || !idx || !w || !out || !aligned16(table) || !aligned16(out))
+    return PKM_ERR_INVALID_ARG;
+  return launch_embbag_range(table, row_lo, n_local, d, dtype, idx, w, n_bags, B, out,
+                             reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PKM_OK
+             : PKM_ERR_CUDA;
 }
 
 pkm_status pkm_get_device_error(pkm_stream_t stream, int32_t* code) {

@@ -1,0 +1,95 @@
+"""The lookup over a value table sharded by rows across ranks.
+
+"Memory Layers at Scale" digest: memories of 64B and 128B parameters do not
+fit one GPU's memory, so the value table is split by row id across the
+ranks (contiguous ranges, ``shard_rows``) while the sub-keys, which are
+small, stay replicated.  Per step, with every rank holding T tokens:
+
+1. each rank selects the rows of its own tokens (``pkm_select``, the
+   replicated sub-keys);
+2. the selections (ids and weights, H*k per token) are all-gathered;
+3. each rank sums, for the tokens of every rank, the selected rows it holds
+   (``embbag_forward_range``, fp32 partial bags of world*T tokens);
+4. a reduce-scatter over tokens sums the partials and hands each rank the
+   bags of its own tokens (fp32, summed in rank order by the collective).
+
+The exchange is one all-gather of T*H*k*8 bytes and one reduce-scatter of
+world*T*d_v*4 bytes per rank, instead of moving value rows: a row is read
+from HBM once, by its owner.  This module only orders the steps; every
+step's arithmetic runs in the CUDA library (steps 1 and 3) or in the
+collective (step 4).  ``comm`` is any object with ``all_gather(t) ->
+[world, *t.shape]`` and ``reduce_scatter_sum(t [world*T, d]) -> [T, d]``;
+``TorchComm`` wraps ``torch.distributed``.
+"""
+
+from __future__ import annotations
+
+import torch
+
+
+def shard_rows(n_rows: int, world: int, rank: int):
+    """(first row, number of rows) of rank's contiguous share of a table of
+    n_rows rows: ceil(n_rows / world) rows each, the last share shorter."""
+    per = -(-n_rows // world)
+    lo = min(n_rows, rank * per)
+    return lo, max(0, min(n_rows, lo + per) - lo)
+
+
+class TorchComm:
+    """The two collectives over a torch.distributed process group.  With
+    NCCL they are all_gather_into_tensor and reduce_scatter_tensor; a
+    backend without a reduce-scatter (gloo, used by the host tests) gets an
+    all-reduce followed by taking this rank's block."""
+
+    def __init__(self, group=None):
+        import torch.distributed as dist
+
+        self.dist = dist
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.nccl = dist.get_backend(group) == "nccl"
+
+    def all_gather(self, t: torch.Tensor) -> torch.Tensor:
+        out = torch.empty((self.world,) + tuple(t.shape), dtype=t.dtype, device=t.device)
+        if self.nccl:
+            self.dist.all_gather_into_tensor(out, t.contiguous(), group=self.group)
+        else:
+            self.dist.all_gather(list(out.unbind(0)), t.contiguous(), group=self.group)
+        return out
+
+    def reduce_scatter_sum(self, t: torch.Tensor) -> torch.Tensor:
+        T = t.shape[0] // self.world
+        if self.nccl:
+            out = torch.empty((T,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+            self.dist.reduce_scatter_tensor(out, t.contiguous(), group=self.group)
+            return out
+        s = t.clone()
+        self.dist.all_reduce(s, group=self.group)
+        return s[self.rank * T:(self.rank + 1) * T].clone()
+
+
+def sharded_lookup(query, subkeys, values_shard, k: int, row_lo: int, comm, select=None,
+                   gather=None):
+    """One rank's step of the row-sharded lookup (steps 1-4 above).
+
+    query [T, H, 2, d_half] (this rank's tokens, T equal on every rank),
+    subkeys [H, 2, n_sub, d_half] (replicated), values_shard [n_local, d_v]
+    (rows row_lo .. of the full table).  Returns (y fp32 [T, d_v], idx,
+    weights).  ``select`` / ``gather`` default to the CUDA library's
+    pkm_select / embbag_forward_range."""
+    if select is None or gather is None:
+        import sparse_key_value_b200 as skv
+
+        select = select or (lambda q, K, kk: skv.pkm_select(q, K, kk, d_v=values_shard.shape[1]))
+        gather = gather or skv.embbag_forward_range
+    T, H = query.shape[0], query.shape[1]
+    idx, w = select(query, subkeys, k)
+    all_idx = comm.all_gather(idx.reshape(T, H * k)).reshape(-1, H * k)
+    all_w = comm.all_gather(w.reshape(T, H * k)).reshape(-1, H * k)
+    if values_shard.shape[0] > 0:
+        part = gather(values_shard, row_lo, all_idx, all_w)
+    else:  # more ranks than rows: this rank holds none
+        part = torch.zeros(all_idx.shape[0], values_shard.shape[1], dtype=torch.float32,
+                           device=values_shard.device)
+    return comm.reduce_scatter_sum(part), idx, w

@@ -226,3 +226,35 @@ def test_engram_rejects_bad_head_config(lib):
 def test_engram_empty_batch_is_ok_without_gpu(lib):
     a = _engram(n_seq=0)
     assert lib.pkm_engram_forward(ctypes.byref(a), None) == 0
+
+
+def test_select_validation(lib):
+    a = _fwd()
+    a.values = None  # the selection needs no value table nor output
+    a.out = None
+    a.workspace_bytes = 1 << 40
+    bad = _fwd(k=0)
+    bad.workspace_bytes = 1 << 40
+    assert lib.pkm_select(ctypes.byref(bad), None) == 1
+    nq = _fwd()
+    nq.query = None
+    nq.workspace_bytes = 1 << 40
+    assert lib.pkm_select(ctypes.byref(nq), None) == 1
+    small = _fwd()
+    small.workspace_bytes = 16
+    assert lib.pkm_select(ctypes.byref(small), None) == 6
+    empty = _fwd(T=0)
+    assert lib.pkm_select(ctypes.byref(empty), None) == 0
+
+
+def test_embbag_range_validation(lib):
+    f = ctypes.c_void_p(1 << 20)
+    ok = dict(table=f, row_lo=0, n_local=10, d=16, dtype=1, idx=f, w=f, n_bags=0, B=4, out=f)
+    call = lambda **kw: lib.embbag_forward_range(*{**ok, **kw}.values(), None)  # noqa: E731
+    assert call() == 0                       # empty batch, no launch
+    assert call(n_bags=1, row_lo=-1) == 1
+    assert call(n_bags=1, n_local=0) == 1
+    assert call(n_bags=1, d=12) == 1
+    assert call(n_bags=1, B=0) == 1
+    assert call(n_bags=1, table=None) == 1
+    assert call(n_bags=1, out=ctypes.c_void_p((1 << 20) + 4)) == 1
