@@ -51,6 +51,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--engram-rows", type=int, default=0,
+                   help="engram workload: rows per head table (0: the workload's own, about "
+                        "2^20; smaller tables for profiling captures)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="target CPU time of the oracle baseline sample")
     return p.parse_args()
@@ -565,6 +568,8 @@ def run_engram(args, rank, world, local):
 
     lib = skv.load()
     w = ENGRAM.scaled(seed=ENGRAM.seed + 7919 * rank)  # own tokens per rank, same tables
+    if args.engram_rows > 0:
+        w = w.scaled(rows_per_head=(args.engram_rows,) * w.heads)
     inp = make_engram_inputs(w, "cuda")
     T, d = w.T, w.d
     v = torch.empty(T, d, dtype=w.torch_dtype, device="cuda")

@@ -35,6 +35,7 @@ struct EngramCfg {
   int order[PKM_ENGRAM_MAX_ORDERS];
   uint64_t seed[PKM_ENGRAM_MAX_HEADS];
   uint64_t M[PKM_ENGRAM_MAX_HEADS];
+  uint64_t R[PKM_ENGRAM_MAX_HEADS];  // floor((2^64 - 1) / M): h mod M by multiply-high
   int64_t offset[PKM_ENGRAM_MAX_HEADS];
 };
 
@@ -75,7 +76,13 @@ __global__ void __launch_bounds__(kEngramThreads, NCH == 1 ? 10 : (NCH == 2 ? 6 
       x *= kEngramMul;
       x ^= x >> 32;
     }
-    const int64_t r = cfg.offset[tid] + (int64_t)(x % cfg.M[tid]);
+    // x mod M without a 64-bit division: q = floor(x R / 2^64) undershoots
+    // floor(x / M) by at most 2, so at most two subtractions remain
+    const uint64_t M = cfg.M[tid];
+    uint64_t rem = x - __umul64hi(x, cfg.R[tid]) * M;
+    if (rem >= M) rem -= M;
+    if (rem >= M) rem -= M;
+    const int64_t r = cfg.offset[tid] + (int64_t)rem;
     s_rows[tid] = (int32_t)r;
     if (rows_out) rows_out[t * cfg.heads + tid] = (int32_t)r;
   }
@@ -221,6 +228,7 @@ PKM_API pkm_status pkm_engram_forward(const pkm_engram_args* a, pkm_stream_t str
     if (a->rows_per_head[j] < 1) return PKM_ERR_INVALID_ARG;
     cfg.seed[j] = a->seeds[j];
     cfg.M[j] = (uint64_t)a->rows_per_head[j];
+    cfg.R[j] = ~0ull / cfg.M[j];
     cfg.offset[j] = total;
     total += a->rows_per_head[j];
     if (total >= (int64_t(1) << 31)) return PKM_ERR_INVALID_ARG;
