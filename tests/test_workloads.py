@@ -66,3 +66,31 @@ def test_distributions():
     assert abs(inp["query"].float().std().item() - 1.0) < 0.02
     assert abs(inp["subkeys"].float().std().item() - 1 / math.sqrt(512)) < 0.002
     assert abs(inp["values"].float().std().item() - 0.02) < 0.001
+
+
+def test_engram_workload_and_bytes():
+    """The Engram workload's shape and the bench's algorithmic bytes per
+    token: one d-row per head, the hidden-state and output rows, alpha and
+    the token id."""
+    import os
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    from sparse_key_value_b200.inputs import ENGRAM, make_engram_inputs
+
+    w = ENGRAM
+    assert (w.T, w.heads, w.d) == (16384, 8, 1024)
+    assert len(set(w.seeds)) == w.heads and all(0 <= x < 2 ** 64 for x in w.seeds)
+    assert w.n_rows == sum(w.rows_per_head) < 2 ** 31
+    assert bench.engram_bytes_per_token(w) == 8 * 1024 * 2 + 2 * 1024 * 2 + 8
+    small = w.scaled(n_seq=2, L=5, rows_per_head=(11,) * 8, d=16)
+    inp = make_engram_inputs(small, "cpu")
+    assert inp["tokens"].shape == (2, 5) and inp["tokens"].dtype == torch.int32
+    assert inp["table"].shape == (88, 16) and inp["h"].shape == (10, 16)
+    assert int(inp["tokens"].min()) >= 0 and int(inp["tokens"].max()) < small.vocab
+    # the tables and hash seeds depend on the table seed only, the tokens on the seed
+    other = make_engram_inputs(small.scaled(seed=small.seed + 1), "cpu")
+    assert torch.equal(other["table"], inp["table"]) and not torch.equal(other["tokens"],
+                                                                          inp["tokens"])
+    assert small.scaled(seed=small.seed + 1).seeds == small.seeds
