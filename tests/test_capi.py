@@ -229,10 +229,6 @@ def test_engram_empty_batch_is_ok_without_gpu(lib):
 
 
 def test_select_validation(lib):
-    a = _fwd()
-    a.values = None  # the selection needs no value table nor output
-    a.out = None
-    a.workspace_bytes = 1 << 40
     bad = _fwd(k=0)
     bad.workspace_bytes = 1 << 40
     assert lib.pkm_select(ctypes.byref(bad), None) == 1
