@@ -51,6 +51,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--shards", type=int, default=0,
+                   help="pkm workloads: also time the compute of a row-sharded step with this "
+                        "many shards held on one GPU (selection + every shard's partial bags)")
     p.add_argument("--engram-rows", type=int, default=0,
                    help="engram workload: rows per head table (0: the workload's own, about "
                         "2^20; smaller tables for profiling captures)")
@@ -405,6 +408,9 @@ def run_ours(args, rank, world, local):
                 "algorithmic_bytes_per_launch": bytes_per_launch, "traffic": traffic}
         phases = None
     extra = {}
+    if args.shards > 1 and not train and not w.memplus and graph is None:
+        extra["row_sharded_compute"] = time_sharded_compute(skv, inp, w, args.shards, flush,
+                                                            peak, peak_kind)
     if train:
         # the lookup's backward (after the Memory+ part, if any) against HBM
         bwd_ms = statistics.mean([b[2].elapsed_time(b[1]) for b in bev])
@@ -476,6 +482,47 @@ def run_ours(args, rank, world, local):
         "gpu_launches": int(launches), "e2e": e2e, **extra,
     }
     return res, w, inp
+
+
+def time_sharded_compute(skv, inp, w, S, flush, peak, peak_kind, reps=20):
+    """The compute of one row-sharded step with all S shards on this GPU:
+    the selection (pkm_select) and each shard's fp32 partial bags over all
+    tokens (embbag_forward_range); the all-gather and reduce-scatter between
+    them are not timed (they need S GPUs).  Bytes: every selected row read
+    once (by its owner), ids and weights read by every shard, the S fp32
+    partial outputs written."""
+    from sparse_key_value_b200.sharded import shard_rows
+
+    T, B = w.T, w.H * w.k
+    N = inp["values"].shape[0]
+    idx = torch.empty(T, w.H, w.k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(T, w.H, w.k, dtype=torch.float32, device="cuda")
+    parts = torch.empty(S, T, w.d_v, dtype=torch.float32, device="cuda")
+    shares = [shard_rows(N, S, r) for r in range(S)]
+    sel, gat = [], []
+    for i in range(reps + 3):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        skv.pkm_select(inp["query"], inp["subkeys"], w.k, d_v=w.d_v, idx=idx, weights=wts)
+        e[1].record()
+        for r, (lo, n) in enumerate(shares):
+            skv.embbag_forward_range(inp["values"][lo:lo + n], lo, idx.view(T, B),
+                                     wts.view(T, B), out=parts[r])
+        e[2].record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            sel.append(e[0].elapsed_time(e[1]))
+            gat.append(e[1].elapsed_time(e[2]))
+    assert skv.device_error() == 0
+    g_ms = statistics.mean(gat)
+    nbytes = T * B * w.d_v * w.elem_bytes + S * T * B * 8 + S * T * w.d_v * 4
+    return {"shards": S, "select_us": round(statistics.mean(sel) * 1e3, 1),
+            "partial_gathers_us": round(g_ms * 1e3, 1), "algorithmic_bytes": nbytes,
+            "GBps": round(nbytes / (g_ms / 1e3) / 1e9, 1),
+            "frac": round(nbytes / (g_ms / 1e3) / 1e9 / peak, 4),
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "note": "all shards on one GPU; the exchange between the steps is not timed"}
 
 
 def time_sparse_adam(skv, table, rows, grads, count, U, w, peak, peak_kind, reps=10):
