@@ -64,6 +64,8 @@ CASES = [
     ("f32-d4096", 1, 10, (4,), 2, 4096, "f32"),
     ("single-token-sequences", 5, 1, (1, 2, 8), 1, 64, "bf16"),
     ("64-heads", 1, 40, (1, 2, 3, 4, 5, 6, 7, 8), 8, 64, "bf16"),
+    ("d8-one-column", 3, 17, (2, 3), 1, 8, "bf16"),
+    ("unigram-only-f32", 4, 33, (1,), 5, 40, "f32"),
 ]
 
 
@@ -72,6 +74,8 @@ def test_engram_matches_oracle(case):
     name, n_seq, L, orders, K, d, dt = case
     heads = len(orders) * K
     M = tuple(PRIMES[j % len(PRIMES)] + 2 * (j // len(PRIMES)) for j in range(heads))
+    if name == "d8-one-column":
+        M = (1,) + M[1:]  # a one-row head table: every n-gram reads its only row
     w = ENGRAM.scaled(name=name, n_seq=n_seq, L=L, orders=orders, K=K, rows_per_head=M, d=d,
                       dtype=dt, seed=sum(map(ord, name)))
     inp = make_engram_inputs(w, "cuda")

@@ -126,3 +126,27 @@ def test_pkm_workload_over_eight_shards_sampled():
     close(y[sample.cuda()].double().cpu().numpy(), ref, RTOL["f32"], "eight shards")
     del inp
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,d,dt", [(70, 256, "bf16"), (1, 64, "bf16"), (33, 128, "f32"),
+                                    (300, 1024, "bf16")])
+def test_range_gather_odd_bags_against_oracle(B, d, dt):
+    """Bags whose size is not a multiple of the 32-entry compaction step,
+    single-entry bags and fp32 tables, over three uneven shards."""
+    import oracle
+    from sparse_key_value_b200.inputs import random_bags
+
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    n_rows, n_bags = 1001, 45
+    g = torch.Generator().manual_seed(B + d)
+    table = (torch.randn(n_rows, d, generator=g) * 0.02).to(tdt).cuda()
+    idx, w = random_bags(n_bags, B, n_rows, seed=B * 7 + d)
+    idx, w = idx.cuda(), w.cuda()
+    cuts = [0, 13, 600, n_rows]  # uneven shares
+    y = None
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        p = skv.embbag_forward_range(table[lo:hi], lo, idx, w)
+        y = p if y is None else y + p
+    torch.cuda.synchronize()
+    ref = oracle.bag(idx.cpu().numpy().astype(np.int64), w.double().cpu().numpy(), table.cpu())
+    close(y.double().cpu().numpy(), ref, RTOL["f32"], f"B={B} d={d} {dt}")
