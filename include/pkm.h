@@ -409,6 +409,18 @@ typedef struct {
 
 PKM_API pkm_status pkm_engram_forward(const pkm_engram_args *args, pkm_stream_t stream);
 
+/*
+ * Failure-path check of the bounded waits (no counterpart on the pages; a
+ * service for tests and operators): one CTA waits, with the wait every
+ * pipelined kernel of the library uses, on an mbarrier phase that nothing
+ * completes.  After `polls` polls (1 .. 2^20) the wait gives up, the device
+ * status word records PKM_ERR_TIMEOUT (read it with pkm_get_device_error)
+ * and the kernel returns, writing 1 to *done (device int32; 2 would mean the
+ * phase completed, which cannot happen).  No GPU fault is involved and the
+ * context stays usable.
+ */
+PKM_API pkm_status pkm_check_wait_timeout(int64_t polls, int32_t *done, pkm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -366,3 +366,17 @@ def embbag_forward_range(table_shard, row_lo: int, idx, w, out=None, stream=None
                                       _stream(table_shard.device, stream)),
           "embbag_forward_range")
     return out
+
+
+def check_wait_timeout(polls: int = 4096, device=None, stream=None) -> int:
+    """Run the bounded-wait failure path (see pkm_check_wait_timeout in
+    include/pkm.h) and return the device status it left (PKM_ERR_TIMEOUT = 5
+    expected), after checking that the waiting kernel returned."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    done = torch.zeros(1, dtype=torch.int32, device=dev)
+    check(load().pkm_check_wait_timeout(polls, _p(done), _stream(dev, stream)),
+          "pkm_check_wait_timeout")
+    code = device_error(stream, dev)
+    if int(done.item()) != 1:
+        raise RuntimeError(f"the waiting kernel did not finish as expected ({int(done.item())})")
+    return code

@@ -79,7 +79,7 @@ EXPORTS = ("pkm_forward_workspace_size", "pkm_forward", "pkm_backward_workspace_
            "pkm_launch_count", "pkm_forward_noalloc", "pkm_memplus_backward_workspace_size",
            "pkm_memplus_backward", "pkm_qproj_workspace_size", "pkm_qproj_forward",
            "pkm_qproj_backward", "pkm_sparse_optimizer_step", "pkm_engram_forward",
-           "pkm_select", "embbag_forward_range")
+           "pkm_select", "embbag_forward_range", "pkm_check_wait_timeout")
 
 _lib = None
 
@@ -95,6 +95,8 @@ def load(path: str = LIB_PATH):
     FA, BA = ctypes.POINTER(FwdArgs), ctypes.POINTER(BwdArgs)
     lib.pkm_forward_workspace_size.argtypes = [FA]
     lib.pkm_forward_workspace_size.restype = SZ
+    lib.pkm_check_wait_timeout.argtypes = [I64, P, P]
+    lib.pkm_check_wait_timeout.restype = ctypes.c_int
     lib.pkm_select.argtypes = [FA, P]
     lib.pkm_select.restype = ctypes.c_int
     lib.embbag_forward_range.argtypes = [P, I64, I64, I32, ctypes.c_int, P, P, I64, I32, P, P]

@@ -142,11 +142,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.  Returns
-// false (and records PKM_ERR_TIMEOUT) if the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
-  for (unsigned long long i = 0; i < kSpinLimit; ++i)
+// Bounded wait for the phase with the given parity to complete, the one
+// every pipelined kernel uses.  Gives up early (false) once another role of
+// the CTA has set *abort; after `limit` polls it sets *abort itself, records
+// PKM_ERR_TIMEOUT and returns false.  The caller then stops issuing work,
+// lets what it already issued complete (bounded again) and returns.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity,
+                                                   volatile int* abort, int32_t* status,
+                                                   unsigned long long limit = kSpinLimit) {
+  for (unsigned long long i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 255 && *abort) return false;
+  }
+  *abort = 1;
   set_status(status, PKM_ERR_TIMEOUT);
   return false;
 }

@@ -41,13 +41,7 @@ struct GemmCtl {
 
 __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, GemmCtl* ctl,
                                           int32_t* status) {
-  for (unsigned long long i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 255 && ctl->abort) return false;
-  }
-  ctl->abort = 1;
-  set_status(status, PKM_ERR_TIMEOUT);
-  return false;
+  return mbar_wait_or_abort(bar, parity, &ctl->abort, status);
 }
 
 // OUT: 0 bf16 store, 1 fp32 store, 2 fp32 accumulate (C += result)

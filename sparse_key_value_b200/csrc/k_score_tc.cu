@@ -86,13 +86,7 @@ struct ScoreSmemCtl {
 // bounded wait that also gives up when another role of the CTA aborted
 __device__ __forceinline__ bool wait_ctl(uint64_t* bar, uint32_t parity, ScoreSmemCtl* ctl,
                                          int32_t* status) {
-  for (unsigned long long i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 255 && ctl->abort) return false;
-  }
-  ctl->abort = 1;
-  set_status(status, PKM_ERR_TIMEOUT);
-  return false;
+  return mbar_wait_or_abort(bar, parity, &ctl->abort, status);
 }
 
 __device__ __forceinline__ uint32_t ord_f32(float s) {

@@ -254,3 +254,11 @@ def test_embbag_range_validation(lib):
     assert call(n_bags=1, B=0) == 1
     assert call(n_bags=1, table=None) == 1
     assert call(n_bags=1, out=ctypes.c_void_p((1 << 20) + 4)) == 1
+
+
+def test_wait_timeout_check_validation(lib):
+    f = ctypes.c_void_p(1 << 20)
+    assert lib.pkm_check_wait_timeout(0, f, None) == 1
+    assert lib.pkm_check_wait_timeout((1 << 20) + 1, f, None) == 1
+    assert lib.pkm_check_wait_timeout(16, None, None) == 1
+    assert lib.pkm_check_wait_timeout(16, ctypes.c_void_p((1 << 20) + 2), None) == 1
