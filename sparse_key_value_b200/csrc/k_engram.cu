@@ -40,7 +40,7 @@ struct EngramCfg {
 };
 
 template <pkm_dtype DT, int NCH>
-__global__ void __launch_bounds__(kEngramThreads, NCH == 1 ? 12 : (NCH == 2 ? 6 : 2)) engram_kernel(
+__global__ void __launch_bounds__(kEngramThreads, NCH == 1 ? 16 : (NCH == 2 ? 6 : 2)) engram_kernel(
     const __grid_constant__ EngramCfg cfg, int L, const int32_t* __restrict__ tokens,
     const typename Elem<DT>::T* __restrict__ table, int d,
     const typename Elem<DT>::T* __restrict__ h, typename Elem<DT>::T* __restrict__ v,
