@@ -39,6 +39,10 @@ struct EngramCfg {
   int64_t offset[PKM_ENGRAM_MAX_HEADS];
 };
 
+// Resident CTAs per SM: a CTA's loads are in flight only between its hash
+// and its reduction, so as many CTAs as the SM's 2048 threads allow for one
+// column per thread (16 measured faster than 10 and 12 despite a 16-byte
+// spill); wider rows keep their loads in registers.
 template <pkm_dtype DT, int NCH>
 __global__ void __launch_bounds__(kEngramThreads, NCH == 1 ? 16 : (NCH == 2 ? 6 : 2)) engram_kernel(
     const __grid_constant__ EngramCfg cfg, int L, const int32_t* __restrict__ tokens,
