@@ -36,10 +36,10 @@ def shard_rows(n_rows: int, world: int, rank: int):
 
 
 class TorchComm:
-    """The two collectives over a torch.distributed process group.  With
-    NCCL they are all_gather_into_tensor and reduce_scatter_tensor; a
-    backend without a reduce-scatter (gloo, used by the host tests) gets an
-    all-reduce followed by taking this rank's block."""
+    """The two collectives over a torch.distributed process group:
+    all_gather_into_tensor (concatenated along the first dimension) and
+    reduce_scatter_tensor (sum).  The same calls run on NCCL and on gloo, so
+    the host tests exercise the code path the GPUs take."""
 
     def __init__(self, group=None):
         import torch.distributed as dist
@@ -48,25 +48,19 @@ class TorchComm:
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
-        self.nccl = dist.get_backend(group) == "nccl"
 
     def all_gather(self, t: torch.Tensor) -> torch.Tensor:
-        out = torch.empty((self.world,) + tuple(t.shape), dtype=t.dtype, device=t.device)
-        if self.nccl:
-            self.dist.all_gather_into_tensor(out, t.contiguous(), group=self.group)
-        else:
-            self.dist.all_gather(list(out.unbind(0)), t.contiguous(), group=self.group)
-        return out
+        t = t.contiguous()
+        out = torch.empty((self.world * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype,
+                          device=t.device)
+        self.dist.all_gather_into_tensor(out, t, group=self.group)
+        return out.view((self.world,) + tuple(t.shape))
 
     def reduce_scatter_sum(self, t: torch.Tensor) -> torch.Tensor:
         T = t.shape[0] // self.world
-        if self.nccl:
-            out = torch.empty((T,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
-            self.dist.reduce_scatter_tensor(out, t.contiguous(), group=self.group)
-            return out
-        s = t.clone()
-        self.dist.all_reduce(s, group=self.group)
-        return s[self.rank * T:(self.rank + 1) * T].clone()
+        out = torch.empty((T,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+        self.dist.reduce_scatter_tensor(out, t.contiguous(), group=self.group)
+        return out
 
 
 def sharded_lookup(query, subkeys, values_shard, k: int, row_lo: int, comm, select=None,
