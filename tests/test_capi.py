@@ -262,3 +262,25 @@ def test_wait_timeout_check_validation(lib):
     assert lib.pkm_check_wait_timeout((1 << 20) + 1, f, None) == 1
     assert lib.pkm_check_wait_timeout(16, None, None) == 1
     assert lib.pkm_check_wait_timeout(16, ctypes.c_void_p((1 << 20) + 2), None) == 1
+
+
+def test_plain_c_consumer(lib, tmp_path):
+    """tests/c_abi_check.c: include/pkm.h compiles as strict C99, a C program
+    links libpkm.so and the host-side paths behave as the header says."""
+    import shutil
+    import subprocess
+
+    from sparse_key_value_b200 import _lib
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = str(tmp_path / "c_abi_check")
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+           os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", exe,
+           _lib.LIB_PATH, f"-Wl,-rpath,{libdir}"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, r.stdout + r.stderr
