@@ -456,8 +456,9 @@ def test_sparse_adam_equals_torch_sparse_adam(orc):
     for step, rows in enumerate(([1, 4, 9], [4, 5], [0, 9, 15]), start=1):
         rows = np.array(rows)
         grads = rng.normal(size=(len(rows), 5))
-        p.grad = torch.sparse_coo_tensor(torch.from_numpy(rows)[None], torch.from_numpy(grads),
-                                         (16, 5), check_invariants=True)
+        with torch.sparse.check_sparse_tensor_invariants():
+            p.grad = torch.sparse_coo_tensor(torch.from_numpy(rows)[None],
+                                             torch.from_numpy(grads), (16, 5))
         opt.step()
         t, m, v = orc.sparse_adam(t, m, v, rows, grads, 0.01, 0.9, 0.99, 1e-30, step)
         np.testing.assert_allclose(t, p.detach().numpy(), rtol=1e-12, atol=1e-14)
