@@ -611,3 +611,29 @@ def test_engram_gate_matches_library(orc):
     np.testing.assert_allclose(r["e"], e.numpy(), rtol=1e-13, atol=1e-13)
     np.testing.assert_allclose(r["alpha"], alpha.numpy(), rtol=1e-12)
     np.testing.assert_allclose(r["v"], (alpha[:, None] * e).numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_engram_rows_golden(orc):
+    """tests/golden/engram_rows.json (written by make_engram_rows.py from the
+    oracle) freezes the hash definition; the stored rows are also re-derived
+    here from the definition in include/pkm.h with Python integers (64-bit
+    wrap-around written out), which checks the C oracle's unsigned
+    arithmetic, seeds at both ends of the 64-bit range and a one-row head."""
+    g = json.load(open(os.path.join(GOLDEN, "engram_rows.json")))
+    seeds = [int(s) for s in g["seeds"]]
+    rows = orc.engram_rows(g["tokens"], g["orders"], g["K"], seeds, g["M"])
+    np.testing.assert_array_equal(rows, np.array(g["rows"]))
+    mask = (1 << 64) - 1
+    off = np.concatenate([[0], np.cumsum(g["M"])[:-1]])
+    L = len(g["tokens"][0])
+    for s, seq in enumerate(g["tokens"]):
+        for p in range(L):
+            for o, n in enumerate(g["orders"]):
+                for k in range(g["K"]):
+                    j = o * g["K"] + k
+                    h = seeds[j]
+                    for q in range(p - n + 1, p + 1):
+                        x = seq[q] & 0xFFFFFFFF if q >= 0 else 0xFFFFFFFF
+                        h = ((h ^ x) * 0x9E3779B97F4A7C15) & mask
+                        h ^= h >> 32
+                    assert rows[s * L + p, j] == off[j] + h % g["M"][j]
