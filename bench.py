@@ -1,15 +1,20 @@
 #!/usr/bin/env python
 """Benchmark of the product-key memory lookup forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload pkm]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload memplus]
+                    [--impl ours|reference] [--sharded]
 
-One step = one pkm_forward over a batch of the workload (norms, sub-key
-scoring + per-half top-k, k x k combine + softmax, bag gather [+ Memory+
-GEMMs]).  For N > 1 the script runs under torch.distributed.run, one rank
-per GPU: every rank holds a replica of the tables and processes its own
-batch (weak scaling, no data-path collective); the timing is the maximum
-over ranks.  Rank 0 prints one JSON line.
+One step = one pkm_forward over a batch of the workload (sub-key norms, the
+selection -- query norms, sub-key scoring, per-half top-k, k x k combine,
+softmax --, bag gather [+ Memory+ GEMMs]).  The default workload is the
+Memory+ forward (16,384 tokens, 16.8 M keys, 32 GiB value table).  For
+N > 1 one rank runs per GPU: run directly, ``--gpus N`` starts itself under
+torch.distributed.run; under torchrun WORLD_SIZE must equal N.  By default
+every rank holds a replica of the tables and processes its own batch (weak
+scaling, no data-path collective).  ``--sharded`` instead splits the value
+table by rows over the ranks and times the row-sharded step (selection,
+all-gather of the selections, each shard's partial bags, reduce-scatter)
+over NCCL.  Timings are the maximum over ranks; rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (plain fp64 C, all host cores) on a
 bounded token sample per step, rank 0 only.
@@ -43,7 +48,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", default="pkm",
+    p.add_argument("--workload", default="memplus",
                    choices=["pkm", "memplus", "tiny", "decode", "train", "memplus_train",
                             "engram"])
     p.add_argument("--graph", action="store_true",
@@ -59,7 +64,33 @@ def parse():
                         "2^20; smaller tables for profiling captures)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="target CPU time of the oracle baseline sample")
+    p.add_argument("--sharded", action="store_true",
+                   help="row-shard the value table over the ranks and time the sharded step "
+                        "(selection, all-gather, partial bags, reduce-scatter) over NCCL")
+    p.add_argument("--launcher-check", action="store_true",
+                   help="start the ranks, join their process group and report the world size "
+                        "(no GPU work): a check of the multi-process launch")
     return p.parse_args()
+
+
+def torchrun_command(args_list, gpus: int, port: int):
+    """The command that runs this script with the same arguments as one
+    process per GPU under torch.distributed.run (rendezvous on 127.0.0.1)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__)] + list(args_list)
+
+
+def relaunch(gpus: int) -> int:
+    """``--gpus N`` run without torchrun: start the N ranks and return their
+    launcher's exit code."""
+    import socket
+
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    return subprocess.call(torchrun_command(sys.argv[1:], gpus, port))
 
 
 # ------------------------------------------------------------ plumbing --
@@ -68,8 +99,17 @@ def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but {world} ranks were started")
     if args.impl == "reference":
         return rank, world, local  # rank 0 alone works; no process group
+    if args.launcher_check:
+        if world > 1:
+            import datetime
+            torch.distributed.init_process_group(
+                "nccl" if torch.cuda.is_available() else "gloo",
+                timeout=datetime.timedelta(seconds=60))
+        return rank, world, local
     if world > 1:
         import datetime
         torch.cuda.set_device(local)
@@ -390,6 +430,7 @@ def run_ours(args, rank, world, local):
     peak = float(peaks["hbm_gbs"])
     bytes_per_launch = gather_bytes_per_token(w) * T
     traffic = traffic_record(args.workload)
+    sel = None
     if phase_ms is not None:
         gather_ms = statistics.mean(phase_ms[4])
         achieved = bytes_per_launch / (gather_ms / 1e3) / 1e9
@@ -400,6 +441,8 @@ def run_ours(args, rank, world, local):
                 "traffic": traffic, "gather_us": round(gather_ms * 1e3, 2)}
         phases = dict(zip(["norms", "score_topk", "combine_softmax", "gate_gemm", "gather",
                            "out_gemm"], [round(statistics.mean(p) * 1e3, 2) for p in phase_ms]))
+        sel = selection_roofline(w, statistics.mean(phase_ms[1]) + statistics.mean(phase_ms[2]),
+                                 peaks, peak_kind)
     else:  # graph replay: only whole steps are timed
         achieved = bytes_per_launch / (ms_per_step / 1e3) / 1e9
         roof = {"kernel": "whole step (graph replay)", "bound": "hbm",
@@ -408,6 +451,11 @@ def run_ours(args, rank, world, local):
                 "algorithmic_bytes_per_launch": bytes_per_launch, "traffic": traffic}
         phases = None
     extra = {}
+    if sel is not None:
+        extra["roofline_select"] = sel
+    if args.workload == "decode":
+        extra["decode"] = decode_report(skv, w, inp, kw, out, idx, wts, ws, step_ms, K,
+                                        bytes_per_launch, peak, peak_kind)
     if args.shards > 1 and not train and not w.memplus and graph is None:
         extra["row_sharded_compute"] = time_sharded_compute(skv, inp, w, args.shards, flush,
                                                             peak, peak_kind)
@@ -484,6 +532,84 @@ def run_ours(args, rank, world, local):
     return res, w, inp
 
 
+def selection_flops(w) -> int:
+    """Sub-key scoring FLOPs of one forward: every token, head and half
+    against its n_sub sub-keys, 2 d_half FLOPs each (the tensor-core work)."""
+    return 2 * w.T * w.H * 2 * w.n_sub * w.d_half
+
+
+def selection_roofline(w, sel_ms: float, peaks, peak_kind):
+    """The selection (sub-key norms and the selection kernel(s)) against the
+    measured bf16 tensor peak: the scoring GEMM is its dense contraction."""
+    flops = selection_flops(w)
+    tf = flops / (sel_ms / 1e3) / 1e12
+    pk = float(peaks["bf16_tflops"])
+    return {"kernel": "select_tc_kernel (query norms, scoring, per-half top-k, k x k combine, "
+                      "softmax) after the sub-key norms", "bound": "tensor",
+            "achieved": round(tf, 1), "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
+            "peak_source": f"{peak_kind} bf16_tflops", "flops_per_launch": flops,
+            "traffic": None, "select_us": round(sel_ms * 1e3, 2)}
+
+
+def dist_stats(ms):
+    """mean / p50 / p99 of per-step times (ms) in microseconds."""
+    us = sorted(x * 1e3 for x in ms)
+    pick = lambda q: us[min(len(us) - 1, int(round(q * (len(us) - 1))))]  # noqa: E731
+    return {"mean": round(statistics.mean(us), 2), "p50": round(pick(0.5), 2),
+            "p99": round(pick(0.99), 2), "steps": len(us)}
+
+
+def decode_report(skv, w, inp, kw, out, idx, wts, ws, graph_step_ms, K, gather_bytes, peak,
+                  peak_kind):
+    """Decode steps: the per-step time distribution with the CUDA graph (the
+    timed steps, back to back) and without it (eager launches), and the bag
+    gather's own time and GB/s in both.  In the graph the library's phase
+    events are recorded as event nodes, read after each replay."""
+
+    def phase_events():
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(7)]
+        for e in ev:
+            e.record()
+        torch.cuda.synchronize()
+        return ev
+
+    def fwd(ev):
+        skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k, out=out, idx=idx,
+                        weights=wts, workspace=ws, phase_events=ev, **kw)
+
+    eager_ms, eager_gather = [], []
+    ev = phase_events()
+    for i in range(K + 3):
+        fwd(ev)
+        torch.cuda.synchronize()
+        if i >= 3:
+            eager_ms.append(ev[0].elapsed_time(ev[6]))
+            eager_gather.append(ev[4].elapsed_time(ev[5]))
+    gev = phase_events()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd(gev)
+    graph_gather = []
+    for i in range(K + 3):
+        g.replay()
+        torch.cuda.synchronize()
+        if i >= 3:
+            graph_gather.append(gev[4].elapsed_time(gev[5]))
+    del g
+    assert skv.device_error() == 0
+    ge, gg = statistics.mean(eager_gather), statistics.mean(graph_gather)
+    return {"step_us_graph": dist_stats(graph_step_ms), "step_us_eager": dist_stats(eager_ms),
+            "gather_bytes_per_step": gather_bytes,
+            "gather_us_graph": round(gg * 1e3, 2),
+            "gather_GBps_graph": round(gather_bytes / (gg / 1e3) / 1e9, 1),
+            "gather_us_eager": round(ge * 1e3, 2),
+            "gather_GBps_eager": round(gather_bytes / (ge / 1e3) / 1e9, 1),
+            "peak": peak, "peak_source": f"{peak_kind} hbm_gbs",
+            "note": "graph steps timed back to back (events outside the graph); the gather's "
+                    "time in the graph from the library's phase events, recorded as graph "
+                    "event nodes, one replay at a time"}
+
+
 def time_sharded_compute(skv, inp, w, S, flush, peak, peak_kind, reps=20):
     """The compute of one row-sharded step with all S shards on this GPU:
     the selection (pkm_select) and each shard's fp32 partial bags over all
@@ -523,6 +649,99 @@ def time_sharded_compute(skv, inp, w, S, flush, peak, peak_kind, reps=20):
             "frac": round(nbytes / (g_ms / 1e3) / 1e9 / peak, 4),
             "peak_source": f"{peak_kind} hbm_gbs",
             "note": "all shards on one GPU; the exchange between the steps is not timed"}
+
+
+def run_sharded(args, rank, world, local, select=None, gather=None, device="cuda"):
+    """The row-sharded step (sparse_key_value_b200.sharded): every rank holds
+    ceil(N / world) rows of the value table and the replicated sub-keys,
+    selects the rows of its own T tokens, and the ranks all-gather the
+    selections, sum the partial bags of the rows they hold for every rank's
+    tokens and reduce-scatter them (NCCL).  Weak scaling: T tokens per rank.
+    The Memory+ GEMMs are not part of this step.  ``select`` / ``gather`` /
+    ``device`` are for host tests of the step order (gloo ranks, injected
+    reference steps); the benchmark uses the CUDA library."""
+    from sparse_key_value_b200.inputs import WORKLOADS, make_inputs, value_shard
+    from sparse_key_value_b200.sharded import (LocalComm, TorchComm, exchange_bytes, shard_rows,
+                                               sharded_lookup)
+
+    w = args.workload_obj if hasattr(args, "workload_obj") else WORKLOADS[args.workload]
+    w = rank_workload(w, rank)
+    if device == "cuda":
+        import sparse_key_value_b200 as skv
+        skv.load()
+    inp = make_inputs(w, device, with_values=False)
+    lo, n_local = shard_rows(w.N, world, rank)
+    shard = value_shard(w, n_local, rank, device)
+    comm = TorchComm() if world > 1 else LocalComm()
+    cuda = device == "cuda"
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device) if cuda else None
+
+    def step():
+        return sharded_lookup(inp["query"], inp["subkeys"], shard, w.k, lo, comm, select, gather)
+
+    for _ in range(args.warmup):
+        if cuda:
+            flush.zero_()
+        step()
+    if cuda:
+        torch.cuda.synchronize()
+    barrier(world)
+    K = args.steps
+    ms = []
+    clk = Clocks(local) if cuda else None
+    if clk is not None:
+        clk.__enter__()
+    for _ in range(K):
+        if cuda:
+            flush.zero_()  # L2 flush between timed steps (outside the events)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            y, _, _ = step()
+            e1.record()
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        else:
+            t0 = time.perf_counter()
+            y, _, _ = step()
+            ms.append((time.perf_counter() - t0) * 1e3)
+    if clk is not None:
+        clk.__exit__(None, None, None)
+    barrier(world)
+    total = max_over_ranks(sum(ms), world)
+    ms_per_step = total / K
+    value = whole_job_tokens_per_s(w.T, world, ms_per_step)
+    B = w.H * w.k
+    # per rank: its shard's rows of every rank's bags (world*T*B rows spread over world
+    # shards: T*B in expectation), every rank's ids and weights, the fp32 partials written
+    hbm = w.T * B * w.d_v * w.elem_bytes + world * w.T * B * 8 + world * w.T * w.d_v * 4
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded generators; no dataset)",
+        "config": dict(w.describe(), step="row-sharded lookup (selection, all-gather, partial "
+                                          "bags, reduce-scatter); no Memory+ GEMMs",
+                       rows_per_rank=n_local, l2="256 MiB L2 flush write before every step",
+                       parallelism=f"value table row-sharded x{world}, sub-keys replicated, "
+                                   f"{w.T} tokens per rank"),
+        "exchange_bytes_per_rank": exchange_bytes(w.T, w.H, w.k, w.d_v, world),
+        "hbm_bytes_per_rank": hbm, "y_shape": list(y.shape),
+        "clocks": clk.summary() if clk is not None else None,
+        "cpu_baseline": None, "e2e": None,
+    }
+
+
+def launcher_check(rank, world):
+    """Every rank joined the process group: the sum of the ranks over it."""
+    total = 0.0
+    if world > 1:
+        dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+        if dev == "cuda":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        t = torch.tensor([float(rank)], device=dev)
+        torch.distributed.all_reduce(t)
+        total = float(t.item())
+    return {"launcher_check": True, "n_gpus": world, "rank_sum": total}
 
 
 def time_sparse_adam(skv, table, rows, grads, count, U, w, peak, peak_kind, reps=10):
@@ -881,10 +1100,16 @@ def engram_reference(args, world):
 
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args.gpus))
     rank, world, local = dist_setup(args)
     try:
-        if args.impl == "reference":
+        if args.launcher_check:
+            res = launcher_check(rank, world)
+        elif args.impl == "reference":
             res = run_reference(args, rank, world)
+        elif args.sharded:
+            res = run_sharded(args, rank, world, local)
         elif args.workload == "engram":
             res, w, inp = run_engram(args, rank, world, local)
             res["cpu_baseline"] = engram_cpu_baseline(args, w, inp) \

@@ -85,7 +85,8 @@ typedef enum { PKM_F32 = 0, PKM_BF16 = 1 } pkm_dtype;
  *           W2 [d_v, d_model] (bf16 only).
  *
  * Limits: 1 <= k <= min(n_sub, 64); d_half, d_v, d_model multiples of 8;
- * n_sub*n_sub < 2^31.  T = 0 is a valid empty call.
+ * n_sub*n_sub < 2^31; 0 <= T <= 2^36 (PKM_ERR_INVALID_ARG otherwise).
+ * T = 0 is a valid empty call.
  */
 typedef struct {
     int64_t T;
@@ -108,7 +109,11 @@ typedef struct {
        [0] start, [1] after the norms, [2] after scoring + per-half top-k,
        [3] after combine + softmax, [4] before the bag gather (after the
        Memory+ gate GEMM), [5] after the bag gather, [6] end (after the
-       Memory+ output GEMM). */
+       Memory+ output GEMM).  When the selection runs as one kernel (bf16,
+       d_half % 64 == 0, 256 <= n_sub < 65536, n_sub % 4 == 0, k <= 32,
+       T > 64), [1] follows the sub-key norms only and [2] = [3] follow the
+       whole selection.  Under stream capture the events are recorded as
+       external event nodes of the graph, so every replay records them. */
     void **phase_events;
     /* Optional, Memory+ only: NULL, or [T, d_v] (dtype) receiving the bag
        output y before the gate, as pkm_memplus_backward needs it.  With it
@@ -175,6 +180,11 @@ PKM_API pkm_status pkm_select(const pkm_fwd_args *args, pkm_stream_t stream);
  *   and/or dense: dvalues_dense fp32 [n_sub^2, d_v] receives += per row.
  *   Either may be NULL (not both).  dscores [T,H,k] fp32 (optional) gets dS.
  * Every sum runs in a fixed order: results are bitwise reproducible.
+ *
+ * Limits beyond the forward's: d_half a multiple of 256 (bf16) or 128 (fp32)
+ * and at most 2048 (one warp holds a query half in registers, 16 bytes per
+ * lane per step); T*H*k*2 < 2^32.  Other sizes return PKM_ERR_UNSUPPORTED
+ * and launch nothing.
  */
 typedef struct {
     int64_t T;

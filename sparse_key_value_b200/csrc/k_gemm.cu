@@ -1,10 +1,11 @@
 // k_gemm.cu -- dense pieces of the Memory+ block ("Memory Layers at
 // Scale" digest, "Memory+ 블록": out = (y ⊙ silu(x W1)) W2).
 //
-// The weights arrive row-major ([d_model, d_v] and [d_v, d_model]); a small
-// transpose puts each into the K-major layout both GEMM operands use.  The
-// GEMM runs on the tensor cores (k_gemm_tc.cu) when the shape allows it,
-// else on this SIMT kernel.
+// The GEMM runs on the tensor cores (k_gemm_tc.cu) when the shape allows it,
+// else on this SIMT kernel; both read every operand in the layout the caller
+// holds it (K-major, or MN-major for a weight [d_in, d_out] used as x W and
+// for the tokens of a weight gradient x^T dy).  The transpose kernel serves
+// the backward's small steps that want a transposed copy.
 #include <math.h>
 
 #include "common.cuh"
@@ -85,11 +86,13 @@ cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
 // C[M,N] = epi(sum_k A[m,k] B[n,k]); 64x64 tile, 256 threads, 4x4 each.
-// out_mode: 0 bf16 (epi applied), 1 fp32, 2 fp32 accumulate.
+// out_mode: 0 bf16 (epi applied), 1 fp32, 2 fp32 accumulate.  a_mn / b_mn:
+// A held as [K][M] / B as [K][N].
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const __nv_bfloat16* __restrict__ A,
                                                         const __nv_bfloat16* __restrict__ B,
                                                         int64_t M, int N, int K, int epi,
-                                                        int out_mode, void* __restrict__ Cv) {
+                                                        int out_mode, bool a_mn, bool b_mn,
+                                                        void* __restrict__ Cv) {
   __shared__ float As[16][64 + 1];
   __shared__ float Bs[16][64 + 1];
   const int64_t m0 = (int64_t)blockIdx.y * 64;
@@ -101,8 +104,10 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const __nv_bfloat16* __r
       int r = i / 16, kk = i % 16;
       int64_t m = m0 + r;
       int nn = n0 + r;
-      As[kk][r] = (m < M && k0 + kk < K) ? __bfloat162float(A[m * K + k0 + kk]) : 0.f;
-      Bs[kk][r] = (nn < N && k0 + kk < K) ? __bfloat162float(B[(int64_t)nn * K + k0 + kk]) : 0.f;
+      const int64_t kq = k0 + kk;
+      As[kk][r] = (m < M && kq < K) ? __bfloat162float(A[a_mn ? kq * M + m : m * K + kq]) : 0.f;
+      Bs[kk][r] = (nn < N && kq < K) ? __bfloat162float(B[b_mn ? kq * N + nn : (int64_t)nn * K + kq])
+                                     : 0.f;
     }
     __syncthreads();
 #pragma unroll
@@ -140,32 +145,41 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const __nv_bfloat16* __r
 }
 
 cudaError_t launch_gemm_simt(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                             int out_mode, void* C, cudaStream_t stream) {
+                             int out_mode, void* C, cudaStream_t stream, bool a_mn, bool b_mn) {
   dim3 grid((N + 63) / 64, (unsigned)((M + 63) / 64));
   gemm_simt_kernel<<<grid, 256, 0, stream>>>((const __nv_bfloat16*)A, (const __nv_bfloat16*)B,
-                                             M, N, K, epi, out_mode, C);
+                                             M, N, K, epi, out_mode, a_mn, b_mn, C);
   note_launch();
   return cudaGetLastError();
 }
 cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
                            int out_mode, void* C, int32_t* status, cudaStream_t stream,
-                           int splits, int64_t c_split);
+                           int splits, int64_t c_split, bool a_mn, bool b_mn);
+
+// Shapes the tensor-core GEMM takes: the TMA rows of every operand are a
+// multiple of 16 bytes (K for a K-major operand, M / N for an MN-major one).
+static bool tc_ok(int64_t M, int N, int K, bool a_mn, bool b_mn) {
+  if (M < 1 || N < 16 || K < 64 || N % 8) return false;
+  if ((!a_mn || !b_mn) && K % 8) return false;
+  return !a_mn || M % 8 == 0;
+}
 
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                             void* C, int32_t* status, cudaStream_t stream) {
+                             void* C, int32_t* status, cudaStream_t stream, bool b_mn) {
   if (M <= 0) return cudaSuccess;
-  if (gemm_tc_supported(M, N, K))
-    return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream, 1, 0);
-  return launch_gemm_simt(A, B, M, N, K, epi, 0, C, stream);
+  if (tc_ok(M, N, K, false, b_mn))
+    return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream, 1, 0, false, b_mn);
+  return launch_gemm_simt(A, B, M, N, K, epi, 0, C, stream, false, b_mn);
 }
 
 cudaError_t launch_gemm_f32(const void* A, const void* B, int64_t M, int N, int K,
-                            bool accumulate, float* C, int32_t* status, cudaStream_t stream) {
+                            bool accumulate, float* C, int32_t* status, cudaStream_t stream,
+                            bool a_mn, bool b_mn) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   const int mode = accumulate ? 2 : 1;
-  if (gemm_tc_supported(M, N, K))
-    return launch_gemm_tc(A, B, M, N, K, 0, mode, C, status, stream, 1, 0);
-  return launch_gemm_simt(A, B, M, N, K, 0, mode, C, stream);
+  if (tc_ok(M, N, K, a_mn, b_mn))
+    return launch_gemm_tc(A, B, M, N, K, 0, mode, C, status, stream, 1, 0, a_mn, b_mn);
+  return launch_gemm_simt(A, B, M, N, K, 0, mode, C, stream, a_mn, b_mn);
 }
 
 // C = sum over s of part[s] (fixed order)
@@ -180,7 +194,7 @@ __global__ void sum_slices_kernel(const float* __restrict__ part, int S, int64_t
 }
 
 int gemm_splitk_slices(int64_t M, int N, int K) {
-  if (!gemm_tc_supported(M, N, K)) return 1;
+  if (M < 1 || N < 16 || K < 64 || N % 8) return 1;
   const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
   const int KB = (K + 63) / 64;
   int s = 1;
@@ -194,10 +208,12 @@ size_t gemm_splitk_workspace(int64_t M, int N, int K) {
 }
 
 cudaError_t launch_gemm_f32_splitk(const void* A, const void* B, int64_t M, int N, int K,
-                                   float* C, float* part, int32_t* status, cudaStream_t stream) {
+                                   float* C, float* part, int32_t* status, cudaStream_t stream,
+                                   bool a_mn, bool b_mn) {
   const int S = gemm_splitk_slices(M, N, K);
-  if (S <= 1 || !part) return launch_gemm_f32(A, B, M, N, K, false, C, status, stream);
-  cudaError_t e = launch_gemm_tc(A, B, M, N, K, 0, 1, part, status, stream, S, M * N);
+  if (S <= 1 || !part || !tc_ok(M, N, K, a_mn, b_mn))
+    return launch_gemm_f32(A, B, M, N, K, false, C, status, stream, a_mn, b_mn);
+  cudaError_t e = launch_gemm_tc(A, B, M, N, K, 0, 1, part, status, stream, S, M * N, a_mn, b_mn);
   if (e != cudaSuccess) return e;
   // the GEMM launcher makes ceil(KB / ceil(KB / S)) slices; with KB >= 8 S this is S
   const int KB = (K + 63) / 64, kbps = (KB + S - 1) / S, nz = (KB + kbps - 1) / kbps;

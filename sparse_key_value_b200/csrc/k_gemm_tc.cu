@@ -1,17 +1,28 @@
 // k_gemm_tc.cu -- the dense GEMMs of the Memory+ block on the tensor cores
 // ("Memory Layers at Scale" digest, "Memory+ 블록": out = (y ⊙ silu(x W1)) W2).
 //
-//   C[M, N] = epi(A[M, K] * B[N, K]^T),  A, B bf16 K-major, C row-major,
-//   epi = silu (gate) or identity, fp32 accumulation; C is bf16 (rounded to
-//   nearest even), fp32, or fp32 accumulated into (C += A B^T).
+//   C[M, N] = epi(A[M, K] * B[N, K]^T), bf16 operands, fp32 accumulation;
+//   epi = silu (gate) or identity; C is bf16 (rounded to nearest even), fp32,
+//   or fp32 accumulated into (C += A B^T).
+// Each operand is read in the layout the caller holds it, so no operand is
+// transposed in memory:
+//   K-major   A as [M][K] (or B as [N][K]), K contiguous;
+//   MN-major  A as [K][M] (or B as [K][N]), M (N) contiguous -- a weight
+//             W [d_in, d_out] used as x W, or the tokens' rows used as the
+//             contraction of a weight gradient (x^T dy).
+// The TMA loads 64-wide k-blocks with the 128-byte swizzle: a K-major tile is
+// [rows][64 k] (one 128-byte line per row), an MN-major tile is a stack of
+// [64 k][64 rows] boxes (one line per k); the MMA's shared-memory descriptor
+// and the instruction descriptor's transpose bit say which.
 //
-// One CTA per 128 x 256 output tile:
-//   warp 0     TMA producer: 64-wide k-blocks of A [128 x 64] and B [256 x 64]
-//              (128-byte swizzle) into a 4-stage ring.
-//   warp 1     TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128, N=256.
-//   warps 2-5  epilogue: one thread per output row reads 32 accumulator
-//              columns at a time (tcgen05.ld), applies the epilogue, rounds to
-//              bf16 (nearest even) and stores 64 contiguous bytes.
+// Persistent: one CTA per SM loops over the output tiles (128 x 256, N
+// fastest so neighbouring tiles share their A rows, then split-K slices).
+//   warp 0     TMA producer: a 4-stage ring of (A, B) k-blocks, continuing
+//              across tiles.
+//   warp 1     TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128,
+//              N=256, into one of two 256-column accumulators (TMEM 512).
+//   warps 2-5  epilogue: one thread per output row; while it reads and stores
+//              one accumulator the MMAs of the next tile fill the other.
 // Spin-waits are bounded; on a timeout the CTA records PKM_ERR_TIMEOUT,
 // drains what it issued, frees its TMEM and exits.
 #include <math.h>
@@ -23,17 +34,19 @@
 namespace pkm {
 
 namespace gm {
-constexpr int kM = 128, kN = 256, kKB = 64, kStages = 4;
+constexpr int kM = 128, kN = 256, kKB = 64, kStages = 4, kAcc = 2;
 constexpr int kABytes = kM * kKB * 2, kBBytes = kN * kKB * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 192;
+constexpr int kBox = 64;  // rows of an MN-major box (128 bytes of bf16)
 constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256;
 }  // namespace gm
 
 struct GemmCtl {
   uint64_t full[gm::kStages];
   uint64_t empty[gm::kStages];
-  uint64_t accf;
+  uint64_t accf[gm::kAcc];
+  uint64_t acce[gm::kAcc];
   uint64_t drain;
   uint32_t tmem;
   volatile int abort;
@@ -44,32 +57,63 @@ __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, GemmCt
   return mbar_wait_or_abort(bar, parity, &ctl->abort, status);
 }
 
-// OUT: 0 bf16 store, 1 fp32 store, 2 fp32 accumulate (C += result)
-template <int EPI, int OUT>
+// Shared-memory descriptor of an MN-major operand tile with the 128-byte
+// swizzle: atoms of 8 k-lines x 64 elements (1024 B); consecutive atoms along
+// K are 1024 B apart (stride byte offset), consecutive 64-element groups
+// along M/N are one box (8 KiB) apart (leading byte offset).
+__device__ __forceinline__ uint64_t smem_desc_mn128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((gm::kBox * 128) >> 4) << 16;  // leading byte offset: next box
+  d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: next 8 k-lines
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+struct TileCoord {
+  int64_t m0;
+  int n0, z;
+};
+
+__device__ __forceinline__ TileCoord tile_of(int t, int tiles_m, int tiles_n) {
+  const int nt = t % tiles_n;
+  const int r = t / tiles_n;
+  return TileCoord{(int64_t)(r % tiles_m) * gm::kM, nt * gm::kN, r / tiles_m};
+}
+
+// OUT: 0 bf16 store, 1 fp32 store, 2 fp32 accumulate (C += result).
+// AMN / BMN: the operand is MN-major.
+template <int EPI, int OUT, bool AMN, bool BMN>
 __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t M,
-    int N, int K, void* __restrict__ Cv, int kb_per_split, int64_t c_split,
+    int N, int K, void* __restrict__ Cv, int kb_per_split, int nz, int64_t c_split,
     int32_t* status) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* stages = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmCtl* ctl = reinterpret_cast<GemmCtl*>(stages + gm::kStages * gm::kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * gm::kM;
-  const int n0 = blockIdx.y * gm::kN;
-  // split-K (grid.z): this CTA adds k-blocks [kb0, kb0 + KB) into the
-  // output slice blockIdx.z (c_split elements apart)
+  const int tiles_m = (int)((M + gm::kM - 1) / gm::kM);
+  const int tiles_n = (N + gm::kN - 1) / gm::kN;
+  const int n_tiles = tiles_m * tiles_n * nz;
+  // split-K: slice z adds k-blocks [z * kb_per_split, ...) into the output
+  // slice z (c_split elements apart)
   const int KB_all = (K + gm::kKB - 1) / gm::kKB;
-  const int kb0 = kb_per_split > 0 ? (int)blockIdx.z * kb_per_split : 0;
-  const int KB = kb_per_split > 0 ? min(kb_per_split, KB_all - kb0) : KB_all;
-  Cv = static_cast<char*>(Cv) + (int64_t)blockIdx.z * c_split * (OUT != 0 ? 4 : 2);
+  auto kb_range = [&](int z, int& kb0, int& nkb) {
+    kb0 = kb_per_split > 0 ? z * kb_per_split : 0;
+    nkb = kb_per_split > 0 ? min(kb_per_split, KB_all - kb0) : KB_all;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < gm::kStages; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
-    mbar_init(&ctl->accf, 1);
+    for (int b = 0; b < gm::kAcc; ++b) {
+      mbar_init(&ctl->accf[b], 1);
+      mbar_init(&ctl->acce[b], 4);
+    }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_barrier_init();
@@ -79,7 +123,7 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem, gm::kN);
+    tmem_alloc(&ctl->tmem, gm::kAcc * gm::kN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -88,19 +132,42 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
   const uint32_t tmem = ctl->tmem;
 
   if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int stage = kb % gm::kStages;
-        const uint32_t phase = (uint32_t)(kb / gm::kStages) & 1;
-        if (!gemm_wait(&ctl->empty[stage], phase ^ 1, ctl, status)) { ok = false; break; }
-        unsigned char* sa = stages + stage * gm::kStageBytes;
-        mbar_arrive_expect_tx(&ctl->full[stage], gm::kStageBytes);
-        tma_load_2d(sa, &tmA, &ctl->full[stage], (kb0 + kb) * gm::kKB, (int32_t)m0);
-        tma_load_2d(sa + gm::kABytes, &tmB, &ctl->full[stage], (kb0 + kb) * gm::kKB, n0);
-        issued_mask |= 1u << stage;
-        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+      int f = 0;  // stage fills so far
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = tile_of(t, tiles_m, tiles_n);
+        int kb0, nkb;
+        kb_range(tc.z, kb0, nkb);
+        for (int kb = 0; kb < nkb; ++kb, ++f) {
+          const int stage = f % gm::kStages;
+          const uint32_t phase = (uint32_t)(f / gm::kStages) & 1;
+          if (!gemm_wait(&ctl->empty[stage], phase ^ 1, ctl, status)) { ok = false; break; }
+          unsigned char* sa = stages + stage * gm::kStageBytes;
+          unsigned char* sb = sa + gm::kABytes;
+          const int kc = (kb0 + kb) * gm::kKB;
+          mbar_arrive_expect_tx(&ctl->full[stage], gm::kStageBytes);
+          if (AMN) {
+#pragma unroll
+            for (int j = 0; j < gm::kM / gm::kBox; ++j)
+              tma_load_2d(sa + j * gm::kBox * 128, &tmA, &ctl->full[stage],
+                          (int32_t)tc.m0 + j * gm::kBox, kc);
+          } else {
+            tma_load_2d(sa, &tmA, &ctl->full[stage], kc, (int32_t)tc.m0);
+          }
+          if (BMN) {
+#pragma unroll
+            for (int j = 0; j < gm::kN / gm::kBox; ++j)
+              tma_load_2d(sb + j * gm::kBox * 128, &tmB, &ctl->full[stage],
+                          tc.n0 + j * gm::kBox, kc);
+          } else {
+            tma_load_2d(sb, &tmB, &ctl->full[stage], kc, tc.n0);
+          }
+          issued_mask |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        }
       }
       if (!ok) {
         for (int s = 0; s < gm::kStages; ++s)
@@ -110,42 +177,64 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
       }
     }
   } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(gm::kM, gm::kN);
+      const uint32_t idesc = idesc_bf16_f32(gm::kM, gm::kN) | (AMN ? (1u << 15) : 0u) |
+                             (BMN ? (1u << 16) : 0u);
       bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int stage = kb % gm::kStages;
-        const uint32_t phase = (uint32_t)(kb / gm::kStages) & 1;
-        if (!gemm_wait(&ctl->full[stage], phase, ctl, status)) { ok = false; break; }
+      int f = 0, li = 0;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++li) {
+        const TileCoord tc = tile_of(t, tiles_m, tiles_n);
+        int kb0, nkb;
+        kb_range(tc.z, kb0, nkb);
+        const int buf = li & 1;
+        // this accumulator is free once the epilogue has read its last tile
+        if (!gemm_wait(&ctl->acce[buf], ((li >> 1) & 1) ^ 1, ctl, status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sa = smem_u32(stages + stage * gm::kStageBytes);
-        const uint32_t sb = sa + gm::kABytes;
+        const uint32_t dt = tmem + (uint32_t)(buf * gm::kN);
+        for (int kb = 0; kb < nkb; ++kb, ++f) {
+          const int stage = f % gm::kStages;
+          const uint32_t phase = (uint32_t)(f / gm::kStages) & 1;
+          if (!gemm_wait(&ctl->full[stage], phase, ctl, status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stages + stage * gm::kStageBytes);
+          const uint32_t sb = sa + gm::kABytes;
 #pragma unroll
-        for (int kk = 0; kk < gm::kKB / 16; ++kk)
-          tc_mma_f16(tmem, smem_desc_k128(sa + kk * 32), smem_desc_k128(sb + kk * 32), idesc,
-                     (kb | kk) != 0);
-        tc_commit(&ctl->empty[stage]);
+          for (int kk = 0; kk < gm::kKB / 16; ++kk) {
+            // K = 16 per MMA: 32 bytes along a K-major line, 16 lines of an MN-major box
+            const uint64_t ad = AMN ? smem_desc_mn128(sa + kk * 2048) : smem_desc_k128(sa + kk * 32);
+            const uint64_t bd = BMN ? smem_desc_mn128(sb + kk * 2048) : smem_desc_k128(sb + kk * 32);
+            tc_mma_f16(dt, ad, bd, idesc, (kb | kk) != 0);
+          }
+          tc_commit(&ctl->empty[stage]);
+        }
+        if (ok) tc_commit(&ctl->accf[buf]);
       }
-      if (ok) tc_commit(&ctl->accf);
       tc_commit(&ctl->drain);
       for (unsigned long long i = 0; i < kSpinLimit; ++i)
         if (mbar_try_wait(&ctl->drain, 0)) break;
     }
   } else {
+    // ----------------------------------------------------------- epilogue
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int64_t m = m0 + row;
-    const bool got = gemm_wait(&ctl->accf, 0, ctl, status);
-    if (__all_sync(0xffffffffu, got)) {
+    int li = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++li) {
+      const TileCoord tc = tile_of(t, tiles_m, tiles_n);
+      const int buf = li & 1;
+      const bool got = gemm_wait(&ctl->accf[buf], (li >> 1) & 1, ctl, status);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
+      const int64_t m = tc.m0 + row;
+      void* Cz = static_cast<char*>(Cv) + (int64_t)tc.z * c_split * (OUT != 0 ? 4 : 2);
       for (int g = 0; g < gm::kN / 32; ++g) {
-        const int col0 = n0 + g * 32;
+        const int col0 = tc.n0 + g * 32;
         if (col0 >= N) break;
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + g * 32, r);
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + buf * gm::kN + g * 32, r);
         tmem_ld_wait();
         if (m < M && OUT != 0) {
-          float* dst = static_cast<float*>(Cv) + m * N + col0;
+          float* dst = static_cast<float*>(Cz) + m * N + col0;
           const int nq = col0 + 32 <= N ? 8 : (N - col0) / 4;  // N % 8 == 0
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -176,7 +265,7 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
             }
             packed[j] = pack_bf16x2(a, b);
           }
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(Cv) + m * N + col0;
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(Cz) + m * N + col0;
           if (col0 + 32 <= N) {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -188,6 +277,9 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->acce[buf]);
     }
   }
 
@@ -195,7 +287,7 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, gm::kN);
+    tmem_dealloc(tmem, gm::kAcc * gm::kN);
   }
 }
 
@@ -203,20 +295,45 @@ bool gemm_tc_supported(int64_t M, int N, int K) {
   return M >= 1 && N >= 16 && K >= gm::kKB && N % 8 == 0 && K % 8 == 0;
 }
 
+static int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      sms = v;
+    else
+      return 148;
+  }
+  return sms;
+}
+
 // out_mode: 0 bf16 (epi applied), 1 fp32, 2 fp32 accumulate; epi only with bf16 output.
 // splits > 1: split-K into `splits` slices of C, c_split elements apart.
+// a_mn / b_mn: A is [K][M] / B is [K][N] (M / N contiguous) instead of [M][K] / [N][K].
 cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
                            int out_mode, void* C, int32_t* status, cudaStream_t stream,
-                           int splits, int64_t c_split) {
+                           int splits, int64_t c_split, bool a_mn, bool b_mn) {
   if (M <= 0) return cudaSuccess;
   CUtensorMap tmA, tmB;
-  {
+  if (a_mn) {
+    if (M % 8) return cudaErrorInvalidValue;  // the row stride of [K][M] is 16-byte aligned
+    const uint64_t dims[2] = {(uint64_t)M, (uint64_t)K};
+    const uint64_t strides[1] = {(uint64_t)M * 2};
+    const uint32_t box[2] = {(uint32_t)gm::kBox, (uint32_t)gm::kKB};
+    if (!make_tmap_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  } else {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
     const uint64_t strides[1] = {(uint64_t)K * 2};
     const uint32_t box[2] = {(uint32_t)gm::kKB, (uint32_t)gm::kM};
     if (!make_tmap_bf16(&tmA, A, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  {
+  if (b_mn) {
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)K};
+    const uint64_t strides[1] = {(uint64_t)N * 2};
+    const uint32_t box[2] = {(uint32_t)gm::kBox, (uint32_t)gm::kKB};
+    if (!make_tmap_bf16(&tmB, B, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  } else {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)N};
     const uint64_t strides[1] = {(uint64_t)K * 2};
     const uint32_t box[2] = {(uint32_t)gm::kKB, (uint32_t)gm::kN};
@@ -228,25 +345,32 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K
     kbps = (KB + splits - 1) / splits;
     nz = (KB + kbps - 1) / kbps;
   }
-  dim3 grid((unsigned)((M + gm::kM - 1) / gm::kM), (unsigned)((N + gm::kN - 1) / gm::kN),
-            (unsigned)nz);
-  cudaError_t e;
-#define PKM_GEMM_TC(E_, O_)                                                                  \
-  e = cudaFuncSetAttribute(gemm_tc_kernel<E_, O_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                           (int)gm::kSmemBytes);                                             \
-  if (e != cudaSuccess) return e;                                                            \
-  gemm_tc_kernel<E_, O_><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(tmA, tmB, M, N, K, C, \
-                                                                        kbps, c_split, status)
+  const int64_t tiles = (M + gm::kM - 1) / gm::kM * ((N + gm::kN - 1) / gm::kN) * nz;
+  const unsigned grid = (unsigned)(tiles < num_sms() ? tiles : num_sms());
+  cudaError_t e = cudaSuccess;
+  auto go = [&](auto kern) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)gm::kSmemBytes);
+    if (e != cudaSuccess) return;
+    kern<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(tmA, tmB, M, N, K, C, kbps, nz, c_split,
+                                                         status);
+  };
+#define PKM_GEMM_LAYOUTS(E_, O_)                                   \
+  if (a_mn && b_mn) go(gemm_tc_kernel<E_, O_, true, true>);        \
+  else if (a_mn) go(gemm_tc_kernel<E_, O_, true, false>);          \
+  else if (b_mn) go(gemm_tc_kernel<E_, O_, false, true>);          \
+  else go(gemm_tc_kernel<E_, O_, false, false>)
   if (out_mode == 1) {
-    PKM_GEMM_TC(0, 1);
+    PKM_GEMM_LAYOUTS(0, 1);
   } else if (out_mode == 2) {
-    PKM_GEMM_TC(0, 2);
+    PKM_GEMM_LAYOUTS(0, 2);
   } else if (epi == 1) {
-    PKM_GEMM_TC(1, 0);
+    PKM_GEMM_LAYOUTS(1, 0);
   } else {
-    PKM_GEMM_TC(0, 0);
+    PKM_GEMM_LAYOUTS(0, 0);
   }
-#undef PKM_GEMM_TC
+#undef PKM_GEMM_LAYOUTS
+  if (e != cudaSuccess) return e;
   note_launch();
   return cudaGetLastError();
 }

@@ -1,0 +1,739 @@
+// k_select_tc.cu -- the whole product-key selection in one kernel: query
+// norms, sub-key scores on the tensor cores, per-half top-k, the k x k
+// combine, the final top-k and the softmax weights.
+//
+// "Memory Layers at Scale" digest, "Product-key 검색": the key is split in
+// two sub-keys and the top-k of N full keys is found from 2*sqrt(N)
+// comparisons; "Memory+ 블록": qk-normalization.  "모델 안의 메모리", "작동
+// 방식": each half of the query is compared with its ~sqrt(N) half-keys, the
+// best of each half are combined (a 1,000 x 1,000 grid searched with 2,000
+// comparisons) and the values read are averaged with weights.
+//
+// Grid: (token tiles of 128) x (2H); the two CTAs (h, half 0) and (h, half 1)
+// of a token tile form a cluster of two.  Each CTA scores its 128 tokens
+// against all n sub-keys of its (head, half), 256 columns per chunk:
+//   warp 0     TMA producer: per chunk and 64-wide k-block the query tile
+//              [128 x 64] and the sub-key tile [256 x 64] (bf16, 128-byte
+//              swizzle) into a 2-stage ring.
+//   warp 1     TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128,
+//              N=256, K=16, fp32 accumulator in 256 TMEM columns.
+//   warps 2-5  epilogue, one thread per token row (TMEM lane).
+// Two CTAs share an SM, so the MMAs of one overlap the epilogue of the other.
+//
+// Query norms: while the first chunk's k-blocks pass through shared memory,
+// every epilogue thread sums the squares of its row of the query tile (the
+// swizzle only permutes 16-byte pieces within a row, so the sum needs no
+// unswizzling); the producer refills such a stage only after the epilogue
+// has read it.  So the query is read from memory once, by the TMA.
+//
+// Per-row top-k over the scores s = sqrt(d_half) * rq * rk[a] * acc:
+//   * the epilogue filters raw products p = acc * rk[a] against a threshold
+//     thr (a lower bound of the row's final k-th best p) and appends the
+//     survivors (p, a) to a 16-entry per-row buffer in shared memory;
+//   * whenever some row of the warp holds more than 8, the warp merges each
+//     row's buffer into the row's sorted list of the k best (keys in
+//     registers, bitonic sort and merge networks) and raises thr to the
+//     list's k-th best;
+//   * before the first chunk's filter pass a histogram pass over the same
+//     chunk (still in TMEM) counts the maxima of groups of 4 columns into
+//     score bins of 1/16; the lower edge of the bin where the count from the
+//     top reaches k bounds the chunk's (and so the row's) k-th best score
+//     from below, since group maxima are distinct elements.  That starts the
+//     filter near its final level instead of at -inf.
+// Keys: 64 bits, the order-preserving bits of the fp32 score above the
+// complemented column (equal scores order the smaller column first).
+// Measured: packing the column into the low mantissa bits of an fp64 key
+// and exchanging with fp64 min/max ran 2.5x slower on B200.
+//
+// Combine: each CTA writes its rows' sorted lists to shared memory; after a
+// cluster barrier, CTA c takes rows [64c, 64c+64), copies the other half's
+// lists for them from the peer CTA's shared memory (DSMEM), and one thread
+// per row runs the max-heap frontier over the k x k grid S[i][j] = s1[i] +
+// s2[j] (rows and columns non-increasing), keeps k cells, forms the row ids
+// a*n+b and the softmax weights and writes them.  A second cluster barrier
+// keeps each CTA's shared memory alive until its peer has read it.
+//
+// Every spin-wait is bounded: on a timeout the CTA records PKM_ERR_TIMEOUT,
+// stops issuing work, waits (bounded) for its copies and MMAs in flight,
+// skips the combine (both CTAs of the pair), frees its TMEM and exits.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tmap.h"
+
+namespace pkm {
+
+namespace sl {
+constexpr int kM = 128;           // tokens per tile (TMEM lanes)
+constexpr int kN = 256;           // sub-key columns per chunk
+constexpr int kKB = 64;           // k-block width (128 bytes of bf16)
+constexpr int kStages = 2;
+constexpr int kABytes = kM * kKB * 2;   // 16 KiB
+constexpr int kBBytes = kN * kKB * 2;   // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr int kBuf = 16;          // pending candidates per row
+constexpr int kFlushAt = 8;       // merge once a row holds more (checked every 8 columns)
+constexpr int kMaxK = 32;
+constexpr int kGroup = 4;         // columns per group maximum in the histogram pass
+constexpr int kBins = 64;         // histogram bins per row, one byte each
+constexpr float kBinsPerUnit = 16.0f;
+constexpr float kBinOffset = 16.0f;     // bin = floor(16 s + 16) over [-1, 3): bin 1 starts at -15/16
+constexpr int kPendBytes = kBuf * kM * 4 + kBuf * kM * 2;   // p (fp32) and column (u16)
+// a row's bins are the words [w][row] of the fp32 part of the pending buffers,
+// which hold only that row's entries: no row's bins overlap another row's data
+static_assert(kBins / 4 <= kBuf, "the histogram aliases the row's own fp32 entries");
+static_assert(kN / kGroup <= 255, "bin counts fit in a byte");
+constexpr int kRkBytes = 4 * kN * 4;                        // each epilogue warp's chunk norms
+constexpr int kCombRows = kM / 2;                           // rows combined per CTA
+constexpr size_t kSmemBytes =
+    (size_t)kStages * kStageBytes + kPendBytes + kRkBytes + 256 /*barriers*/;
+// after the last MMA the stage ring holds the CTA's lists [32][128] keys
+// (32 KiB) in stage 0, and in stage 1 both halves' lists of the rows this
+// CTA combines (scores and positions, [2][32][65]) and their heaps
+constexpr int kHeapPad = kCombRows + 1;
+static_assert(kMaxK * kM * 8 <= kStageBytes, "lists fit in stage 0");
+static_assert(2 * kMaxK * kHeapPad * 6 + (kMaxK + 2) * kHeapPad * 6 + kMaxK * kHeapPad * 2 <=
+                  kStageBytes,
+              "both halves' lists of the combined rows and the heaps fit in stage 1");
+}  // namespace sl
+
+struct SelectCtl {
+  uint64_t full[sl::kStages];
+  uint64_t empty[sl::kStages];
+  uint64_t aread[sl::kStages];  // the epilogue has read the query rows of a first-chunk stage
+  uint64_t accf;
+  uint64_t acce;
+  uint64_t drain;
+  uint32_t tmem;
+  volatile int abort;
+};
+
+// ------------------------------------------------------------- cluster --
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// every thread of both CTAs arrives, then waits (release / acquire)
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint64_t ld_cluster_u64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// 16 columns of the accumulator; the wait names the registers so that no
+// use of them is moved above it
+__device__ __forceinline__ void tmem_wait_x16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+
+// ---------------------------------------------------------------- keys --
+
+// a row's candidate: the order-preserving bits of the score above the
+// complemented column, so that equal scores order the smaller column first
+using Key = uint64_t;
+__device__ __forceinline__ uint32_t ord_score(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ Key make_key(float s, int col) {
+  s += 0.0f;  // -0 -> +0: both zeros are one score
+  return ((uint64_t)ord_score(s) << 32) | (uint64_t)(0xffffffffu - (uint32_t)col);
+}
+__device__ __forceinline__ float key_score(Key k) {
+  const uint32_t u = (uint32_t)(k >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+__device__ __forceinline__ int key_col(Key k) { return (int)(0xffffffffu - (uint32_t)k); }
+// the empty slot: below every score's key
+__device__ __forceinline__ Key empty_key() { return 0ull; }
+__device__ __forceinline__ Key key_max(Key a, Key b) { return a > b ? a : b; }
+__device__ __forceinline__ Key key_min(Key a, Key b) { return a > b ? b : a; }
+
+#define SL_CAS(a, b)            \
+  {                             \
+    const Key x_ = (a);         \
+    (a) = key_max(x_, (b));     \
+    (b) = key_min(x_, (b));     \
+  }
+
+// sort 16 keys descending (bitonic network)
+__device__ __forceinline__ void sort16_desc(Key* v) {
+#pragma unroll
+  for (int size = 2; size <= 16; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          if ((i & size) == 0) {
+            SL_CAS(v[i], v[j]);
+          } else {
+            SL_CAS(v[j], v[i]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// L (sorted desc, 32) <- top 32 of L u B (B sorted desc, 16): the larger of
+// L[i] and B[31-i] for i >= 16 makes L bitonic, five exchange stages sort it
+__device__ __forceinline__ void merge16_desc(Key* L, const Key* B) {
+#pragma unroll
+  for (int i = 16; i < 32; ++i) L[i] = key_max(L[i], B[31 - i]);
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & stride) == 0) SL_CAS(L[i], L[i + stride]);
+    }
+  }
+}
+
+// thr_raw <- max(thr_raw, a filter level for the raw products): any column
+// whose score s = p * rowf (rounded) is >= thr has p above the returned
+// level, which is thr * (1/rowf) lowered by 2^-20 relative (more than the
+// two roundings of the estimate).  A level that overflows is ignored.
+__device__ __forceinline__ void raise_threshold(float& thr_raw, float thr, float inv_rowf) {
+  const float r = thr * inv_rowf;
+  const float t = r - fabsf(r) * 9.5367431640625e-7f;
+  if (fabsf(t) < INFINITY) thr_raw = fmaxf(thr_raw, t);
+}
+
+// Merge the row's pending candidates (cnt entries of p and column, at a
+// stride of 128) into its sorted list L, empty the buffer and raise the
+// filter level to the list's k-th best.
+template <bool K32>
+__device__ __forceinline__ void flush_pending(Key (&L)[32], const float* pp,
+                                              const uint16_t* pc, int& cnt, float& thr_raw,
+                                              int k, float rowf, float inv_rowf) {
+  Key B[sl::kBuf];
+#pragma unroll
+  for (int j = 0; j < sl::kBuf; ++j)
+    B[j] = j < cnt ? make_key(pp[j * sl::kM] * rowf, (int)pc[j * sl::kM]) : empty_key();
+  sort16_desc(B);
+  merge16_desc(L, B);
+  cnt = 0;
+  Key kth;
+  if constexpr (K32) {
+    kth = L[31];
+  } else {
+    kth = L[0];
+#pragma unroll
+    for (int i = 1; i < 32; ++i)
+      if (i == k - 1) kth = L[i];
+  }
+  if (kth != empty_key()) raise_threshold(thr_raw, key_score(kth), inv_rowf);
+}
+
+// ------------------------------------------------------------- combine --
+
+__device__ __forceinline__ uint32_t ord_of(float s) {
+  uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One thread per (token, head).  s1/a1: the first half's k best (scores,
+// positions; best first), s2/b2 the second half's, at a stride of
+// kHeapPad.  The k x k grid S[i][j] = s1[i] + s2[j] decreases along rows and
+// columns, so its cells can be taken best first with a max-heap frontier:
+// start at (0, 0); taking (i, j) admits (i, j+1) and, on the first column,
+// (i+1, 0).  Equal scores are ordered by the row id a*n+b (smaller first).
+// Writes the k row ids and softmax weights of the row.
+__device__ void combine_row(const float* s1, const uint16_t* a1, const float* s2,
+                            const uint16_t* b2, uint32_t* hk, uint16_t* hc, uint16_t* rec, int n,
+                            int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  constexpr int P = sl::kHeapPad;
+  auto id_of = [&](int cell) { return (int32_t)a1[(cell >> 6) * P] * n + (int32_t)b2[(cell & 63) * P]; };
+  auto ahead = [&](uint32_t s, int c, uint32_t t, int d) {
+    return s != t ? s > t : id_of(c) < id_of(d);
+  };
+  auto score_at = [&](int i, int j) { return ord_of(s1[i * P] + s2[j * P]); };
+  int size = 0;
+  auto push = [&](uint32_t key, int cell) {
+    int pos = ++size;
+    while (pos > 1) {
+      const int par = pos >> 1;
+      const uint32_t pk = hk[par * P];
+      const int pcell = hc[par * P];
+      if (!ahead(key, cell, pk, pcell)) break;
+      hk[pos * P] = pk;
+      hc[pos * P] = (uint16_t)pcell;
+      pos = par;
+    }
+    hk[pos * P] = key;
+    hc[pos * P] = (uint16_t)cell;
+  };
+  push(score_at(0, 0), 0);
+  for (int r = 0; r < k; ++r) {
+    const int cell = hc[1 * P];
+    const uint32_t lk = hk[size * P];
+    const int lc = hc[size * P];
+    --size;
+    int pos = 1;
+    while (true) {
+      int ch = pos * 2;
+      if (ch > size) break;
+      uint32_t ck = hk[ch * P];
+      int cc = hc[ch * P];
+      if (ch < size) {
+        const uint32_t k2 = hk[(ch + 1) * P];
+        const int c2 = hc[(ch + 1) * P];
+        if (ahead(k2, c2, ck, cc)) {
+          ck = k2;
+          cc = c2;
+          ++ch;
+        }
+      }
+      if (!ahead(ck, cc, lk, lc)) break;
+      hk[pos * P] = ck;
+      hc[pos * P] = (uint16_t)cc;
+      pos = ch;
+    }
+    if (size > 0 || pos > 1) {
+      hk[pos * P] = lk;
+      hc[pos * P] = (uint16_t)lc;
+    }
+    rec[r * P] = (uint16_t)cell;
+    const int i = cell >> 6, j = cell & 63;
+    if (j + 1 < k) push(score_at(i, j + 1), i * 64 + j + 1);
+    if (j == 0 && i + 1 < k) push(score_at(i + 1, 0), (i + 1) * 64);
+  }
+  // softmax over the k kept scores; the first is the maximum
+  const int c0 = rec[0];
+  const float m = s1[(c0 >> 6) * P] + s2[(c0 & 63) * P];
+  float z = 0.f;
+  for (int r = 0; r < k; ++r) {
+    const int c = rec[r * P];
+    z += expf(s1[(c >> 6) * P] + s2[(c & 63) * P] - m);
+  }
+  const float inv = 1.0f / z;
+  for (int r = 0; r < k; ++r) {
+    const int c = rec[r * P];
+    const int i = c >> 6, j = c & 63;
+    idx_out[r] = id_of(c);
+    w_out[r] = expf(s1[i * P] + s2[j * P] - m) * inv;
+  }
+}
+
+// bounded wait that also gives up when another role of the CTA aborted
+__device__ __forceinline__ bool wait_sel(uint64_t* bar, uint32_t parity, SelectCtl* ctl,
+                                         int32_t* status) {
+  return mbar_wait_or_abort(bar, parity, &ctl->abort, status);
+}
+
+// The products p = acc * rk of 16 columns (norms from the warp's shared
+// copy of the chunk's inverse sub-key norms); columns at or past ncols read
+// as -inf.
+__device__ __forceinline__ void products16(const uint32_t (&r)[16], const float* rkw, int g,
+                                           int ncols, float (&p)[16]) {
+  const float4* kv = reinterpret_cast<const float4*>(rkw + g * 16);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 v = kv[q];
+    p[4 * q + 0] = __uint_as_float(r[4 * q + 0]) * v.x;
+    p[4 * q + 1] = __uint_as_float(r[4 * q + 1]) * v.y;
+    p[4 * q + 2] = __uint_as_float(r[4 * q + 2]) * v.z;
+    p[4 * q + 3] = __uint_as_float(r[4 * q + 3]) * v.w;
+  }
+  if (g * 16 + 16 > ncols) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (g * 16 + j >= ncols) p[j] = -INFINITY;
+  }
+}
+
+template <bool K32>
+__global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t T,
+    int H, int dh, int n, int k, const float* __restrict__ rk, int32_t* __restrict__ idx,
+    float* __restrict__ wout, int32_t* status) {
+  using namespace sl;
+  // dynamic shared memory starts 1024-byte aligned (the 128-byte swizzle of
+  // the TMA tiles needs it); checked below
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* stages = smem_raw;
+  float* pend_p = reinterpret_cast<float*>(smem_raw + kStages * kStageBytes);  // [kBuf][128]
+  uint16_t* pend_c = reinterpret_cast<uint16_t*>(pend_p + kBuf * kM);          // [kBuf][128]
+  unsigned char* hist = reinterpret_cast<unsigned char*>(pend_p);  // words [kBins/4][128]
+  float* rkbuf = reinterpret_cast<float*>(smem_raw + kStages * kStageBytes + kPendBytes);
+  SelectCtl* ctl =
+      reinterpret_cast<SelectCtl*>(smem_raw + kStages * kStageBytes + kPendBytes + kRkBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hc = blockIdx.y;  // 2h + half
+  const int h = hc >> 1;
+  const uint32_t crank = cluster_ctarank();  // the half: (h, 0) and (h, 1) pair up
+  const int64_t m0 = (int64_t)blockIdx.x * kM;
+  const int nch = (n + kN - 1) / kN;
+  const int KB = dh / kKB;
+  const bool misaligned = (smem_u32(smem_raw) & 1023u) != 0;  // the same in every CTA
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+      mbar_init(&ctl->aread[s], 4);
+    }
+    mbar_init(&ctl->accf, 1);
+    mbar_init(&ctl->acce, 4);
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = misaligned ? 1 : 0;
+    if (misaligned) set_status(status, PKM_ERR_DEVICE);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1 && !misaligned) {
+    tmem_alloc(&ctl->tmem, kN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem;
+  const bool run = !misaligned;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0 && run) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_par = 0;
+      bool ok = true;
+      int f = 0;  // stage fills so far
+      for (int c = 0; c < nch && ok; ++c) {
+        for (int kb = 0; kb < KB; ++kb, ++f) {
+          if (!wait_sel(&ctl->empty[stage], phase ^ 1, ctl, status)) { ok = false; break; }
+          // a first-chunk stage is refilled only after the epilogue read its query rows
+          if (f >= kStages && f - kStages < KB &&
+              !wait_sel(&ctl->aread[stage], ((f - kStages) / kStages) & 1, ctl, status)) {
+            ok = false;
+            break;
+          }
+          unsigned char* sa = stages + stage * kStageBytes;
+          mbar_arrive_expect_tx(&ctl->full[stage], kStageBytes);
+          tma_load_3d(sa, &tmA, &ctl->full[stage], kb * kKB, hc, (int32_t)m0);
+          tma_load_3d(sa + kABytes, &tmB, &ctl->full[stage], kb * kKB, c * kN, hc);
+          issued_mask |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {  // let every copy in flight land before the CTA moves on
+        for (int s = 0; s < kStages; ++s)
+          if (issued_mask & (1u << s)) {
+            for (unsigned long long i = 0; i < kSpinLimit; ++i)
+              if (mbar_try_wait(&ctl->full[s], (issued_par >> s) & 1)) break;
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0 && run) {
+      const uint32_t idesc = idesc_bf16_f32(kM, kN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      uint32_t use = 0;
+      for (int c = 0; c < nch && ok; ++c, use ^= 1) {
+        // the accumulator is free once the epilogue has read the last chunk
+        if (!wait_sel(&ctl->acce, use ^ 1, ctl, status)) { ok = false; break; }
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!wait_sel(&ctl->full[stage], phase, ctl, status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stages + stage * kStageBytes);
+          const uint32_t sb = sa + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kKB / 16; ++kk)
+            tc_mma_f16(tmem, smem_desc_k128(sa + kk * 32), smem_desc_k128(sb + kk * 32), idesc,
+                       (kb | kk) != 0);
+          tc_commit(&ctl->empty[stage]);  // the stage is free once these MMAs finish
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (ok) tc_commit(&ctl->accf);
+      }
+      // every MMA issued must complete before TMEM is released
+      tc_commit(&ctl->drain);
+      for (unsigned long long i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(&ctl->drain, 0)) break;
+    }
+  } else if (run) {
+    // ----------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may read
+    const int row = quarter * 32 + lane;
+    const int64_t t = m0 + row;
+    const bool live = t < T;
+    float* pp = pend_p + row;   // entry j at pp[128 j]
+    uint16_t* pc = pend_c + row;
+    float* rkw = rkbuf + (warp - 2) * kN;  // this warp's copy of the chunk's norms
+    const float* rkc = rk + (int64_t)hc * n;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+
+    // 1. the row's query norm from the first chunk's stages
+    float ss = 0.f;
+    for (int kb = 0; kb < KB; ++kb) {
+      const int stage = kb % kStages;
+      const bool got = wait_sel(&ctl->full[stage], (kb / kStages) & 1, ctl, status);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      const uint4* arow = reinterpret_cast<const uint4*>(stages + stage * kStageBytes + row * 128);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint4 v = arow[u];
+        float f[8];
+        unpack16<PKM_BF16>(v, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->aread[stage]);
+    }
+    const float rq = 1.0f / fmaxf(sqrtf(ss), kNormEps);
+    const float rowf = sqrtf((float)dh) * rq;
+    const float inv_rowf = 1.0f / rowf;
+
+    Key L[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) L[i] = empty_key();
+    int cnt = 0;
+    // rows past the end of the batch keep nothing
+    float thr_raw = live ? -INFINITY : INFINITY;
+
+    // 2. the chunks
+    float4 kn0 = make_float4(0.f, 0.f, 0.f, 0.f), kn1 = kn0;
+    if (ok) {
+      const float4* src = reinterpret_cast<const float4*>(rkc + lane * 8);
+      kn0 = __ldg(src);
+      kn1 = __ldg(src + 1);
+    }
+    for (int it = 0; it < nch && ok; ++it) {
+      const int c0 = it * kN;
+      const int ncols = min(kN, n - c0);
+      __syncwarp();  // every lane is done with the previous chunk's norms
+      reinterpret_cast<float4*>(rkw + lane * 8)[0] = kn0;
+      reinterpret_cast<float4*>(rkw + lane * 8)[1] = kn1;
+      __syncwarp();
+      if (it + 1 < nch) {  // the norm buffer is padded by a chunk: in bounds
+        const float4* src = reinterpret_cast<const float4*>(rkc + c0 + kN + lane * 8);
+        kn0 = __ldg(src);
+        kn1 = __ldg(src + 1);
+      }
+      const bool got = wait_sel(&ctl->accf, it & 1, ctl, status);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem + lane_base;
+      uint32_t ra[16], rb[16];
+
+      if (it == 0) {
+        // histogram pass: maxima of groups of 4 columns into score bins
+        uint32_t* hw = reinterpret_cast<uint32_t*>(hist) + row;  // word w at hw[128 w]
+#pragma unroll
+        for (int w = 0; w < kBins / 4; ++w) hw[w * kM] = 0u;
+        unsigned char* hb = hist + row * 4;  // bin b at hb[512 (b >> 2) + (b & 3)]
+        const float c16 = rowf * kBinsPerUnit;
+        auto count = [&](const uint32_t (&r)[16], int g) {
+          float p[16];
+          products16(r, rkw, g, ncols, p);
+#pragma unroll
+          for (int q = 0; q < 16 / kGroup; ++q) {
+            const float gm = fmaxf(fmaxf(p[4 * q], p[4 * q + 1]), fmaxf(p[4 * q + 2], p[4 * q + 3]));
+            const float tb = fminf(fmaxf(fmaf(gm, c16, kBinOffset), 0.f), (float)(kBins - 1));
+            const int b = (int)tb;
+            hb[512 * (b >> 2) + (b & 3)] += 1;
+          }
+        };
+        tmem_ld_32x32b_x16(taddr, ra);
+        tmem_wait_x16(ra);
+        for (int g = 0; g < kN / 16; g += 2) {
+          tmem_ld_32x32b_x16(taddr + (g + 1) * 16, rb);
+          count(ra, g);
+          tmem_wait_x16(rb);
+          if (g + 2 < kN / 16) tmem_ld_32x32b_x16(taddr + (g + 2) * 16, ra);
+          count(rb, g + 1);
+          if (g + 2 < kN / 16) tmem_wait_x16(ra);
+        }
+        // the bound: lower edge of the bin where the count from the top reaches k
+        int cum = 0, bstar = 0;
+        for (int w = kBins / 4 - 1; w >= 0; --w) {
+          const uint32_t word = hw[w * kM];
+          const int s4 = (int)__dp4a(word, 0x01010101u, 0u);
+          if (cum + s4 >= k) {
+            for (int e = 3; e >= 0; --e) {
+              cum += (int)((word >> (8 * e)) & 255u);
+              if (cum >= k) { bstar = 4 * w + e; break; }
+            }
+            break;
+          }
+          cum += s4;
+        }
+        // members of bin b >= 1 have s >= (b - 16) / 16 up to rounding; 2^-10 covers it
+        if (bstar > 0)
+          raise_threshold(thr_raw, ((float)bstar - kBinOffset) / kBinsPerUnit - 9.765625e-4f,
+                          inv_rowf);
+        __syncwarp();  // the bins become the pending buffers
+      }
+
+      // filter pass: products above the level into the row's buffer
+      auto filter = [&](const uint32_t (&r)[16], int g) {
+        float p[16];
+        products16(r, rkw, g, ncols, p);
+        const int col0 = c0 + g * 16;
+#pragma unroll
+        for (int hh = 0; hh < 16; hh += 8) {
+#pragma unroll
+          for (int j = hh; j < hh + 8; ++j) {
+            if (p[j] > thr_raw) {
+              pp[cnt * kM] = p[j];
+              pc[cnt * kM] = (uint16_t)(col0 + j);
+              ++cnt;
+            }
+          }
+          if (__any_sync(0xffffffffu, cnt > kFlushAt))
+            flush_pending<K32>(L, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
+        }
+      };
+      tmem_ld_32x32b_x16(taddr, ra);
+      tmem_wait_x16(ra);
+      for (int g = 0; g < kN / 16; g += 2) {
+        tmem_ld_32x32b_x16(taddr + (g + 1) * 16, rb);
+        filter(ra, g);
+        tmem_wait_x16(rb);
+        if (g + 2 < kN / 16) tmem_ld_32x32b_x16(taddr + (g + 2) * 16, ra);
+        filter(rb, g + 1);
+        if (g + 2 < kN / 16) tmem_wait_x16(ra);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->acce);
+    }
+    if (ok) {
+      if (__any_sync(0xffffffffu, cnt > 0))
+        flush_pending<K32>(L, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
+      // the sorted list into stage 0 (free: the CTA's last MMA has completed)
+      Key* list = reinterpret_cast<Key*>(stages);  // [32][128]
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < k) list[i * kM + row] = L[i];
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1 && run) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kN);
+  }
+
+  // ------------------------------------------------ k x k combine (cluster)
+  cluster_sync_all();  // both CTAs' lists are in their shared memory
+  const uint32_t peer = crank ^ 1u;
+  const int peer_abort = ld_cluster_s32(map_to_rank(smem_u32((const void*)&ctl->abort), peer));
+  const bool combine = ctl->abort == 0 && peer_abort == 0;
+  if (combine) {
+    constexpr int P = kHeapPad;
+    const Key* own = reinterpret_cast<const Key*>(stages);
+    const uint32_t peer_list = map_to_rank(smem_u32(stages), peer);
+    unsigned char* s1b = stages + kStageBytes;
+    float* sv = reinterpret_cast<float*>(s1b);                       // [2][32][P] scores
+    uint16_t* cv = reinterpret_cast<uint16_t*>(sv + 2 * kMaxK * P);  // [2][32][P] positions
+    uint32_t* hk = reinterpret_cast<uint32_t*>(cv + 2 * kMaxK * P);  // heap keys [k+2][P]
+    uint16_t* hcell = reinterpret_cast<uint16_t*>(hk + (kMaxK + 2) * P);  // heap cells [k+2][P]
+    uint16_t* rec = hcell + (kMaxK + 2) * P;                         // taken cells [k][P]
+    const int r0 = (int)crank * kCombRows;
+    // both halves' lists of the combined rows: half c at sv[c][j][rl]
+    for (int e = threadIdx.x; e < 2 * k * kCombRows; e += kThreads) {
+      const int half = e / (k * kCombRows);
+      const int j = (e / kCombRows) % k;
+      const int rl = e % kCombRows;
+      const int src = j * kM + r0 + rl;
+      const Key key = half == (int)crank ? own[src] : ld_cluster_u64(peer_list + src * 8);
+      sv[(half * kMaxK + j) * P + rl] = key_score(key);
+      cv[(half * kMaxK + j) * P + rl] = (uint16_t)key_col(key);
+    }
+    __syncthreads();
+    if (threadIdx.x < kCombRows) {
+      const int rl = threadIdx.x;
+      const int64_t t = m0 + r0 + rl;
+      if (t < T) {
+        const int64_t o = (t * H + h) * k;
+        combine_row(sv + rl, cv + rl, sv + kMaxK * P + rl, cv + kMaxK * P + rl, hk + rl,
+                    hcell + rl, rec + rl, n, k, idx + o, wout + o);
+      }
+    }
+  }
+  cluster_sync_all();  // the peer has finished reading this CTA's lists
+}
+
+bool select_tc_supported(pkm_dtype dt, int dh, int n, int k) {
+  // n % 4: the epilogue reads the inverse sub-key norms as aligned float4;
+  // n < 65536: positions are held as 16 bits
+  return dt == PKM_BF16 && dh % sl::kKB == 0 && dh <= 2048 && n >= sl::kN && n % 4 == 0 &&
+         n < 65536 && k <= sl::kMaxK;
+}
+
+cudaError_t launch_select_tc(const void* q, const void* K, int64_t T, int H, int dh, int n,
+                             int k, const float* rk, int32_t* idx, float* w, int32_t* status,
+                             cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  CUtensorMap tmA, tmB;
+  {
+    const uint64_t dims[3] = {(uint64_t)dh, (uint64_t)H * 2, (uint64_t)T};
+    const uint64_t strides[2] = {(uint64_t)dh * 2, (uint64_t)H * 2 * dh * 2};
+    const uint32_t box[3] = {(uint32_t)sl::kKB, 1, (uint32_t)sl::kM};
+    if (!make_tmap_bf16(&tmA, q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)dh, (uint64_t)n, (uint64_t)H * 2};
+    const uint64_t strides[2] = {(uint64_t)dh * 2, (uint64_t)n * dh * 2};
+    const uint32_t box[3] = {(uint32_t)sl::kKB, (uint32_t)sl::kN, 1};
+    if (!make_tmap_bf16(&tmB, K, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  auto kern = k == 32 ? select_tc_kernel<true> : select_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sl::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((T + sl::kM - 1) / sl::kM), (unsigned)(H * 2), 1);
+  cfg.blockDim = dim3(sl::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = sl::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = 2;  // (h, half 0) and (h, half 1)
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, T, H, dh, n, k, rk, idx, w, status);
+  note_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+}  // namespace pkm

@@ -15,6 +15,12 @@ void note_launch(int n = 1);
 // Device address of the current device's sticky status word.
 int32_t* status_ptr();
 
+// Upper bound of T in every entry point: keeps all size products in range.
+constexpr int64_t kMaxTokens = int64_t(1) << 36;
+
+// The forward's argument checks without the workspace (PKM_OK or the error).
+pkm_status check_fwd_args(const pkm_fwd_args* a);
+
 // pkm_forward with a library-chosen workspace, and the workspace size it needs.
 pkm_status forward_into(const pkm_fwd_args* a, void* workspace, size_t workspace_bytes,
                         cudaStream_t st);
@@ -39,6 +45,15 @@ int score_tc_splits(int64_t T, int H, int n);
 cudaError_t launch_score_topk_tc(const void* q, const void* K, int64_t T, int H, int dh, int n,
                                  int k, int splits, const float* rq, const float* rk, float* hv,
                                  int32_t* hi, int32_t* status, cudaStream_t stream);
+
+// The whole selection in one kernel (k_select_tc.cu): query norms, scores
+// on the tensor cores, per-half top-k, k x k combine, top-k and softmax ->
+// idx [T,H,k], w [T,H,k].  bf16, d_half % 64 == 0, 256 <= n < 65536,
+// n % 4 == 0, k <= 32; rk [2H*n + 256] (padded) from launch_row_rnorm.
+bool select_tc_supported(pkm_dtype dt, int dh, int n, int k);
+cudaError_t launch_select_tc(const void* q, const void* K, int64_t T, int H, int dh, int n,
+                             int k, const float* rk, int32_t* idx, float* w, int32_t* status,
+                             cudaStream_t stream);
 
 // Merge the split lists, combine the two halves' k x k candidates, keep the
 // top k, softmax -> idx [T,H,k] (a*n+b), w [T,H,k].
@@ -75,20 +90,23 @@ cudaError_t launch_gate_mul_bf16(const void* y, const void* g, int64_t n, void* 
 // dst[c][r] = src[r][c]; dst rows are ld >= rows long, zero past rows (ld <= 0: ld = rows).
 cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst,
                                   cudaStream_t stream, int ld = 0);
-// C[M,N] = epi(A[M,K] * B[N,K]^T), A/B bf16 K-major; epi: 0 none, 1 silu.
-// Optional `mul` [M,N] bf16 multiplies the result after the epilogue.
+// C[M,N] = epi(A[M,K] * B[N,K]^T) in bf16; epi: 0 none, 1 silu.  A is
+// [M][K]; B is [N][K], or [K][N] with b_mn (a weight [d_in, d_out] used as x W).
 bool gemm_tc_supported(int64_t M, int N, int K);
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                             void* C, int32_t* status, cudaStream_t stream);
-// C[M,N] (fp32) = A[M,K] B[N,K]^T, or C += it when accumulate.
+                             void* C, int32_t* status, cudaStream_t stream, bool b_mn = false);
+// C[M,N] (fp32) = A B^T, or C += it when accumulate; A [M][K] or, with a_mn,
+// [K][M]; B [N][K] or, with b_mn, [K][N].
 cudaError_t launch_gemm_f32(const void* A, const void* B, int64_t M, int N, int K,
-                            bool accumulate, float* C, int32_t* status, cudaStream_t stream);
+                            bool accumulate, float* C, int32_t* status, cudaStream_t stream,
+                            bool a_mn = false, bool b_mn = false);
 // The same (C overwritten) split over K into slices when the output has few
 // tiles (weight gradients contracting over tokens): partial products in
 // `part` (gemm_splitk_workspace bytes), summed in slice order.
 size_t gemm_splitk_workspace(int64_t M, int N, int K);
 cudaError_t launch_gemm_f32_splitk(const void* A, const void* B, int64_t M, int N, int K,
-                                   float* C, float* part, int32_t* status, cudaStream_t stream);
+                                   float* C, float* part, int32_t* status, cudaStream_t stream,
+                                   bool a_mn = false, bool b_mn = false);
 
 // In-place SGD / touched-rows Adam on the rows of a sparse value gradient
 // (see k_sparse_opt.cu); m, v are [n_rows, d] fp32 Adam moments.

@@ -37,9 +37,10 @@ static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // ------------------------------------------------------------ forward ----
 
 struct FwdLayout {
-  size_t rq, rk, hv, hi, w1t, w2t, g, z, part, total;
+  size_t rq, rk, hv, hi, g, z, part, total;
   int splits;
   bool tc;
+  bool fused;  // the one-kernel selection (k_select_tc.cu)
 };
 
 static bool has_memplus(const pkm_fwd_args* a) { return a->x || a->W1 || a->W2; }
@@ -48,7 +49,11 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
   FwdLayout L{};
   const size_t T = (size_t)(a->T > 0 ? a->T : 0);
   const size_t H = (size_t)a->H, n = (size_t)a->n_sub, k = (size_t)a->k;
-  L.tc = score_tc_supported(a->dtype, a->d_half, a->n_sub, a->k);
+  // batches beyond the decode sizes run the one-kernel selection; small ones
+  // split the sub-key columns over CTAs (score_topk_tc) and combine apart
+  L.fused = select_tc_supported(a->dtype, a->d_half, a->n_sub, a->k) &&
+            a->T > kSplitGatherMaxBags;
+  L.tc = !L.fused && score_tc_supported(a->dtype, a->d_half, a->n_sub, a->k);
   L.splits = L.tc ? score_tc_splits(a->T, a->H, a->n_sub) : 1;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -56,15 +61,15 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
     off = round_up(off + bytes, 256);
     return o;
   };
-  L.rq = take(T * H * 2 * sizeof(float));
-  // padded by one chunk of columns: the scoring epilogue reads 8 at a time
+  // padded by one chunk of columns: the scoring epilogues read 8 at a time
   L.rk = take((H * 2 * n + 256) * sizeof(float));
-  L.hv = take((size_t)L.splits * T * H * 2 * k * sizeof(float));
-  L.hi = take((size_t)L.splits * T * H * 2 * k * sizeof(int32_t));
+  if (!L.fused) {
+    L.rq = take(T * H * 2 * sizeof(float));
+    L.hv = take((size_t)L.splits * T * H * 2 * k * sizeof(float));
+    L.hi = take((size_t)L.splits * T * H * 2 * k * sizeof(int32_t));
+  }
   if (has_memplus(a)) {
-    const size_t dm = (size_t)a->d_model, dv = (size_t)a->d_v;
-    L.w1t = take(dv * dm * 2);
-    L.w2t = take(dm * dv * 2);
+    const size_t dv = (size_t)a->d_v;
     L.g = take(T * dv * 2);
     L.z = take(T * dv * 2);
   }
@@ -75,9 +80,12 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
   return L;
 }
 
-static pkm_status validate_fwd(const pkm_fwd_args* a) {
+// Arguments of a forward, without the workspace (sizes, dtype, pointers).
+// T is bounded so that no workspace size computed from the arguments wraps.
+pkm_status check_fwd_args(const pkm_fwd_args* a) {
   if (!a) return PKM_ERR_INVALID_ARG;
-  if (a->T < 0 || a->H < 1 || a->n_sub < 1 || a->k < 1 || a->k > 64 || a->k > a->n_sub)
+  if (a->T < 0 || a->T > kMaxTokens || a->H < 1 || a->n_sub < 1 || a->k < 1 || a->k > 64 ||
+      a->k > a->n_sub)
     return PKM_ERR_INVALID_ARG;
   if (a->d_half < 8 || a->d_half % 8 || a->d_v < 8 || a->d_v % 8) return PKM_ERR_INVALID_ARG;
   if ((int64_t)a->n_sub * a->n_sub >= (int64_t(1) << 31)) return PKM_ERR_INVALID_ARG;
@@ -95,6 +103,12 @@ static pkm_status validate_fwd(const pkm_fwd_args* a) {
     if (a->d_model < 8 || a->d_model % 8) return PKM_ERR_INVALID_ARG;
     if (a->dtype != PKM_BF16) return PKM_ERR_UNSUPPORTED;
   }
+  return PKM_OK;
+}
+
+static pkm_status validate_fwd(const pkm_fwd_args* a) {
+  const pkm_status s = check_fwd_args(a);
+  if (s != PKM_OK || a->T == 0) return s;
   const FwdLayout L = fwd_layout(a);
   if (!a->workspace || !aligned16(a->workspace) || a->workspace_bytes < L.total)
     return PKM_ERR_WORKSPACE;
@@ -107,9 +121,16 @@ static pkm_status validate_fwd(const pkm_fwd_args* a) {
     if (e_ != cudaSuccess) return PKM_ERR_CUDA; \
   } while (0)
 
+// Phase event i on the stream; under stream capture it becomes an event
+// record node of the graph, so replays time their phases too.
 static void mark(const pkm_fwd_args* a, int i, cudaStream_t st) {
-  if (a->phase_events && a->phase_events[i])
-    cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), st);
+  if (a->phase_events && a->phase_events[i]) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) cs = cudaStreamCaptureStatusNone;
+    cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a->phase_events[i]), st,
+                             cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                 : cudaEventRecordDefault);
+  }
 }
 
 static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
@@ -127,35 +148,37 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
   const int64_t N = (int64_t)n * n;
   const bool mp = has_memplus(a);
   const int dm = a->d_model, dv = a->d_v;
-  void* w1t = mp ? ws + L.w1t : nullptr;
-  void* w2t = mp ? ws + L.w2t : nullptr;
   char* g = mp ? ws + L.g : nullptr;
   char* z = mp ? ws + L.z : nullptr;
 
-  // a1: qk-normalisation factors
+  // a1: qk-normalisation factors (the query's inside the one-kernel selection)
   mark(a, 0, st);
-  PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
+  if (!L.fused) PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
   PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
   mark(a, 1, st);
 
-  // a2 + a3: sub-key scores and per-half top-k
-  if (L.tc)
-    PKM_TRY(launch_score_topk_tc(a->query, a->subkeys, T, H, dh, n, k, L.splits, rq, rk, hv, hi,
-                                 status, st));
-  else
-    PKM_TRY(launch_score_topk_simt(a->query, a->subkeys, a->dtype, T, H, dh, n, k, rq, rk, hv,
-                                   hi, st));
-  mark(a, 2, st);
-  // a4 + a5: k x k combine, top-k, softmax
-  PKM_TRY(launch_combine(hv, hi, L.splits, T, H, n, k, a->idx, a->weights, st));
+  if (L.fused) {
+    // a1 (query) + a2 .. a5 in one kernel
+    PKM_TRY(launch_select_tc(a->query, a->subkeys, T, H, dh, n, k, rk, a->idx, a->weights,
+                             status, st));
+    mark(a, 2, st);
+  } else {
+    // a2 + a3: sub-key scores and per-half top-k
+    if (L.tc)
+      PKM_TRY(launch_score_topk_tc(a->query, a->subkeys, T, H, dh, n, k, L.splits, rq, rk, hv,
+                                   hi, status, st));
+    else
+      PKM_TRY(launch_score_topk_simt(a->query, a->subkeys, a->dtype, T, H, dh, n, k, rq, rk,
+                                     hv, hi, st));
+    mark(a, 2, st);
+    // a4 + a5: k x k combine, top-k, softmax
+    PKM_TRY(launch_combine(hv, hi, L.splits, T, H, n, k, a->idx, a->weights, st));
+  }
   mark(a, 3, st);
   if (select_only) return PKM_OK;
   // (a7) gate GEMM, a6 bag gather over the H*k selected rows of each token
-  if (mp) {
-    PKM_TRY(launch_transpose_bf16(a->W1, dm, dv, w1t, st));  // [dv, dm]
-    PKM_TRY(launch_transpose_bf16(a->W2, dv, dm, w2t, st));  // [dm, dv]
-    PKM_TRY(launch_gemm_bf16(a->x, w1t, T, dv, dm, /*silu*/ 1, g, status, st));
-  }
+  if (mp)  // g = silu(x W1), W1 [d_model][d_v] read as it is held
+    PKM_TRY(launch_gemm_bf16(a->x, a->W1, T, dv, dm, /*silu*/ 1, g, status, st, /*b_mn*/ true));
   mark(a, 4, st);
   // with y_out the bag output is kept and the gate applied in a second pass
   const void* gate = a->y_out ? nullptr : g;
@@ -169,7 +192,8 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
                               bag_out, status, st));
   if (a->y_out) PKM_TRY(launch_gate_mul_bf16(a->y_out, g, T * dv, z, st));
   mark(a, 5, st);
-  if (mp) PKM_TRY(launch_gemm_bf16(z, w2t, T, dm, dv, /*none*/ 0, a->out, status, st));
+  if (mp)  // out = z W2, W2 [d_v][d_model] read as it is held
+    PKM_TRY(launch_gemm_bf16(z, a->W2, T, dm, dv, /*none*/ 0, a->out, status, st, true));
   mark(a, 6, st);
   return PKM_OK;
 }
@@ -185,7 +209,8 @@ static pkm_fwd_args select_args(const pkm_fwd_args* a) {
 }
 
 static pkm_status validate_select(const pkm_fwd_args* b) {
-  if (b->T < 0 || b->H < 1 || b->n_sub < 1 || b->k < 1 || b->k > 64 || b->k > b->n_sub)
+  if (b->T < 0 || b->T > kMaxTokens || b->H < 1 || b->n_sub < 1 || b->k < 1 || b->k > 64 ||
+      b->k > b->n_sub)
     return PKM_ERR_INVALID_ARG;
   if (b->d_half < 8 || b->d_half % 8 || b->d_v < 8 || b->d_v % 8) return PKM_ERR_INVALID_ARG;
   if ((int64_t)b->n_sub * b->n_sub >= (int64_t(1) << 31)) return PKM_ERR_INVALID_ARG;

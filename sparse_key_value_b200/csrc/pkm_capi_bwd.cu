@@ -48,7 +48,8 @@ BwdLayout bwd_layout(const pkm_bwd_args* a) {
 
 pkm_status validate_bwd(const pkm_bwd_args* a) {
   if (!a) return PKM_ERR_INVALID_ARG;
-  if (a->T < 0 || a->H < 1 || a->n_sub < 1 || a->k < 1 || a->k > 64 || a->k > a->n_sub)
+  if (a->T < 0 || a->T > kMaxTokens || a->H < 1 || a->n_sub < 1 || a->k < 1 || a->k > 64 ||
+      a->k > a->n_sub)
     return PKM_ERR_INVALID_ARG;
   if (a->d_half < 8 || a->d_half % 8 || a->d_v < 8 || a->d_v % 8) return PKM_ERR_INVALID_ARG;
   if ((int64_t)a->n_sub * a->n_sub >= (int64_t(1) << 31)) return PKM_ERR_INVALID_ARG;

@@ -5,9 +5,11 @@
 // Per token, a = x W1, g = silu(a), z = y ⊙ g:
 //   dz = dout W2^T, dy = dz ⊙ g, da = dz ⊙ y ⊙ silu'(a), dx = da W1^T,
 //   dW1 = x^T da, dW2 = z^T dout.
-// The products run on the tcgen05 GEMM (A B^T with both operands K-major,
-// fp32 accumulation); the token-contracting weight gradients take transposed
-// copies of their operands with the token dimension padded to 64 by zeros.
+// The products run on the tcgen05 GEMM (fp32 accumulation), every operand
+// read in the layout it is held: W1 [d_model][d_v] as the MN-major B of x W1,
+// and the token rows x, da, z, dout as MN-major operands of the weight
+// gradients, which contract over the tokens (split over K when the output
+// has few tiles, the slices summed in order).
 #include <math.h>
 
 #include "common.cuh"
@@ -18,7 +20,6 @@ namespace pkm {
 namespace {
 
 size_t rup(size_t x) { return (x + 255) / 256 * 256; }
-int64_t pad_tokens(int64_t T) { return (T + 63) / 64 * 64; }
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 #define PKM_TRY(expr)                           \
@@ -57,30 +58,24 @@ unsigned elem_grid(int64_t n) {
 }
 
 struct MpLayout {
-  size_t w1t, a, dz, da, z, xt, dat, zt, dot, part, total;
+  size_t a, dz, da, z, part, total;
 };
 
 MpLayout mp_layout(const pkm_memplus_bwd_args* g) {
   MpLayout L{};
   const size_t T = (size_t)(g->T > 0 ? g->T : 0), dm = (size_t)g->d_model, dv = (size_t)g->d_v;
-  const size_t Tp = (size_t)pad_tokens((int64_t)T);
   size_t off = 0;
   auto take = [&](size_t b) {
     const size_t o = off;
     off += rup(b);
     return o;
   };
-  L.w1t = take(dv * dm * 2);
   L.a = take(T * dv * 4);
   L.dz = take(T * dv * 4);
   L.da = take(T * dv * 2);
   L.z = take(T * dv * 2);
-  L.xt = take(dm * Tp * 2);
-  L.dat = take(dv * Tp * 2);
-  L.zt = take(dv * Tp * 2);
-  L.dot = take(dm * Tp * 2);
-  const size_t p1 = gemm_splitk_workspace((int64_t)dm, (int)dv, (int)Tp);
-  const size_t p2 = gemm_splitk_workspace((int64_t)dv, (int)dm, (int)Tp);
+  const size_t p1 = gemm_splitk_workspace((int64_t)dm, (int)dv, (int)T);
+  const size_t p2 = gemm_splitk_workspace((int64_t)dv, (int)dm, (int)T);
   L.part = take(p1 > p2 ? p1 : p2);
   L.total = off;
   return L;
@@ -104,24 +99,20 @@ pkm_status mp_validate(const pkm_memplus_bwd_args* g) {
 }
 
 struct QpLayout {
-  size_t wqt, dqb, dqt, xt, part, total;
+  size_t dqb, part, total;
 };
 
 QpLayout qp_layout(const pkm_qproj_args* g) {
   QpLayout L{};
   const size_t T = (size_t)(g->T > 0 ? g->T : 0), dm = (size_t)g->d_model, dq = (size_t)g->d_q;
-  const size_t Tp = (size_t)pad_tokens((int64_t)T);
   size_t off = 0;
   auto take = [&](size_t b) {
     const size_t o = off;
     off += rup(b);
     return o;
   };
-  L.wqt = take(dq * dm * 2);
   L.dqb = take(T * dq * 2);
-  L.dqt = take(dq * Tp * 2);
-  L.xt = take(dm * Tp * 2);
-  L.part = take(gemm_splitk_workspace((int64_t)dm, (int)dq, (int)Tp));
+  L.part = take(gemm_splitk_workspace((int64_t)dm, (int)dq, (int)T));
   L.total = off;
   return L;
 }
@@ -175,15 +166,12 @@ pkm_status memplus_backward_impl(const pkm_memplus_bwd_args* g, cudaStream_t st)
   }
   const MpLayout L = mp_layout(g);
   char* ws = static_cast<char*>(g->workspace);
-  const int64_t Tp = pad_tokens(T);
-  auto* w1t = ws + L.w1t;
   auto* a = reinterpret_cast<float*>(ws + L.a);
   auto* dz = reinterpret_cast<float*>(ws + L.dz);
   auto* da = reinterpret_cast<__nv_bfloat16*>(ws + L.da);
   auto* z = reinterpret_cast<__nv_bfloat16*>(ws + L.z);
-  // a = x W1 (W1 transposed to [d_v, d_model]), dz = dout W2^T (W2 is [d_v, d_model])
-  PKM_TRY(launch_transpose_bf16(g->W1, dm, dv, w1t, st));
-  PKM_TRY(launch_gemm_f32(g->x, w1t, T, dv, dm, false, a, status, st));
+  // a = x W1 (W1 [d_model][d_v] read as held), dz = dout W2^T (W2 is [d_v, d_model])
+  PKM_TRY(launch_gemm_f32(g->x, g->W1, T, dv, dm, false, a, status, st, false, /*b_mn*/ true));
   PKM_TRY(launch_gemm_f32(g->dout, g->W2, T, dv, dm, false, dz, status, st));
   const int64_t n = T * dv;
   memplus_bwd_elem_kernel<<<elem_grid(n), 256, 0, st>>>(
@@ -193,16 +181,13 @@ pkm_status memplus_backward_impl(const pkm_memplus_bwd_args* g, cudaStream_t st)
   PKM_TRY(cudaGetLastError());
   // dx = da W1^T (W1 is [d_model, d_v])
   PKM_TRY(launch_gemm_f32(da, g->W1, T, dm, dv, false, g->dx, status, st));
-  // dW1 = x^T da, dW2 = z^T dout: contract over the (zero-padded) tokens
-  PKM_TRY(launch_transpose_bf16(g->x, (int)T, dm, ws + L.xt, st, (int)Tp));
-  PKM_TRY(launch_transpose_bf16(da, (int)T, dv, ws + L.dat, st, (int)Tp));
-  PKM_TRY(launch_transpose_bf16(z, (int)T, dv, ws + L.zt, st, (int)Tp));
-  PKM_TRY(launch_transpose_bf16(g->dout, (int)T, dm, ws + L.dot, st, (int)Tp));
+  // dW1 = x^T da, dW2 = z^T dout: contract over the tokens, every operand read
+  // as held ([T][d] rows: MN-major for these products)
   float* part = reinterpret_cast<float*>(ws + L.part);
-  PKM_TRY(launch_gemm_f32_splitk(ws + L.xt, ws + L.dat, dm, dv, (int)Tp, g->dW1, part, status,
-                                 st));
-  PKM_TRY(launch_gemm_f32_splitk(ws + L.zt, ws + L.dot, dv, dm, (int)Tp, g->dW2, part, status,
-                                 st));
+  PKM_TRY(launch_gemm_f32_splitk(g->x, da, dm, dv, (int)T, g->dW1, part, status, st, true,
+                                 true));
+  PKM_TRY(launch_gemm_f32_splitk(z, g->dout, dv, dm, (int)T, g->dW2, part, status, st, true,
+                                 true));
   return PKM_OK;
 }
 
@@ -234,9 +219,10 @@ PKM_API pkm_status pkm_qproj_forward(const pkm_qproj_args* g, pkm_stream_t strea
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const QpLayout L = qp_layout(g);
   char* ws = static_cast<char*>(g->workspace);
-  // q = x Wq with Wq transposed to [d_q, d_model]
-  PKM_TRY(launch_transpose_bf16(g->Wq, g->d_model, g->d_q, ws + L.wqt, st));
-  PKM_TRY(launch_gemm_bf16(g->x, ws + L.wqt, g->T, g->d_q, g->d_model, 0, g->q, status, st));
+  // q = x Wq, Wq [d_model][d_q] read as held
+  (void)L;
+  (void)ws;
+  PKM_TRY(launch_gemm_bf16(g->x, g->Wq, g->T, g->d_q, g->d_model, 0, g->q, status, st, true));
   return PKM_OK;
 }
 
@@ -253,18 +239,16 @@ PKM_API pkm_status pkm_qproj_backward(const pkm_qproj_args* g, pkm_stream_t stre
   if (!status) return PKM_ERR_CUDA;
   const QpLayout L = qp_layout(g);
   char* ws = static_cast<char*>(g->workspace);
-  const int64_t T = g->T, Tp = pad_tokens(T);
+  const int64_t T = g->T;
   const int dm = g->d_model, dq = g->d_q;
   auto* dqb = reinterpret_cast<__nv_bfloat16*>(ws + L.dqb);
   f32_to_bf16_kernel<<<elem_grid(T * dq), 256, 0, st>>>(g->dq, T * dq, dqb);
   note_launch();
   PKM_TRY(cudaGetLastError());
-  // dx += dq Wq^T (Wq is [d_model, d_q]); dWq = x^T dq over the padded tokens
+  // dx += dq Wq^T (Wq is [d_model, d_q]); dWq = x^T dq over the tokens
   PKM_TRY(launch_gemm_f32(dqb, g->Wq, T, dm, dq, true, g->dx, status, st));
-  PKM_TRY(launch_transpose_bf16(g->x, (int)T, dm, ws + L.xt, st, (int)Tp));
-  PKM_TRY(launch_transpose_bf16(dqb, (int)T, dq, ws + L.dqt, st, (int)Tp));
-  PKM_TRY(launch_gemm_f32_splitk(ws + L.xt, ws + L.dqt, dm, dq, (int)Tp, g->dWq,
-                                 reinterpret_cast<float*>(ws + L.part), status, st));
+  PKM_TRY(launch_gemm_f32_splitk(g->x, dqb, dm, dq, (int)T, g->dWq,
+                                 reinterpret_cast<float*>(ws + L.part), status, st, true, true));
   return PKM_OK;
 }
 

@@ -50,7 +50,9 @@ void* noalloc_scratch() {
 
 extern "C" pkm_status pkm_forward_noalloc(const pkm_fwd_args* args, pkm_stream_t stream) {
   using namespace pkm;
-  if (!args) return PKM_ERR_INVALID_ARG;
+  // invalid arguments are refused as such before any size is computed from them
+  const pkm_status s = check_fwd_args(args);
+  if (s != PKM_OK || args->T == 0) return s;
   // the sizes alone decide the scratch need; refuse anything beyond the array
   if (forward_workspace_bytes(args) > kNoAllocScratchBytes) return PKM_ERR_WORKSPACE;
   void* scratch = noalloc_scratch();

@@ -154,6 +154,22 @@ def value_table(w: Workload, device) -> torch.Tensor:
     return out
 
 
+def value_shard(w: Workload, n_rows: int, rank: int, device) -> torch.Tensor:
+    """[n_rows, d_v] rows N(0, 0.02) standing in for one rank's share of the
+    value table in a row-sharded run: the same distribution as value_table,
+    drawn from the rank's own stream (not the full table's values)."""
+    out = torch.empty(max(0, n_rows), w.d_v, dtype=w.torch_dtype, device=device)
+    g = torch.Generator(device=device)
+    g.manual_seed(w.table_seed * 1000003 + 7 + rank)
+    chunk = max(1, (32 << 20) // w.d_v)
+    for r0 in range(0, n_rows, chunk):
+        r1 = min(n_rows, r0 + chunk)
+        tmp = torch.randn(r1 - r0, w.d_v, generator=g, device=device, dtype=torch.float32)
+        out[r0:r1].copy_(tmp.mul_(0.02))
+        del tmp
+    return out
+
+
 def _zipf_direction(w: Workload, g: torch.Generator) -> torch.Tensor:
     e = torch.randn(w.H, 2, w.d_half, generator=g, dtype=torch.float32)
     return e / e.norm(dim=-1, keepdim=True)

@@ -63,6 +63,27 @@ class TorchComm:
         return out
 
 
+class LocalComm:
+    """The exchange of a single rank: the all-gather stacks its one input and
+    the reduce-scatter returns it."""
+
+    world, rank = 1, 0
+
+    def all_gather(self, t: torch.Tensor) -> torch.Tensor:
+        return t.unsqueeze(0)
+
+    def reduce_scatter_sum(self, t: torch.Tensor) -> torch.Tensor:
+        return t
+
+
+def exchange_bytes(T: int, H: int, k: int, d_v: int, world: int) -> dict:
+    """Bytes one rank receives per step: the other ranks' selections (ids
+    and weights, 8 bytes per entry) in the all-gather, and their partial
+    bags of this rank's tokens (fp32) in the reduce-scatter."""
+    return {"all_gather": (world - 1) * T * H * k * 8,
+            "reduce_scatter": (world - 1) * T * d_v * 4}
+
+
 def sharded_lookup(query, subkeys, values_shard, k: int, row_lo: int, comm, select=None,
                    gather=None):
     """One rank's step of the row-sharded lookup (steps 1-4 above).

@@ -82,6 +82,46 @@ def test_forward_small(case):
     run_forward(w)
 
 
+
+# Batches of more than 64 tokens with bf16, d_half % 64 == 0, n >= 256,
+# n % 4 == 0 and k <= 32 run the one-kernel selection (query norms, scores,
+# per-half top-k, k x k combine and softmax in one launch, the two halves of
+# a head in a cluster of two CTAs); smaller batches split the sub-key columns
+# over CTAs and combine in a second kernel.
+FUSED = [
+    # name, T, H, d_half, n_sub, k, d_v
+    ("fused-k32-ragged-tile", 333, 2, 64, 512, 32, 64),
+    ("fused-k7-three-heads", 200, 3, 128, 768, 7, 32),
+    ("fused-ragged-chunk", 129, 1, 192, 1100, 32, 16),
+    ("fused-k1", 65, 2, 64, 256, 1, 16),
+    ("fused-wide-query", 160, 2, 512, 2048, 32, 32),
+    ("fused-many-chunks", 130, 1, 64, 4096, 32, 16),
+    ("fused-k31", 300, 1, 256, 300, 31, 24),
+]
+
+
+@pytest.mark.parametrize("case", FUSED, ids=[c[0] for c in FUSED])
+def test_forward_fused_selection(case):
+    name, T, H, dh, n, k, dv = case
+    w = WORKLOADS["pkm"].scaled(name=name, T=T, H=H, d_half=dh, n_sub=n, k=k, d_v=dv,
+                                dtype="bf16", seed=sum(map(ord, name)))
+    run_forward(w)
+
+
+def test_forward_fused_launches():
+    """A batch on the one-kernel selection launches three kernels in all:
+    the sub-key norms, the selection and the bag gather."""
+    w = WORKLOADS["pkm"].scaled(T=300, H=2, d_half=64, n_sub=512, k=32, d_v=64)
+    inp = make_inputs(w, "cuda")
+    lib = skv.load()
+    skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k)
+    torch.cuda.synchronize()
+    c0 = lib.pkm_launch_count()
+    skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k)
+    torch.cuda.synchronize()
+    assert lib.pkm_launch_count() - c0 == 3
+    assert skv.device_error() == 0
+
 @pytest.mark.parametrize("sign", [1.0, -1.0], ids=["aligned", "anti-aligned"])
 def test_forward_extreme_scores(sign):
     """Queries (anti-)aligned with every sub-key of their (head, half): the
