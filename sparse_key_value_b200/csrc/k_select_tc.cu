@@ -9,9 +9,9 @@
 // best of each half are combined (a 1,000 x 1,000 grid searched with 2,000
 // comparisons) and the values read are averaged with weights.
 //
-// Grid: (token tiles of 128) x (2H); the two CTAs (h, half 0) and (h, half 1)
-// of a token tile form a cluster of two.  Each CTA scores its 128 tokens
-// against all n sub-keys of its (head, half), 256 columns per chunk:
+// Grid: (token tiles of 128) x (2H), one CTA per (token tile, head, half).
+// Each CTA scores its 128 tokens against all n sub-keys of its (head, half),
+// 256 columns per chunk:
 //   warp 0     TMA producer: per chunk and 64-wide k-block the query tile
 //              [128 x 64] and the sub-key tile [256 x 64] (bf16, 128-byte
 //              swizzle) into a 2-stage ring.
@@ -45,17 +45,20 @@
 // Measured: packing the column into the low mantissa bits of an fp64 key
 // and exchanging with fp64 min/max ran 2.5x slower on B200.
 //
-// Combine: each CTA writes its rows' sorted lists to shared memory; after a
-// cluster barrier, CTA c takes rows [64c, 64c+64), copies the other half's
-// lists for them from the peer CTA's shared memory (DSMEM), and one thread
-// per row runs the max-heap frontier over the k x k grid S[i][j] = s1[i] +
-// s2[j] (rows and columns non-increasing), keeps k cells, forms the row ids
-// a*n+b and the softmax weights and writes them.  A second cluster barrier
-// keeps each CTA's shared memory alive until its peer has read it.
+// Combine: each CTA writes its rows' sorted lists to the workspace (they
+// stay in L2), then counts itself in on its (token tile, head) pair with an
+// atomic after a fence; the second CTA of the pair to arrive reads both
+// halves' lists back and, one thread per token, runs the max-heap frontier
+// over the k x k grid S[i][j] = s1[i] + s2[j] (rows and columns
+// non-increasing), keeps k cells, forms the row ids a*n+b and the softmax
+// weights and writes them.  The first CTA of the pair just exits.  (A 2-CTA
+// cluster exchanging the lists through distributed shared memory was
+// measured first: cluster launch held this kernel to one CTA per SM.)
 //
 // Every spin-wait is bounded: on a timeout the CTA records PKM_ERR_TIMEOUT,
 // stops issuing work, waits (bounded) for its copies and MMAs in flight,
-// skips the combine (both CTAs of the pair), frees its TMEM and exits.
+// marks its half's lists invalid (the pair is then not combined), frees its
+// TMEM and exits.
 #include <math.h>
 
 #include "common.cuh"
@@ -86,17 +89,15 @@ constexpr int kPendBytes = kBuf * kM * 4 + kBuf * kM * 2;   // p (fp32) and colu
 static_assert(kBins / 4 <= kBuf, "the histogram aliases the row's own fp32 entries");
 static_assert(kN / kGroup <= 255, "bin counts fit in a byte");
 constexpr int kRkBytes = 4 * kN * 4;                        // each epilogue warp's chunk norms
-constexpr int kCombRows = kM / 2;                           // rows combined per CTA
 constexpr size_t kSmemBytes =
     (size_t)kStages * kStageBytes + kPendBytes + kRkBytes + 256 /*barriers*/;
-// after the last MMA the stage ring holds the CTA's lists [32][128] keys
-// (32 KiB) in stage 0, and in stage 1 both halves' lists of the rows this
-// CTA combines (scores and positions, [2][32][65]) and their heaps
-constexpr int kHeapPad = kCombRows + 1;
-static_assert(kMaxK * kM * 8 <= kStageBytes, "lists fit in stage 0");
+// after the last MMA the stage ring holds the combine's arrays: both halves'
+// lists (scores and positions, [2][32][129]) and the heaps, one column per row
+constexpr int kHeapPad = kM + 1;
 static_assert(2 * kMaxK * kHeapPad * 6 + (kMaxK + 2) * kHeapPad * 6 + kMaxK * kHeapPad * 2 <=
-                  kStageBytes,
-              "both halves' lists of the combined rows and the heaps fit in stage 1");
+                  kStages * kStageBytes,
+              "both halves' lists and the heaps fit in the stage ring");
+constexpr int kListKeys = kMaxK * kM;  // keys of one (tile, head, half) list block [32][128]
 }  // namespace sl
 
 struct SelectCtl {
@@ -108,42 +109,22 @@ struct SelectCtl {
   uint64_t drain;
   uint32_t tmem;
   volatile int abort;
+  int combine;  // this CTA is the second of its pair and both halves are valid
 };
 
-// ------------------------------------------------------------- cluster --
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// every thread of both CTAs arrives, then waits (release / acquire)
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ uint64_t ld_cluster_u64(uint32_t addr) {
+// L2-coherent load (skips L1): the other CTA of the pair wrote these
+__device__ __forceinline__ uint64_t ld_cg_u64(const uint64_t* p) {
   uint64_t v;
-  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 
-// 16 columns of the accumulator; the wait names the registers so that no
-// use of them is moved above it
-__device__ __forceinline__ void tmem_wait_x16(uint32_t (&r)[16]) {
+// 8 columns of the accumulator; the wait names the registers so that no use
+// of them is moved above it
+__device__ __forceinline__ void tmem_wait_x8(uint32_t (&r)[8]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 "+r"(r[6]), "+r"(r[7])
                :
                : "memory");
 }
@@ -345,24 +326,25 @@ __device__ __forceinline__ bool wait_sel(uint64_t* bar, uint32_t parity, SelectC
   return mbar_wait_or_abort(bar, parity, &ctl->abort, status);
 }
 
-// The products p = acc * rk of 16 columns (norms from the warp's shared
-// copy of the chunk's inverse sub-key norms); columns at or past ncols read
-// as -inf.
-__device__ __forceinline__ void products16(const uint32_t (&r)[16], const float* rkw, int g,
-                                           int ncols, float (&p)[16]) {
-  const float4* kv = reinterpret_cast<const float4*>(rkw + g * 16);
+// The products p = acc * rk of 8 columns (norms from the warp's shared copy
+// of the chunk's inverse sub-key norms, read as broadcasts); columns at or
+// past ncols read as -inf.
+__device__ __forceinline__ void products8(const uint32_t (&r)[8], const float* rkw, int g,
+                                          int ncols, float (&p)[8]) {
+  const float4* kv = reinterpret_cast<const float4*>(rkw + g * 8);
+  const float4 a = kv[0], b = kv[1];
+  p[0] = __uint_as_float(r[0]) * a.x;
+  p[1] = __uint_as_float(r[1]) * a.y;
+  p[2] = __uint_as_float(r[2]) * a.z;
+  p[3] = __uint_as_float(r[3]) * a.w;
+  p[4] = __uint_as_float(r[4]) * b.x;
+  p[5] = __uint_as_float(r[5]) * b.y;
+  p[6] = __uint_as_float(r[6]) * b.z;
+  p[7] = __uint_as_float(r[7]) * b.w;
+  if (g * 8 + 8 > ncols) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 v = kv[q];
-    p[4 * q + 0] = __uint_as_float(r[4 * q + 0]) * v.x;
-    p[4 * q + 1] = __uint_as_float(r[4 * q + 1]) * v.y;
-    p[4 * q + 2] = __uint_as_float(r[4 * q + 2]) * v.z;
-    p[4 * q + 3] = __uint_as_float(r[4 * q + 3]) * v.w;
-  }
-  if (g * 16 + 16 > ncols) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (g * 16 + j >= ncols) p[j] = -INFINITY;
+    for (int j = 0; j < 8; ++j)
+      if (g * 8 + j >= ncols) p[j] = -INFINITY;
   }
 }
 
@@ -370,7 +352,8 @@ template <bool K32>
 __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t T,
     int H, int dh, int n, int k, const float* __restrict__ rk, int32_t* __restrict__ idx,
-    float* __restrict__ wout, int32_t* status) {
+    float* __restrict__ wout, uint64_t* __restrict__ lists, int32_t* __restrict__ pair_count,
+    int32_t* __restrict__ half_ok, int32_t* status) {
   using namespace sl;
   // dynamic shared memory starts 1024-byte aligned (the 128-byte swizzle of
   // the TMA tiles needs it); checked below
@@ -386,7 +369,6 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hc = blockIdx.y;  // 2h + half
   const int h = hc >> 1;
-  const uint32_t crank = cluster_ctarank();  // the half: (h, 0) and (h, 1) pair up
   const int64_t m0 = (int64_t)blockIdx.x * kM;
   const int nch = (n + kN - 1) / kN;
   const int KB = dh / kKB;
@@ -549,7 +531,7 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + lane_base;
-      uint32_t ra[16], rb[16];
+      uint32_t nxt[8], cur[8];
 
       if (it == 0) {
         // histogram pass: maxima of groups of 4 columns into score bins
@@ -558,26 +540,22 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
         for (int w = 0; w < kBins / 4; ++w) hw[w * kM] = 0u;
         unsigned char* hb = hist + row * 4;  // bin b at hb[512 (b >> 2) + (b & 3)]
         const float c16 = rowf * kBinsPerUnit;
-        auto count = [&](const uint32_t (&r)[16], int g) {
-          float p[16];
-          products16(r, rkw, g, ncols, p);
+        tmem_ld_32x32b_x8(taddr, nxt);
+#pragma unroll 1
+        for (int g = 0; g < kN / 8; ++g) {
+          tmem_wait_x8(nxt);
 #pragma unroll
-          for (int q = 0; q < 16 / kGroup; ++q) {
+          for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
+          if (g + 1 < kN / 8) tmem_ld_32x32b_x8(taddr + (g + 1) * 8, nxt);
+          float p[8];
+          products8(cur, rkw, g, ncols, p);
+#pragma unroll
+          for (int q = 0; q < 8 / kGroup; ++q) {
             const float gm = fmaxf(fmaxf(p[4 * q], p[4 * q + 1]), fmaxf(p[4 * q + 2], p[4 * q + 3]));
             const float tb = fminf(fmaxf(fmaf(gm, c16, kBinOffset), 0.f), (float)(kBins - 1));
-            const int b = (int)tb;
-            hb[512 * (b >> 2) + (b & 3)] += 1;
+            const int bin = (int)tb;
+            hb[512 * (bin >> 2) + (bin & 3)] += 1;
           }
-        };
-        tmem_ld_32x32b_x16(taddr, ra);
-        tmem_wait_x16(ra);
-        for (int g = 0; g < kN / 16; g += 2) {
-          tmem_ld_32x32b_x16(taddr + (g + 1) * 16, rb);
-          count(ra, g);
-          tmem_wait_x16(rb);
-          if (g + 2 < kN / 16) tmem_ld_32x32b_x16(taddr + (g + 2) * 16, ra);
-          count(rb, g + 1);
-          if (g + 2 < kN / 16) tmem_wait_x16(ra);
         }
         // the bound: lower edge of the bin where the count from the top reaches k
         int cum = 0, bstar = 0;
@@ -600,34 +578,28 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
         __syncwarp();  // the bins become the pending buffers
       }
 
-      // filter pass: products above the level into the row's buffer
-      auto filter = [&](const uint32_t (&r)[16], int g) {
-        float p[16];
-        products16(r, rkw, g, ncols, p);
-        const int col0 = c0 + g * 16;
+      // filter pass: products above the level into the row's buffer; one
+      // merge site for the whole loop keeps the code (and its misses) small
+      tmem_ld_32x32b_x8(taddr, nxt);
+#pragma unroll 1
+      for (int g = 0; g < kN / 8; ++g) {
+        tmem_wait_x8(nxt);
 #pragma unroll
-        for (int hh = 0; hh < 16; hh += 8) {
+        for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
+        if (g + 1 < kN / 8) tmem_ld_32x32b_x8(taddr + (g + 1) * 8, nxt);
+        float p[8];
+        products8(cur, rkw, g, ncols, p);
+        const int col0 = c0 + g * 8;
 #pragma unroll
-          for (int j = hh; j < hh + 8; ++j) {
-            if (p[j] > thr_raw) {
-              pp[cnt * kM] = p[j];
-              pc[cnt * kM] = (uint16_t)(col0 + j);
-              ++cnt;
-            }
+        for (int j = 0; j < 8; ++j) {
+          if (p[j] > thr_raw) {
+            pp[cnt * kM] = p[j];
+            pc[cnt * kM] = (uint16_t)(col0 + j);
+            ++cnt;
           }
-          if (__any_sync(0xffffffffu, cnt > kFlushAt))
-            flush_pending<K32>(L, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
         }
-      };
-      tmem_ld_32x32b_x16(taddr, ra);
-      tmem_wait_x16(ra);
-      for (int g = 0; g < kN / 16; g += 2) {
-        tmem_ld_32x32b_x16(taddr + (g + 1) * 16, rb);
-        filter(ra, g);
-        tmem_wait_x16(rb);
-        if (g + 2 < kN / 16) tmem_ld_32x32b_x16(taddr + (g + 2) * 16, ra);
-        filter(rb, g + 1);
-        if (g + 2 < kN / 16) tmem_wait_x16(ra);
+        if (__any_sync(0xffffffffu, cnt > kFlushAt))
+          flush_pending<K32>(L, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
       }
       tc_fence_before();
       __syncwarp();
@@ -636,11 +608,12 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     if (ok) {
       if (__any_sync(0xffffffffu, cnt > 0))
         flush_pending<K32>(L, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
-      // the sorted list into stage 0 (free: the CTA's last MMA has completed)
-      Key* list = reinterpret_cast<Key*>(stages);  // [32][128]
+      // the sorted list into this (tile, head, half)'s block [32][128] of the workspace
+      uint64_t* list = lists + ((int64_t)blockIdx.x * gridDim.y + hc) * kListKeys;
 #pragma unroll
       for (int i = 0; i < 32; ++i)
         if (i < k) list[i * kM + row] = L[i];
+      __threadfence();  // the list is visible device-wide before the pair count below
     }
   }
 
@@ -651,44 +624,50 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     tmem_dealloc(tmem, kN);
   }
 
-  // ------------------------------------------------ k x k combine (cluster)
-  cluster_sync_all();  // both CTAs' lists are in their shared memory
-  const uint32_t peer = crank ^ 1u;
-  const int peer_abort = ld_cluster_s32(map_to_rank(smem_u32((const void*)&ctl->abort), peer));
-  const bool combine = ctl->abort == 0 && peer_abort == 0;
-  if (combine) {
+  // -------------------------------------------------------- k x k combine
+  // count this half in on its (tile, head) pair; the second to arrive combines
+  const int64_t pair = (int64_t)blockIdx.x * H + h;
+  if (threadIdx.x == 0) {
+    half_ok[pair * 2 + (hc & 1)] = ctl->abort == 0 ? 1 : 0;
+    __threadfence();  // this CTA's lists and flag before the count
+    const int prev = atomicAdd(pair_count + pair, 1);
+    int go = 0;
+    if (prev == 1) {
+      __threadfence();  // the other half's lists and flag after the count
+      const volatile int32_t* other = half_ok + pair * 2 + ((hc & 1) ^ 1);
+      go = ctl->abort == 0 && *other != 0;
+    }
+    ctl->combine = go;
+  }
+  __syncthreads();
+  if (ctl->combine) {
     constexpr int P = kHeapPad;
-    const Key* own = reinterpret_cast<const Key*>(stages);
-    const uint32_t peer_list = map_to_rank(smem_u32(stages), peer);
-    unsigned char* s1b = stages + kStageBytes;
-    float* sv = reinterpret_cast<float*>(s1b);                       // [2][32][P] scores
+    float* sv = reinterpret_cast<float*>(stages);                    // [2][32][P] scores
     uint16_t* cv = reinterpret_cast<uint16_t*>(sv + 2 * kMaxK * P);  // [2][32][P] positions
     uint32_t* hk = reinterpret_cast<uint32_t*>(cv + 2 * kMaxK * P);  // heap keys [k+2][P]
     uint16_t* hcell = reinterpret_cast<uint16_t*>(hk + (kMaxK + 2) * P);  // heap cells [k+2][P]
     uint16_t* rec = hcell + (kMaxK + 2) * P;                         // taken cells [k][P]
-    const int r0 = (int)crank * kCombRows;
-    // both halves' lists of the combined rows: half c at sv[c][j][rl]
-    for (int e = threadIdx.x; e < 2 * k * kCombRows; e += kThreads) {
-      const int half = e / (k * kCombRows);
-      const int j = (e / kCombRows) % k;
-      const int rl = e % kCombRows;
-      const int src = j * kM + r0 + rl;
-      const Key key = half == (int)crank ? own[src] : ld_cluster_u64(peer_list + src * 8);
-      sv[(half * kMaxK + j) * P + rl] = key_score(key);
-      cv[(half * kMaxK + j) * P + rl] = (uint16_t)key_col(key);
+    const uint64_t* pl = lists + ((int64_t)blockIdx.x * gridDim.y + 2 * h) * kListKeys;
+    // both halves' lists of the tile's rows (L2): half c's entry j of row r at sv[c][j][r]
+    for (int e = threadIdx.x; e < 2 * k * kM; e += kThreads) {
+      const int half = e / (k * kM);
+      const int j = (e / kM) % k;
+      const int r = e % kM;
+      const Key key = ld_cg_u64(pl + (int64_t)half * kListKeys + j * kM + r);
+      sv[(half * kMaxK + j) * P + r] = key_score(key);
+      cv[(half * kMaxK + j) * P + r] = (uint16_t)key_col(key);
     }
     __syncthreads();
-    if (threadIdx.x < kCombRows) {
-      const int rl = threadIdx.x;
-      const int64_t t = m0 + r0 + rl;
+    if (threadIdx.x < kM) {
+      const int r = threadIdx.x;
+      const int64_t t = m0 + r;
       if (t < T) {
         const int64_t o = (t * H + h) * k;
-        combine_row(sv + rl, cv + rl, sv + kMaxK * P + rl, cv + kMaxK * P + rl, hk + rl,
-                    hcell + rl, rec + rl, n, k, idx + o, wout + o);
+        combine_row(sv + r, cv + r, sv + kMaxK * P + r, cv + kMaxK * P + r, hk + r, hcell + r,
+                    rec + r, n, k, idx + o, wout + o);
       }
     }
   }
-  cluster_sync_all();  // the peer has finished reading this CTA's lists
 }
 
 bool select_tc_supported(pkm_dtype dt, int dh, int n, int k) {
@@ -698,10 +677,23 @@ bool select_tc_supported(pkm_dtype dt, int dh, int n, int k) {
          n < 65536 && k <= sl::kMaxK;
 }
 
+size_t select_tc_workspace(int64_t T, int H) {
+  const size_t tiles = (size_t)((T + sl::kM - 1) / sl::kM);
+  const size_t lists = tiles * H * 2 * sl::kListKeys * sizeof(uint64_t);
+  const size_t counts = (tiles * H * 3 * sizeof(int32_t) + 255) / 256 * 256;
+  return lists + counts;
+}
+
 cudaError_t launch_select_tc(const void* q, const void* K, int64_t T, int H, int dh, int n,
-                             int k, const float* rk, int32_t* idx, float* w, int32_t* status,
-                             cudaStream_t stream) {
+                             int k, const float* rk, int32_t* idx, float* w, void* workspace,
+                             int32_t* status, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
+  const int64_t tiles = (T + sl::kM - 1) / sl::kM;
+  uint64_t* lists = static_cast<uint64_t*>(workspace);
+  int32_t* pair_count = reinterpret_cast<int32_t*>(lists + tiles * H * 2 * sl::kListKeys);
+  int32_t* half_ok = pair_count + tiles * H;
+  cudaError_t e = cudaMemsetAsync(pair_count, 0, sizeof(int32_t) * tiles * H, stream);
+  if (e != cudaSuccess) return e;
   CUtensorMap tmA, tmB;
   {
     const uint64_t dims[3] = {(uint64_t)dh, (uint64_t)H * 2, (uint64_t)T};
@@ -716,24 +708,14 @@ cudaError_t launch_select_tc(const void* q, const void* K, int64_t T, int H, int
     if (!make_tmap_bf16(&tmB, K, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   auto kern = k == 32 ? select_tc_kernel<true> : select_tc_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)sl::kSmemBytes);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sl::kSmemBytes);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((T + sl::kM - 1) / sl::kM), (unsigned)(H * 2), 1);
-  cfg.blockDim = dim3(sl::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = sl::kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = 1;
-  at[0].val.clusterDim.y = 2;  // (h, half 0) and (h, half 1)
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, T, H, dh, n, k, rk, idx, w, status);
+  dim3 grid((unsigned)tiles, (unsigned)(H * 2), 1);
+  kern<<<grid, sl::kThreads, sl::kSmemBytes, stream>>>(tmA, tmB, T, H, dh, n, k, rk, idx, w,
+                                                       lists, pair_count, half_ok, status);
   note_launch();
-  return e != cudaSuccess ? e : cudaGetLastError();
+  return cudaGetLastError();
 }
 
 }  // namespace pkm

@@ -49,11 +49,14 @@ cudaError_t launch_score_topk_tc(const void* q, const void* K, int64_t T, int H,
 // The whole selection in one kernel (k_select_tc.cu): query norms, scores
 // on the tensor cores, per-half top-k, k x k combine, top-k and softmax ->
 // idx [T,H,k], w [T,H,k].  bf16, d_half % 64 == 0, 256 <= n < 65536,
-// n % 4 == 0, k <= 32; rk [2H*n + 256] (padded) from launch_row_rnorm.
+// n % 4 == 0, k <= 32; rk [2H*n + 256] (padded) from launch_row_rnorm;
+// `workspace` (select_tc_workspace bytes, 256-aligned) holds the per-half
+// lists the two CTAs of a (token tile, head) exchange and their counters.
 bool select_tc_supported(pkm_dtype dt, int dh, int n, int k);
+size_t select_tc_workspace(int64_t T, int H);
 cudaError_t launch_select_tc(const void* q, const void* K, int64_t T, int H, int dh, int n,
-                             int k, const float* rk, int32_t* idx, float* w, int32_t* status,
-                             cudaStream_t stream);
+                             int k, const float* rk, int32_t* idx, float* w, void* workspace,
+                             int32_t* status, cudaStream_t stream);
 
 // Merge the split lists, combine the two halves' k x k candidates, keep the
 // top k, softmax -> idx [T,H,k] (a*n+b), w [T,H,k].

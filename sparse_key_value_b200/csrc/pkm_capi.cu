@@ -37,7 +37,7 @@ static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // ------------------------------------------------------------ forward ----
 
 struct FwdLayout {
-  size_t rq, rk, hv, hi, g, z, part, total;
+  size_t rq, rk, hv, hi, sel, g, z, part, total;
   int splits;
   bool tc;
   bool fused;  // the one-kernel selection (k_select_tc.cu)
@@ -63,7 +63,9 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
   };
   // padded by one chunk of columns: the scoring epilogues read 8 at a time
   L.rk = take((H * 2 * n + 256) * sizeof(float));
-  if (!L.fused) {
+  if (L.fused) {
+    L.sel = take(select_tc_workspace((int64_t)T, (int)H));
+  } else {
     L.rq = take(T * H * 2 * sizeof(float));
     L.hv = take((size_t)L.splits * T * H * 2 * k * sizeof(float));
     L.hi = take((size_t)L.splits * T * H * 2 * k * sizeof(int32_t));
@@ -160,7 +162,7 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
   if (L.fused) {
     // a1 (query) + a2 .. a5 in one kernel
     PKM_TRY(launch_select_tc(a->query, a->subkeys, T, H, dh, n, k, rk, a->idx, a->weights,
-                             status, st));
+                             ws + L.sel, status, st));
     mark(a, 2, st);
   } else {
     // a2 + a3: sub-key scores and per-half top-k
