@@ -164,9 +164,117 @@ static bool tc_ok(int64_t M, int N, int K, bool a_mn, bool b_mn) {
   return !a_mn || M % 8 == 0;
 }
 
+// Few rows (decode batches): C[M,N] = epi(A[M,K] W) with W [K][N] held
+// N-contiguous, on the SIMT cores.  A 128-row tensor-core tile would be
+// mostly padding and a handful of CTAs would stream all of W, so here every
+// CTA reads a 32-column strip of W exactly once for up to 8 rows of A: its
+// 8 warps split K; lane l takes 8 columns (one 16-byte vector) of the strip
+// and every 8th k of its warp's range, keeping 8 weight loads in flight, and
+// FMAs each vector into 8 rows x 8 columns of fp32 partials; the 8 lanes
+// sharing columns are summed with shuffles, the 8 warps' sums in warp order
+// through shared memory (a fixed order: the result is reproducible).  A^T
+// [K][8] is staged in shared memory so one 16-byte load gives A[0..7][k].
+constexpr int kSmallM = 8;
+constexpr int kSmallCols = 32;
+constexpr int kSmallMaxK = 1024;  // A^T and the partial sums stay within 48 KiB of static shared memory
+constexpr int kSmallBatch = 8;    // weight loads in flight per thread
+
+__global__ void __launch_bounds__(256) gemm_small_m_kernel(const __nv_bfloat16* __restrict__ A,
+                                                           const __nv_bfloat16* __restrict__ W,
+                                                           int M, int N, int K, int epi,
+                                                           __nv_bfloat16* __restrict__ C) {
+  __shared__ __align__(16) uint16_t at[kSmallMaxK * kSmallM];  // A^T: [k][m] bf16 bits
+  __shared__ float part[8][kSmallM][kSmallCols];               // per-warp sums
+  const int n0 = blockIdx.x * kSmallCols;
+  const int m0 = blockIdx.y * kSmallM;
+  const int mc = min(kSmallM, M - m0);
+  // stage A^T: 16-byte row pieces of A, scattered by k (K % 8 == 0)
+  for (int i = threadIdx.x; i < kSmallM * (K / 8); i += blockDim.x) {
+    const int m = i / (K / 8), kc = i % (K / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (m < mc) v = *reinterpret_cast<const uint4*>(A + (int64_t)(m0 + m) * K + kc * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      at[(kc * 8 + 2 * e) * kSmallM + m] = (uint16_t)(w[e] & 0xffffu);
+      at[(kc * 8 + 2 * e + 1) * kSmallM + m] = (uint16_t)(w[e] >> 16);
+    }
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cv = lane & 3, kq = lane >> 2;  // column vector, k phase
+  const int ncol = n0 + cv * 8;
+  const int kw = (K + 7) / 8;  // k range of a warp
+  const int kb = warp * kw, ke = min(K, kb + kw);
+  float acc[kSmallM][8];
+#pragma unroll
+  for (int m = 0; m < kSmallM; ++m)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[m][c] = 0.f;
+  if (ncol < N) {
+    for (int k0 = kb + kq; k0 < ke; k0 += 8 * kSmallBatch) {
+      uint4 wv[kSmallBatch];
+#pragma unroll
+      for (int u = 0; u < kSmallBatch; ++u) {
+        const int kk = k0 + 8 * u;
+        wv[u] = kk < ke ? ldg_nc_16(W + (int64_t)kk * N + ncol) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kSmallBatch; ++u) {
+        const int kk = k0 + 8 * u;
+        if (kk < ke) {
+          const uint4 av = *reinterpret_cast<const uint4*>(at + kk * kSmallM);
+          float wf[8], af[8];
+          unpack16<PKM_BF16>(wv[u], wf);
+          unpack16<PKM_BF16>(av, af);
+#pragma unroll
+          for (int m = 0; m < kSmallM; ++m)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[m][c] = fmaf(af[m], wf[c], acc[m][c]);
+        }
+      }
+    }
+  }
+  // lanes cv, cv+4, ..., cv+28 hold the same columns: sum them
+#pragma unroll
+  for (int m = 0; m < kSmallM; ++m)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float v = acc[m][c];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      acc[m][c] = v;
+    }
+  if (kq == 0) {
+#pragma unroll
+    for (int m = 0; m < kSmallM; ++m)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) part[warp][m][cv * 8 + c] = acc[m][c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kSmallM * kSmallCols; i += blockDim.x) {
+    const int m = i / kSmallCols, c = i % kSmallCols;
+    if (m >= mc || n0 + c >= N) continue;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += part[w][m][c];
+    if (epi == 1) v = silu_f(v);
+    C[(int64_t)(m0 + m) * N + n0 + c] = __float2bfloat16_rn(v);
+  }
+}
+
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
                              void* C, int32_t* status, cudaStream_t stream, bool b_mn) {
   if (M <= 0) return cudaSuccess;
+  if (b_mn && M <= 64 && K <= kSmallMaxK && K % 8 == 0 && N % 8 == 0) {
+    dim3 grid((unsigned)((N + kSmallCols - 1) / kSmallCols), (unsigned)((M + kSmallM - 1) / kSmallM));
+    gemm_small_m_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(A),
+                                                  static_cast<const __nv_bfloat16*>(B), (int)M, N,
+                                                  K, epi, static_cast<__nv_bfloat16*>(C));
+    note_launch();
+    return cudaGetLastError();
+  }
   if (tc_ok(M, N, K, false, b_mn))
     return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream, 1, 0, false, b_mn);
   return launch_gemm_simt(A, B, M, N, K, epi, 0, C, stream, false, b_mn);

@@ -31,19 +31,17 @@
 //     thr (a lower bound of the row's final k-th best p) and appends the
 //     survivors (p, a) to a 16-entry per-row buffer in shared memory;
 //   * whenever some row of the warp holds more than 8, the warp merges each
-//     row's buffer into the row's sorted list of the k best (keys in
-//     registers, bitonic sort and merge networks) and raises thr to the
-//     list's k-th best;
+//     row's buffer into the row's sorted list of the k best (scores and
+//     positions in registers, bitonic sort and merge networks) and raises
+//     thr to the list's k-th best;
 //   * before the first chunk's filter pass a histogram pass over the same
 //     chunk (still in TMEM) counts the maxima of groups of 4 columns into
 //     score bins of 1/16; the lower edge of the bin where the count from the
 //     top reaches k bounds the chunk's (and so the row's) k-th best score
 //     from below, since group maxima are distinct elements.  That starts the
 //     filter near its final level instead of at -inf.
-// Keys: 64 bits, the order-preserving bits of the fp32 score above the
-// complemented column (equal scores order the smaller column first).
-// Measured: packing the column into the low mantissa bits of an fp64 key
-// and exchanging with fp64 min/max ran 2.5x slower on B200.
+// Candidates are fp32 scores with their positions carried alongside (see
+// "keys" below); exactly equal scores are ties in either order.
 //
 // Combine: each CTA writes its rows' sorted lists to the workspace (they
 // stay in L2), then counts itself in on its (token tile, head) pair with an
@@ -69,11 +67,12 @@ namespace pkm {
 
 namespace sl {
 constexpr int kM = 128;           // tokens per tile (TMEM lanes)
-constexpr int kN = 256;           // sub-key columns per chunk
+constexpr int kN = 128;           // sub-key columns per chunk
 constexpr int kKB = 64;           // k-block width (128 bytes of bf16)
-constexpr int kStages = 2;
+constexpr int kStages = 3;
+constexpr int kAcc = 2;           // TMEM accumulators: the MMA fills one while the epilogue reads the other
 constexpr int kABytes = kM * kKB * 2;   // 16 KiB
-constexpr int kBBytes = kN * kKB * 2;   // 32 KiB
+constexpr int kBBytes = kN * kKB * 2;   // 16 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 192;
 constexpr int kBuf = 16;          // pending candidates per row
@@ -87,16 +86,17 @@ constexpr int kPendBytes = kBuf * kM * 4 + kBuf * kM * 2;   // p (fp32) and colu
 // a row's bins are the words [w][row] of the fp32 part of the pending buffers,
 // which hold only that row's entries: no row's bins overlap another row's data
 static_assert(kBins / 4 <= kBuf, "the histogram aliases the row's own fp32 entries");
-static_assert(kN / kGroup <= 255, "bin counts fit in a byte");
-constexpr int kRkBytes = 4 * kN * 4;                        // each epilogue warp's chunk norms
+static_assert(2 * kN / kGroup <= 255, "bin counts (two chunks) fit in a byte");
+constexpr int kRkBytes = 4 * kAcc * kN * 4;  // each epilogue warp's norms of the chunks in TMEM
 constexpr size_t kSmemBytes =
     (size_t)kStages * kStageBytes + kPendBytes + kRkBytes + 256 /*barriers*/;
 // after the last MMA the stage ring holds the combine's arrays: both halves'
-// lists (scores and positions, [2][32][129]) and the heaps, one column per row
+// lists (scores and positions, [2][32][129]) and each row's candidate buffer
+// (score, row id: [16][128] each), one column per row
 constexpr int kHeapPad = kM + 1;
-static_assert(2 * kMaxK * kHeapPad * 6 + (kMaxK + 2) * kHeapPad * 6 + kMaxK * kHeapPad * 2 <=
-                  kStages * kStageBytes,
-              "both halves' lists and the heaps fit in the stage ring");
+constexpr int kCombOff = (2 * kMaxK * kHeapPad * 6 + 255) / 256 * 256;
+static_assert(kCombOff + kBuf * kM * 8 <= kStages * kStageBytes,
+              "both halves' lists and the candidate buffers fit in the stage ring");
 constexpr int kListKeys = kMaxK * kM;  // keys of one (tile, head, half) list block [32][128]
 }  // namespace sl
 
@@ -104,8 +104,8 @@ struct SelectCtl {
   uint64_t full[sl::kStages];
   uint64_t empty[sl::kStages];
   uint64_t aread[sl::kStages];  // the epilogue has read the query rows of a first-chunk stage
-  uint64_t accf;
-  uint64_t acce;
+  uint64_t accf[sl::kAcc];
+  uint64_t acce[sl::kAcc];
   uint64_t drain;
   uint32_t tmem;
   volatile int abort;
@@ -130,37 +130,27 @@ __device__ __forceinline__ void tmem_wait_x8(uint32_t (&r)[8]) {
 }
 
 // ---------------------------------------------------------------- keys --
+// A candidate is its fp32 score (-inf: empty) and its position or row id
+// (u32), held as two parallel register arrays: the exchange networks compare
+// the scores with fp32 max / min and move the ids with one select each, all
+// 32-bit work (a 64-bit key ordering the id too was measured 3.8x slower per
+// exchange on B200).  Exactly equal scores may come out in either order; the
+// selection rules treat equal scores as ties.
 
-// a row's candidate: the order-preserving bits of the score above the
-// complemented column, so that equal scores order the smaller column first
-using Key = uint64_t;
-__device__ __forceinline__ uint32_t ord_score(float s) {
-  const uint32_t u = __float_as_uint(s);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ Key make_key(float s, int col) {
-  s += 0.0f;  // -0 -> +0: both zeros are one score
-  return ((uint64_t)ord_score(s) << 32) | (uint64_t)(0xffffffffu - (uint32_t)col);
-}
-__device__ __forceinline__ float key_score(Key k) {
-  const uint32_t u = (uint32_t)(k >> 32);
-  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
-}
-__device__ __forceinline__ int key_col(Key k) { return (int)(0xffffffffu - (uint32_t)k); }
-// the empty slot: below every score's key
-__device__ __forceinline__ Key empty_key() { return 0ull; }
-__device__ __forceinline__ Key key_max(Key a, Key b) { return a > b ? a : b; }
-__device__ __forceinline__ Key key_min(Key a, Key b) { return a > b ? b : a; }
+__device__ __forceinline__ float canon(float s) { return s + 0.0f; }  // -0 -> +0
 
-#define SL_CAS(a, b)            \
-  {                             \
-    const Key x_ = (a);         \
-    (a) = key_max(x_, (b));     \
-    (b) = key_min(x_, (b));     \
-  }
+__device__ __forceinline__ void cas_desc(float& a, uint32_t& ai, float& b, uint32_t& bi) {
+  const bool sw = b > a;
+  const float hi = fmaxf(a, b), lo = fminf(a, b);
+  const uint32_t h = sw ? bi : ai, l = sw ? ai : bi;
+  a = hi;
+  b = lo;
+  ai = h;
+  bi = l;
+}
 
-// sort 16 keys descending (bitonic network)
-__device__ __forceinline__ void sort16_desc(Key* v) {
+// sort 16 candidates descending (bitonic network)
+__device__ __forceinline__ void sort16_desc(float* v, uint32_t* c) {
 #pragma unroll
   for (int size = 2; size <= 16; size <<= 1) {
 #pragma unroll
@@ -170,9 +160,9 @@ __device__ __forceinline__ void sort16_desc(Key* v) {
         const int j = i ^ stride;
         if (j > i) {
           if ((i & size) == 0) {
-            SL_CAS(v[i], v[j]);
+            cas_desc(v[i], c[i], v[j], c[j]);
           } else {
-            SL_CAS(v[j], v[i]);
+            cas_desc(v[j], c[j], v[i], c[i]);
           }
         }
       }
@@ -182,17 +172,29 @@ __device__ __forceinline__ void sort16_desc(Key* v) {
 
 // L (sorted desc, 32) <- top 32 of L u B (B sorted desc, 16): the larger of
 // L[i] and B[31-i] for i >= 16 makes L bitonic, five exchange stages sort it
-__device__ __forceinline__ void merge16_desc(Key* L, const Key* B) {
+__device__ __forceinline__ void merge16_desc(float* L, uint32_t* Lc, const float* B,
+                                             const uint32_t* Bc) {
 #pragma unroll
-  for (int i = 16; i < 32; ++i) L[i] = key_max(L[i], B[31 - i]);
+  for (int i = 16; i < 32; ++i) {
+    const bool sw = B[31 - i] > L[i];
+    L[i] = fmaxf(L[i], B[31 - i]);
+    Lc[i] = sw ? Bc[31 - i] : Lc[i];
+  }
 #pragma unroll
   for (int stride = 16; stride > 0; stride >>= 1) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      if ((i & stride) == 0) SL_CAS(L[i], L[i + stride]);
+      if ((i & stride) == 0) cas_desc(L[i], Lc[i], L[i + stride], Lc[i + stride]);
     }
   }
 }
+
+// list entries in the workspace: the score's bits, then the position / id
+__device__ __forceinline__ uint64_t pack_entry(float s, uint32_t c) {
+  return ((uint64_t)c << 32) | (uint64_t)__float_as_uint(s);
+}
+__device__ __forceinline__ float entry_score(uint64_t e) { return __uint_as_float((uint32_t)e); }
+__device__ __forceinline__ uint32_t entry_id(uint64_t e) { return (uint32_t)(e >> 32); }
 
 // thr_raw <- max(thr_raw, a filter level for the raw products): any column
 // whose score s = p * rowf (rounded) is >= thr has p above the returned
@@ -204,21 +206,25 @@ __device__ __forceinline__ void raise_threshold(float& thr_raw, float thr, float
   if (fabsf(t) < INFINITY) thr_raw = fmaxf(thr_raw, t);
 }
 
-// Merge the row's pending candidates (cnt entries of p and column, at a
-// stride of 128) into its sorted list L, empty the buffer and raise the
-// filter level to the list's k-th best.
+// Merge the row's pending candidates (pairs (p, column) at a stride of 128
+// entries, cnt of them) into its sorted list (L, Lc), empty the buffer and
+// raise the filter level to the list's k-th best.
 template <bool K32>
-__device__ __forceinline__ void flush_pending(Key (&L)[32], const float* pp,
-                                              const uint16_t* pc, int& cnt, float& thr_raw,
-                                              int k, float rowf, float inv_rowf) {
-  Key B[sl::kBuf];
+__device__ __forceinline__ void flush_pending(float (&L)[32], uint32_t (&Lc)[32],
+                                              const float* pp, const uint16_t* pc, int& cnt,
+                                              float& thr_raw, int k, float rowf,
+                                              float inv_rowf) {
+  float B[sl::kBuf];
+  uint32_t Bc[sl::kBuf];
 #pragma unroll
-  for (int j = 0; j < sl::kBuf; ++j)
-    B[j] = j < cnt ? make_key(pp[j * sl::kM] * rowf, (int)pc[j * sl::kM]) : empty_key();
-  sort16_desc(B);
-  merge16_desc(L, B);
+  for (int j = 0; j < sl::kBuf; ++j) {
+    B[j] = j < cnt ? canon(pp[j * sl::kM] * rowf) : -INFINITY;
+    Bc[j] = j < cnt ? (uint32_t)pc[j * sl::kM] : 0xffffffffu;
+  }
+  sort16_desc(B, Bc);
+  merge16_desc(L, Lc, B, Bc);
   cnt = 0;
-  Key kth;
+  float kth;
   if constexpr (K32) {
     kth = L[31];
   } else {
@@ -227,97 +233,80 @@ __device__ __forceinline__ void flush_pending(Key (&L)[32], const float* pp,
     for (int i = 1; i < 32; ++i)
       if (i == k - 1) kth = L[i];
   }
-  if (kth != empty_key()) raise_threshold(thr_raw, key_score(kth), inv_rowf);
+  if (kth > -INFINITY) raise_threshold(thr_raw, kth, inv_rowf);
 }
 
-// ------------------------------------------------------------- combine --
-
-__device__ __forceinline__ uint32_t ord_of(float s) {
-  uint32_t u = __float_as_uint(s);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// One thread per (token, head).  s1/a1: the first half's k best (scores,
-// positions; best first), s2/b2 the second half's, at a stride of
-// kHeapPad.  The k x k grid S[i][j] = s1[i] + s2[j] decreases along rows and
-// columns, so its cells can be taken best first with a max-heap frontier:
-// start at (0, 0); taking (i, j) admits (i, j+1) and, on the first column,
-// (i+1, 0).  Equal scores are ordered by the row id a*n+b (smaller first).
-// Writes the k row ids and softmax weights of the row.
+// One thread per (token, head); all kM threads of the group call it (its
+// merges are warp-collective), `live` says whether the row is a token.
+// s1/a1: the first half's k best (scores, positions; best first), s2/b2 the
+// second half's, at a stride of kHeapPad.  In the k x k grid S[i][j] =
+// s1[i] + s2[j] (non-increasing along rows and columns) cell (i, j) is beaten
+// by the (i+1)(j+1) - 1 cells above and left of it, so
+//   tau = max over i of S[i][ceil(k/(i+1)) - 1]
+// is at most the k-th best cell, and only cells with (i+1)(j+1) <= k and
+// S >= tau can be among the k best.  Those candidates go through the same
+// buffer, sort and merge steps as the per-half top-k (the score, carrying
+// the row id a*n+b); ps / pi are the row's buffer (stride kM).
+// Writes the k row ids and softmax weights.
+template <bool K32>
 __device__ void combine_row(const float* s1, const uint16_t* a1, const float* s2,
-                            const uint16_t* b2, uint32_t* hk, uint16_t* hc, uint16_t* rec, int n,
-                            int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+                            const uint16_t* b2, int n, int k, bool live, float* ps, int* pi,
+                            int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
   constexpr int P = sl::kHeapPad;
-  auto id_of = [&](int cell) { return (int32_t)a1[(cell >> 6) * P] * n + (int32_t)b2[(cell & 63) * P]; };
-  auto ahead = [&](uint32_t s, int c, uint32_t t, int d) {
-    return s != t ? s > t : id_of(c) < id_of(d);
-  };
-  auto score_at = [&](int i, int j) { return ord_of(s1[i * P] + s2[j * P]); };
-  int size = 0;
-  auto push = [&](uint32_t key, int cell) {
-    int pos = ++size;
-    while (pos > 1) {
-      const int par = pos >> 1;
-      const uint32_t pk = hk[par * P];
-      const int pcell = hc[par * P];
-      if (!ahead(key, cell, pk, pcell)) break;
-      hk[pos * P] = pk;
-      hc[pos * P] = (uint16_t)pcell;
-      pos = par;
+  float tau = -INFINITY;
+  for (int i = 0; i < k; ++i) tau = fmaxf(tau, s1[i * P] + s2[((k + i) / (i + 1) - 1) * P]);
+  float L[32];
+  uint32_t Lc[32];
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    L[q] = -INFINITY;
+    Lc[q] = 0xffffffffu;
+  }
+  int cnt = 0;
+  auto merge = [&]() {
+    float B[sl::kBuf];
+    uint32_t Bc[sl::kBuf];
+#pragma unroll
+    for (int j = 0; j < sl::kBuf; ++j) {
+      B[j] = j < cnt ? ps[j * sl::kM] : -INFINITY;
+      Bc[j] = j < cnt ? (uint32_t)pi[j * sl::kM] : 0xffffffffu;
     }
-    hk[pos * P] = key;
-    hc[pos * P] = (uint16_t)cell;
+    sort16_desc(B, Bc);
+    merge16_desc(L, Lc, B, Bc);
+    cnt = 0;
   };
-  push(score_at(0, 0), 0);
-  for (int r = 0; r < k; ++r) {
-    const int cell = hc[1 * P];
-    const uint32_t lk = hk[size * P];
-    const int lc = hc[size * P];
-    --size;
-    int pos = 1;
-    while (true) {
-      int ch = pos * 2;
-      if (ch > size) break;
-      uint32_t ck = hk[ch * P];
-      int cc = hc[ch * P];
-      if (ch < size) {
-        const uint32_t k2 = hk[(ch + 1) * P];
-        const int c2 = hc[(ch + 1) * P];
-        if (ahead(k2, c2, ck, cc)) {
-          ck = k2;
-          cc = c2;
-          ++ch;
-        }
+  for (int i = 0; i < k; ++i) {
+    const float si = s1[i * P];
+    if (!__any_sync(0xffffffffu, live && si + s2[0] >= tau)) break;  // later rows are no larger
+    const int ai = (int)a1[i * P] * n;
+    const int m = k / (i + 1);
+    for (int j = 0; j < m; ++j) {
+      const float S = si + s2[j * P];
+      if (live && S >= tau) {
+        ps[cnt * sl::kM] = canon(S);
+        pi[cnt * sl::kM] = ai + (int)b2[j * P];
+        ++cnt;
       }
-      if (!ahead(ck, cc, lk, lc)) break;
-      hk[pos * P] = ck;
-      hc[pos * P] = (uint16_t)cc;
-      pos = ch;
+      if (__any_sync(0xffffffffu, cnt == sl::kBuf)) merge();
     }
-    if (size > 0 || pos > 1) {
-      hk[pos * P] = lk;
-      hc[pos * P] = (uint16_t)lc;
-    }
-    rec[r * P] = (uint16_t)cell;
-    const int i = cell >> 6, j = cell & 63;
-    if (j + 1 < k) push(score_at(i, j + 1), i * 64 + j + 1);
-    if (j == 0 && i + 1 < k) push(score_at(i + 1, 0), (i + 1) * 64);
   }
+  if (__any_sync(0xffffffffu, cnt > 0)) merge();
+  if (!live) return;
   // softmax over the k kept scores; the first is the maximum
-  const int c0 = rec[0];
-  const float m = s1[(c0 >> 6) * P] + s2[(c0 & 63) * P];
+  const float mx = L[0];
   float z = 0.f;
-  for (int r = 0; r < k; ++r) {
-    const int c = rec[r * P];
-    z += expf(s1[(c >> 6) * P] + s2[(c & 63) * P] - m);
-  }
+#pragma unroll
+  for (int r = 0; r < 32; ++r)
+    if (r < k) z += expf(L[r] - mx);
   const float inv = 1.0f / z;
-  for (int r = 0; r < k; ++r) {
-    const int c = rec[r * P];
-    const int i = c >> 6, j = c & 63;
-    idx_out[r] = id_of(c);
-    w_out[r] = expf(s1[i * P] + s2[j * P] - m) * inv;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    if (r < k) {
+      idx_out[r] = (int32_t)Lc[r];
+      w_out[r] = expf(L[r] - mx) * inv;
+    }
   }
+  (void)K32;
 }
 
 // bounded wait that also gives up when another role of the CTA aborted
@@ -380,8 +369,10 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
       mbar_init(&ctl->empty[s], 1);
       mbar_init(&ctl->aread[s], 4);
     }
-    mbar_init(&ctl->accf, 1);
-    mbar_init(&ctl->acce, 4);
+    for (int b = 0; b < kAcc; ++b) {
+      mbar_init(&ctl->accf[b], 1);
+      mbar_init(&ctl->acce[b], 4);
+    }
     mbar_init(&ctl->drain, 1);
     ctl->abort = misaligned ? 1 : 0;
     if (misaligned) set_status(status, PKM_ERR_DEVICE);
@@ -392,7 +383,7 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     prefetch_tmap(&tmB);
   }
   if (warp == 1 && !misaligned) {
-    tmem_alloc(&ctl->tmem, kN);
+    tmem_alloc(&ctl->tmem, kAcc * kN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -442,11 +433,12 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      uint32_t use = 0;
-      for (int c = 0; c < nch && ok; ++c, use ^= 1) {
-        // the accumulator is free once the epilogue has read the last chunk
-        if (!wait_sel(&ctl->acce, use ^ 1, ctl, status)) { ok = false; break; }
+      for (int c = 0; c < nch && ok; ++c) {
+        // accumulator c % 2 is free once the epilogue has read chunk c - 2
+        const int b = c & 1;
+        if (!wait_sel(&ctl->acce[b], ((c >> 1) & 1) ^ 1, ctl, status)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t dt = tmem + (uint32_t)(b * kN);
         for (int kb = 0; kb < KB; ++kb) {
           if (!wait_sel(&ctl->full[stage], phase, ctl, status)) { ok = false; break; }
           tc_fence_after();
@@ -454,12 +446,12 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
           const uint32_t sb = sa + kABytes;
 #pragma unroll
           for (int kk = 0; kk < kKB / 16; ++kk)
-            tc_mma_f16(tmem, smem_desc_k128(sa + kk * 32), smem_desc_k128(sb + kk * 32), idesc,
+            tc_mma_f16(dt, smem_desc_k128(sa + kk * 32), smem_desc_k128(sb + kk * 32), idesc,
                        (kb | kk) != 0);
           tc_commit(&ctl->empty[stage]);  // the stage is free once these MMAs finish
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
-        if (ok) tc_commit(&ctl->accf);
+        if (ok) tc_commit(&ctl->accf[b]);
       }
       // every MMA issued must complete before TMEM is released
       tc_commit(&ctl->drain);
@@ -474,7 +466,7 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     const bool live = t < T;
     float* pp = pend_p + row;   // entry j at pp[128 j]
     uint16_t* pc = pend_c + row;
-    float* rkw = rkbuf + (warp - 2) * kN;  // this warp's copy of the chunk's norms
+    float* rkw = rkbuf + (warp - 2) * kAcc * kN;  // this warp's norms of chunk c at rkw[128 (c & 1)]
     const float* rkc = rk + (int64_t)hc * n;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
@@ -501,60 +493,80 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     const float rowf = sqrtf((float)dh) * rq;
     const float inv_rowf = 1.0f / rowf;
 
-    Key L[32];
+    float L[32];
+    uint32_t Lc[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) L[i] = empty_key();
+    for (int i = 0; i < 32; ++i) {
+      L[i] = -INFINITY;
+      Lc[i] = 0xffffffffu;
+    }
     int cnt = 0;
     // rows past the end of the batch keep nothing
     float thr_raw = live ? -INFINITY : INFINITY;
 
-    // 2. the chunks
-    float4 kn0 = make_float4(0.f, 0.f, 0.f, 0.f), kn1 = kn0;
+    // 2. the chunks; chunk c sits in accumulator c & 1
+    auto stage_norms = [&](int c, float4 v) {
+      reinterpret_cast<float4*>(rkw + (c & 1) * kN)[lane] = v;
+    };
+    auto load_norms = [&](int c) {  // the norm buffer is padded by 256 columns: in bounds
+      return __ldg(reinterpret_cast<const float4*>(rkc + c * kN) + lane);
+    };
+    float4 kn = make_float4(0.f, 0.f, 0.f, 0.f);
     if (ok) {
-      const float4* src = reinterpret_cast<const float4*>(rkc + lane * 8);
-      kn0 = __ldg(src);
-      kn1 = __ldg(src + 1);
+      stage_norms(0, load_norms(0));
+      if (nch > 1) stage_norms(1, load_norms(1));
+      if (nch > 2) kn = load_norms(2);
+      __syncwarp();
     }
     for (int it = 0; it < nch && ok; ++it) {
+      const int b = it & 1;
       const int c0 = it * kN;
       const int ncols = min(kN, n - c0);
-      __syncwarp();  // every lane is done with the previous chunk's norms
-      reinterpret_cast<float4*>(rkw + lane * 8)[0] = kn0;
-      reinterpret_cast<float4*>(rkw + lane * 8)[1] = kn1;
-      __syncwarp();
-      if (it + 1 < nch) {  // the norm buffer is padded by a chunk: in bounds
-        const float4* src = reinterpret_cast<const float4*>(rkc + c0 + kN + lane * 8);
-        kn0 = __ldg(src);
-        kn1 = __ldg(src + 1);
+      if (it >= 2) {
+        __syncwarp();  // every lane is done with chunk it - 2's norms
+        stage_norms(it, kn);
+        __syncwarp();
+        if (it + 1 < nch) kn = load_norms(it + 1);
       }
-      const bool got = wait_sel(&ctl->accf, it & 1, ctl, status);
+      const bool got = wait_sel(&ctl->accf[b], (it >> 1) & 1, ctl, status);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t taddr = tmem + lane_base;
       uint32_t nxt[8], cur[8];
 
       if (it == 0) {
-        // histogram pass: maxima of groups of 4 columns into score bins
+        // histogram pass over the first two chunks (both in TMEM): maxima of
+        // groups of 4 columns into score bins
+        const int nh = min(nch, 2);
+        if (nh == 2) {
+          const bool got1 = wait_sel(&ctl->accf[1], 0, ctl, status);
+          if (!__all_sync(0xffffffffu, got1)) { ok = false; break; }
+          tc_fence_after();
+        }
         uint32_t* hw = reinterpret_cast<uint32_t*>(hist) + row;  // word w at hw[128 w]
 #pragma unroll
         for (int w = 0; w < kBins / 4; ++w) hw[w * kM] = 0u;
         unsigned char* hb = hist + row * 4;  // bin b at hb[512 (b >> 2) + (b & 3)]
         const float c16 = rowf * kBinsPerUnit;
-        tmem_ld_32x32b_x8(taddr, nxt);
+        for (int hcn = 0; hcn < nh; ++hcn) {
+          const uint32_t ta = tmem + lane_base + hcn * kN;
+          const float* rkv = rkw + hcn * kN;
+          const int nc = min(kN, n - hcn * kN);
+          tmem_ld_32x32b_x8(ta, nxt);
 #pragma unroll 1
-        for (int g = 0; g < kN / 8; ++g) {
-          tmem_wait_x8(nxt);
+          for (int g = 0; g < kN / 8; ++g) {
+            tmem_wait_x8(nxt);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
-          if (g + 1 < kN / 8) tmem_ld_32x32b_x8(taddr + (g + 1) * 8, nxt);
-          float p[8];
-          products8(cur, rkw, g, ncols, p);
+            for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
+            if (g + 1 < kN / 8) tmem_ld_32x32b_x8(ta + (g + 1) * 8, nxt);
+            float p[8];
+            products8(cur, rkv, g, nc, p);
 #pragma unroll
-          for (int q = 0; q < 8 / kGroup; ++q) {
-            const float gm = fmaxf(fmaxf(p[4 * q], p[4 * q + 1]), fmaxf(p[4 * q + 2], p[4 * q + 3]));
-            const float tb = fminf(fmaxf(fmaf(gm, c16, kBinOffset), 0.f), (float)(kBins - 1));
-            const int bin = (int)tb;
-            hb[512 * (bin >> 2) + (bin & 3)] += 1;
+            for (int q = 0; q < 8 / kGroup; ++q) {
+              const float gm = fmaxf(fmaxf(p[4 * q], p[4 * q + 1]), fmaxf(p[4 * q + 2], p[4 * q + 3]));
+              const float tb = fminf(fmaxf(fmaf(gm, c16, kBinOffset), 0.f), (float)(kBins - 1));
+              const int bin = (int)tb;
+              hb[512 * (bin >> 2) + (bin & 3)] += 1;
+            }
           }
         }
         // the bound: lower edge of the bin where the count from the top reaches k
@@ -580,6 +592,8 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
 
       // filter pass: products above the level into the row's buffer; one
       // merge site for the whole loop keeps the code (and its misses) small
+      const uint32_t taddr = tmem + lane_base + b * kN;
+      const float* rkv = rkw + b * kN;
       tmem_ld_32x32b_x8(taddr, nxt);
 #pragma unroll 1
       for (int g = 0; g < kN / 8; ++g) {
@@ -588,7 +602,7 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
         for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
         if (g + 1 < kN / 8) tmem_ld_32x32b_x8(taddr + (g + 1) * 8, nxt);
         float p[8];
-        products8(cur, rkw, g, ncols, p);
+        products8(cur, rkv, g, ncols, p);
         const int col0 = c0 + g * 8;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -599,20 +613,20 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
           }
         }
         if (__any_sync(0xffffffffu, cnt > kFlushAt))
-          flush_pending<K32>(L, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
+          flush_pending<K32>(L, Lc, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->acce);
+      if (lane == 0) mbar_arrive(&ctl->acce[b]);
     }
     if (ok) {
       if (__any_sync(0xffffffffu, cnt > 0))
-        flush_pending<K32>(L, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
+        flush_pending<K32>(L, Lc, pp, pc, cnt, thr_raw, k, rowf, inv_rowf);
       // the sorted list into this (tile, head, half)'s block [32][128] of the workspace
       uint64_t* list = lists + ((int64_t)blockIdx.x * gridDim.y + hc) * kListKeys;
 #pragma unroll
       for (int i = 0; i < 32; ++i)
-        if (i < k) list[i * kM + row] = L[i];
+        if (i < k) list[i * kM + row] = pack_entry(L[i], Lc[i]);
       __threadfence();  // the list is visible device-wide before the pair count below
     }
   }
@@ -621,7 +635,7 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
   __syncthreads();
   if (warp == 1 && run) {
     tc_fence_after();
-    tmem_dealloc(tmem, kN);
+    tmem_dealloc(tmem, kAcc * kN);
   }
 
   // -------------------------------------------------------- k x k combine
@@ -644,28 +658,25 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     constexpr int P = kHeapPad;
     float* sv = reinterpret_cast<float*>(stages);                    // [2][32][P] scores
     uint16_t* cv = reinterpret_cast<uint16_t*>(sv + 2 * kMaxK * P);  // [2][32][P] positions
-    uint32_t* hk = reinterpret_cast<uint32_t*>(cv + 2 * kMaxK * P);  // heap keys [k+2][P]
-    uint16_t* hcell = reinterpret_cast<uint16_t*>(hk + (kMaxK + 2) * P);  // heap cells [k+2][P]
-    uint16_t* rec = hcell + (kMaxK + 2) * P;                         // taken cells [k][P]
+    float* cps = reinterpret_cast<float*>(stages + kCombOff);        // candidates [16][128]
+    int* cpi = reinterpret_cast<int*>(cps + kBuf * kM);
     const uint64_t* pl = lists + ((int64_t)blockIdx.x * gridDim.y + 2 * h) * kListKeys;
     // both halves' lists of the tile's rows (L2): half c's entry j of row r at sv[c][j][r]
     for (int e = threadIdx.x; e < 2 * k * kM; e += kThreads) {
       const int half = e / (k * kM);
       const int j = (e / kM) % k;
       const int r = e % kM;
-      const Key key = ld_cg_u64(pl + (int64_t)half * kListKeys + j * kM + r);
-      sv[(half * kMaxK + j) * P + r] = key_score(key);
-      cv[(half * kMaxK + j) * P + r] = (uint16_t)key_col(key);
+      const uint64_t ent = ld_cg_u64(pl + (int64_t)half * kListKeys + j * kM + r);
+      sv[(half * kMaxK + j) * P + r] = entry_score(ent);
+      cv[(half * kMaxK + j) * P + r] = (uint16_t)entry_id(ent);
     }
     __syncthreads();
     if (threadIdx.x < kM) {
       const int r = threadIdx.x;
       const int64_t t = m0 + r;
-      if (t < T) {
-        const int64_t o = (t * H + h) * k;
-        combine_row(sv + r, cv + r, sv + kMaxK * P + r, cv + kMaxK * P + r, hk + r, hcell + r,
-                    rec + r, n, k, idx + o, wout + o);
-      }
+      const int64_t o = (t * H + h) * k;
+      combine_row<K32>(sv + r, cv + r, sv + kMaxK * P + r, cv + kMaxK * P + r, n, k, t < T,
+                       cps + r, cpi + r, idx + o, wout + o);
     }
   }
 }

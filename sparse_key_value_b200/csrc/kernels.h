@@ -46,6 +46,15 @@ cudaError_t launch_score_topk_tc(const void* q, const void* K, int64_t T, int H,
                                  int k, int splits, const float* rq, const float* rk, float* hv,
                                  int32_t* hi, int32_t* status, cudaStream_t stream);
 
+// Per-half top-k lists for batches of at most 32 tokens (k_score_small.cu):
+// one CTA per (head, half, 256-column chunk), lists hv/hi
+// [chunks][T, H, 2, k] merged by the combine step (splits = chunks).
+bool score_small_supported(pkm_dtype dt, int64_t T, int dh, int n, int k);
+int score_small_chunks(int n);
+cudaError_t launch_score_topk_small(const void* q, const void* K, int64_t T, int H, int dh,
+                                    int n, int k, const float* rq, const float* rk, float* hv,
+                                    int32_t* hi, int32_t* status, cudaStream_t stream);
+
 // The whole selection in one kernel (k_select_tc.cu): query norms, scores
 // on the tensor cores, per-half top-k, k x k combine, top-k and softmax ->
 // idx [T,H,k], w [T,H,k].  bf16, d_half % 64 == 0, 256 <= n < 65536,

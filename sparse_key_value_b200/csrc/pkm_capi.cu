@@ -41,6 +41,7 @@ struct FwdLayout {
   int splits;
   bool tc;
   bool fused;  // the one-kernel selection (k_select_tc.cu)
+  bool small;  // decode-sized batches: per-chunk lists (k_score_small.cu)
 };
 
 static bool has_memplus(const pkm_fwd_args* a) { return a->x || a->W1 || a->W2; }
@@ -53,8 +54,10 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
   // split the sub-key columns over CTAs (score_topk_tc) and combine apart
   L.fused = select_tc_supported(a->dtype, a->d_half, a->n_sub, a->k) &&
             a->T > kSplitGatherMaxBags;
-  L.tc = !L.fused && score_tc_supported(a->dtype, a->d_half, a->n_sub, a->k);
-  L.splits = L.tc ? score_tc_splits(a->T, a->H, a->n_sub) : 1;
+  L.small = !L.fused && score_small_supported(a->dtype, a->T, a->d_half, a->n_sub, a->k);
+  L.tc = !L.fused && !L.small && score_tc_supported(a->dtype, a->d_half, a->n_sub, a->k);
+  L.splits = L.small ? score_small_chunks(a->n_sub)
+                     : (L.tc ? score_tc_splits(a->T, a->H, a->n_sub) : 1);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -166,7 +169,10 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
     mark(a, 2, st);
   } else {
     // a2 + a3: sub-key scores and per-half top-k
-    if (L.tc)
+    if (L.small)
+      PKM_TRY(launch_score_topk_small(a->query, a->subkeys, T, H, dh, n, k, rq, rk, hv, hi,
+                                      status, st));
+    else if (L.tc)
       PKM_TRY(launch_score_topk_tc(a->query, a->subkeys, T, H, dh, n, k, L.splits, rq, rk, hv,
                                    hi, status, st));
     else

@@ -108,6 +108,27 @@ def test_forward_fused_selection(case):
     run_forward(w)
 
 
+# Batches of at most 32 tokens (decode steps) score each 256-column chunk of
+# a (head, half) in its own CTA and sort the chunk's scores per token across a
+# warp; 33..64 tokens keep the column-split kernel with per-thread top-k.
+SMALL_T = [
+    # name, T, H, d_half, n_sub, k, d_v
+    ("small-t8", 8, 4, 64, 1024, 32, 64),
+    ("small-t32-ragged-chunk", 32, 2, 128, 300, 16, 32),
+    ("small-t1-k1", 1, 1, 64, 256, 1, 16),
+    ("small-t5-k7", 5, 3, 192, 700, 7, 24),
+    ("split-t40", 40, 2, 64, 512, 32, 32),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_T, ids=[c[0] for c in SMALL_T])
+def test_forward_small_batches(case):
+    name, T, H, dh, n, k, dv = case
+    w = WORKLOADS["pkm"].scaled(name=name, T=T, H=H, d_half=dh, n_sub=n, k=k, d_v=dv,
+                                dtype="bf16", seed=sum(map(ord, name)))
+    run_forward(w)
+
+
 def test_forward_fused_launches():
     """A batch on the one-kernel selection launches three kernels in all:
     the sub-key norms, the selection and the bag gather."""
@@ -168,6 +189,9 @@ MEMPLUS = [
     (200, 2, 64, 64, 8, 256, 128),     # output projection N < tile
     (300, 1, 128, 256, 16, 512, 320),  # ragged N, tensor-core scoring
     (50, 2, 64, 16, 4, 80, 40),        # K below one k-block: SIMT GEMM
+    (8, 4, 128, 256, 32, 1024, 1024),  # decode-sized: the few-row GEMM
+    (64, 1, 64, 256, 8, 264, 136),     # few-row GEMM, ragged column strips
+    (65, 1, 64, 256, 8, 264, 136),     # just past the few-row GEMM: tensor cores
 ]
 
 
