@@ -24,7 +24,10 @@
  *  - weights: softmax over the k selected full scores.
  *  - heads: each head h has its own sub-key tables; all heads share one
  *    value table; the H bags of a token are summed into one output row.
- *  - order: larger score first; equal scores -> smaller id first.
+ *  - order: larger score first.  Scores that are exactly equal in fp32 are
+ *    ties: the bf16 tensor-core selections (d_half % 64 == 0, k <= 32) may
+ *    keep either and list them in either order; the other paths put the
+ *    smaller id first.
  *
  * Conventions for every entry point:
  *  - Device pointers are caller-owned, row-major, contiguous and 16-byte
@@ -110,9 +113,10 @@ typedef struct {
        [3] after combine + softmax, [4] before the bag gather (after the
        Memory+ gate GEMM), [5] after the bag gather, [6] end (after the
        Memory+ output GEMM).  When the selection runs as one kernel (bf16,
-       d_half % 64 == 0, 256 <= n_sub < 65536, n_sub % 4 == 0, k <= 32,
-       T > 64), [1] follows the sub-key norms only and [2] = [3] follow the
-       whole selection.  Under stream capture the events are recorded as
+       d_half % 64 == 0, 256 <= n_sub < 65536, n_sub % 4 == 0, k <= 32, and
+       T > 64, or T <= 32 with n_sub <= 8192), [2] = [3] follow the whole
+       selection and [1] follows the sub-key norms (T > 64) or equals [0]
+       (T <= 32: the kernel computes them too).  Under stream capture the events are recorded as
        external event nodes of the graph, so every replay records them. */
     void **phase_events;
     /* Optional, Memory+ only: NULL, or [T, d_v] (dtype) receiving the bag

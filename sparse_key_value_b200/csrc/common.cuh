@@ -108,6 +108,16 @@ __device__ __forceinline__ bool better(float s1, int32_t i1, float s2, int32_t i
 
 // ----------------------------------------------------------- mbarriers --
 
+// Programmatic dependent launch.  A kernel launched with programmatic
+// stream serialization may start before the kernel ahead of it in the stream
+// has finished; pdl_wait() blocks until that kernel has completed and its
+// memory is visible (a no-op when the launch was an ordinary one), and
+// pdl_launch_dependents() lets the next such kernel start early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(256) embbag_part_kernel(
   const int nr = min(kGroupRows, B - j0);
   __shared__ int32_t s_idx[kGroupRows];
   __shared__ float s_w[kGroupRows];
+  pdl_launch_dependents();
+  pdl_wait();  // idx and w come from the selection
   if (threadIdx.x < nr) {
     int32_t r = idx[bag * B + j0 + threadIdx.x];
     if (r < 0 || r >= n_rows) {
@@ -76,6 +78,8 @@ __global__ void __launch_bounds__(256) embbag_reduce_kernel(
   constexpr int V = Elem<DT>::kVec;
   const int64_t bag = blockIdx.x;
   const int chunks = d / V;
+  pdl_launch_dependents();
+  pdl_wait();  // the partial sums come from the previous kernel
   for (int ch = threadIdx.x; ch < chunks; ch += blockDim.x) {
     float acc[V];
 #pragma unroll
@@ -109,33 +113,38 @@ size_t embbag_split_workspace(int64_t n_bags, int B, int d) {
 template <pkm_dtype DT>
 static cudaError_t launch_split_t(const void* table, int64_t n_rows, int d, const int32_t* idx,
                                   const float* w, int64_t n_bags, int B, const void* gate,
-                                  void* out, float* part, int32_t* status, cudaStream_t stream) {
+                                  void* out, float* part, int32_t* status, cudaStream_t stream,
+                                  bool pdl) {
   using T = typename Elem<DT>::T;
   const int groups = (B + kGroupRows - 1) / kGroupRows;
   const int chunks = d / Elem<DT>::kVec;
   const int threads = min(256, (chunks + 31) / 32 * 32);
-  embbag_part_kernel<DT><<<dim3((unsigned)n_bags, (unsigned)groups), threads, 0, stream>>>(
-      (const T*)table, n_rows, d, idx, w, B, part, status);
+  cudaError_t e = launch_maybe_pdl(pdl, embbag_part_kernel<DT>,
+                                   dim3((unsigned)n_bags, (unsigned)groups), dim3(threads), 0,
+                                   stream, (const T*)table, n_rows, d, idx, w, B, part, status);
+  if (e != cudaSuccess) return e;
   if (gate)
-    embbag_reduce_kernel<DT, true><<<(unsigned)n_bags, threads, 0, stream>>>(
-        part, groups, d, (const T*)gate, (T*)out);
+    e = launch_maybe_pdl(pdl, embbag_reduce_kernel<DT, true>, dim3((unsigned)n_bags),
+                         dim3(threads), 0, stream, (const float*)part, groups, d, (const T*)gate,
+                         (T*)out);
   else
-    embbag_reduce_kernel<DT, false><<<(unsigned)n_bags, threads, 0, stream>>>(
-        part, groups, d, nullptr, (T*)out);
+    e = launch_maybe_pdl(pdl, embbag_reduce_kernel<DT, false>, dim3((unsigned)n_bags),
+                         dim3(threads), 0, stream, (const float*)part, groups, d, (const T*)nullptr,
+                         (T*)out);
   note_launch(2);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_embbag_fwd_split(const void* table, int64_t n_rows, int d, pkm_dtype dt,
                                     const int32_t* idx, const float* w, int64_t n_bags, int B,
                                     const void* gate, void* out, float* part, int32_t* status,
-                                    cudaStream_t stream) {
+                                    cudaStream_t stream, bool pdl) {
   if (n_bags <= 0) return cudaSuccess;
   if (n_bags > 65535) return cudaErrorInvalidValue;
   return dt == PKM_BF16 ? launch_split_t<PKM_BF16>(table, n_rows, d, idx, w, n_bags, B, gate,
-                                                   out, part, status, stream)
+                                                   out, part, status, stream, pdl)
                         : launch_split_t<PKM_F32>(table, n_rows, d, idx, w, n_bags, B, gate,
-                                                  out, part, status, stream);
+                                                  out, part, status, stream, pdl);
 }
 
 }  // namespace pkm

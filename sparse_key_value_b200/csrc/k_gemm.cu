@@ -179,15 +179,22 @@ constexpr int kSmallCols = 32;
 constexpr int kSmallMaxK = 1024;  // A^T and the partial sums stay within 48 KiB of static shared memory
 constexpr int kSmallBatch = 8;    // weight loads in flight per thread
 
+// pdl_mode (programmatic dependent launch): 1 -- A is the previous kernel's
+// output, wait for it first; 2 -- the inputs do not depend on the previous
+// kernel, wait for it only before finishing (so that this kernel's completion
+// still implies that one's); 0 -- ordinary launch.
 __global__ void __launch_bounds__(256) gemm_small_m_kernel(const __nv_bfloat16* __restrict__ A,
                                                            const __nv_bfloat16* __restrict__ W,
                                                            int M, int N, int K, int epi,
-                                                           __nv_bfloat16* __restrict__ C) {
+                                                           __nv_bfloat16* __restrict__ C,
+                                                           int pdl_mode) {
   __shared__ __align__(16) uint16_t at[kSmallMaxK * kSmallM];  // A^T: [k][m] bf16 bits
   __shared__ float part[8][kSmallM][kSmallCols];               // per-warp sums
   const int n0 = blockIdx.x * kSmallCols;
   const int m0 = blockIdx.y * kSmallM;
   const int mc = min(kSmallM, M - m0);
+  pdl_launch_dependents();
+  if (pdl_mode == 1) pdl_wait();
   // stage A^T: 16-byte row pieces of A, scattered by k (K % 8 == 0)
   for (int i = threadIdx.x; i < kSmallM * (K / 8); i += blockDim.x) {
     const int m = i / (K / 8), kc = i % (K / 8);
@@ -262,18 +269,21 @@ __global__ void __launch_bounds__(256) gemm_small_m_kernel(const __nv_bfloat16* 
     if (epi == 1) v = silu_f(v);
     C[(int64_t)(m0 + m) * N + n0 + c] = __float2bfloat16_rn(v);
   }
+  if (pdl_mode == 2) pdl_wait();
 }
 
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                             void* C, int32_t* status, cudaStream_t stream, bool b_mn) {
+                             void* C, int32_t* status, cudaStream_t stream, bool b_mn,
+                             int pdl_mode) {
   if (M <= 0) return cudaSuccess;
   if (b_mn && M <= 64 && K <= kSmallMaxK && K % 8 == 0 && N % 8 == 0) {
     dim3 grid((unsigned)((N + kSmallCols - 1) / kSmallCols), (unsigned)((M + kSmallM - 1) / kSmallM));
-    gemm_small_m_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(A),
-                                                  static_cast<const __nv_bfloat16*>(B), (int)M, N,
-                                                  K, epi, static_cast<__nv_bfloat16*>(C));
+    const cudaError_t e = launch_maybe_pdl(
+        pdl_mode != 0, gemm_small_m_kernel, grid, dim3(256), 0, stream,
+        static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), (int)M, N, K,
+        epi, static_cast<__nv_bfloat16*>(C), pdl_mode);
     note_launch();
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
   if (tc_ok(M, N, K, false, b_mn))
     return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream, 1, 0, false, b_mn);

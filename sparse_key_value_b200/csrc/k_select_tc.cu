@@ -11,20 +11,16 @@
 //
 // Grid: (token tiles of 128) x (2H), one CTA per (token tile, head, half).
 // Each CTA scores its 128 tokens against all n sub-keys of its (head, half),
-// 256 columns per chunk:
+// 128 columns per chunk:
 //   warp 0     TMA producer: per chunk and 64-wide k-block the query tile
-//              [128 x 64] and the sub-key tile [256 x 64] (bf16, 128-byte
-//              swizzle) into a 2-stage ring.
+//              [128 x 64] and the sub-key tile [128 x 64] (bf16, 128-byte
+//              swizzle) into a 3-stage ring.
 //   warp 1     TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128,
-//              N=256, K=16, fp32 accumulator in 256 TMEM columns.
+//              N=128, K=16, fp32 accumulators in two sets of 128 TMEM
+//              columns: chunk c goes to set c % 2, so the MMAs of the next
+//              chunk run while the epilogue reads this one.
 //   warps 2-5  epilogue, one thread per token row (TMEM lane).
-// Two CTAs share an SM, so the MMAs of one overlap the epilogue of the other.
-//
-// Query norms: while the first chunk's k-blocks pass through shared memory,
-// every epilogue thread sums the squares of its row of the query tile (the
-// swizzle only permutes 16-byte pieces within a row, so the sum needs no
-// unswizzling); the producer refills such a stage only after the epilogue
-// has read it.  So the query is read from memory once, by the TMA.
+// Two CTAs share an SM (112 KiB of shared memory each).
 //
 // Per-row top-k over the scores s = sqrt(d_half) * rq * rk[a] * acc:
 //   * the epilogue filters raw products p = acc * rk[a] against a threshold
@@ -46,10 +42,9 @@
 // Combine: each CTA writes its rows' sorted lists to the workspace (they
 // stay in L2), then counts itself in on its (token tile, head) pair with an
 // atomic after a fence; the second CTA of the pair to arrive reads both
-// halves' lists back and, one thread per token, runs the max-heap frontier
-// over the k x k grid S[i][j] = s1[i] + s2[j] (rows and columns
-// non-increasing), keeps k cells, forms the row ids a*n+b and the softmax
-// weights and writes them.  The first CTA of the pair just exits.  (A 2-CTA
+// halves' lists back and, one warp per token, takes the top k of the cells
+// of the k x k grid S[i][j] = s1[i] + s2[j] that can reach it, forms the row
+// ids a*n+b and the softmax weights and writes them.  The first CTA of the pair just exits.  (A 2-CTA
 // cluster exchanging the lists through distributed shared memory was
 // measured first: cluster launch held this kernel to one CTA per SM.)
 //
@@ -62,6 +57,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tmap.h"
+#include "warp_sort32.cuh"
 
 namespace pkm {
 
@@ -91,12 +87,13 @@ constexpr int kRkBytes = 4 * kAcc * kN * 4;  // each epilogue warp's norms of th
 constexpr size_t kSmemBytes =
     (size_t)kStages * kStageBytes + kPendBytes + kRkBytes + 256 /*barriers*/;
 // after the last MMA the stage ring holds the combine's arrays: both halves'
-// lists (scores and positions, [2][32][129]) and each row's candidate buffer
-// (score, row id: [16][128] each), one column per row
+// lists (scores and positions, [2][32][129], one column per row) and the
+// table of the k x k cells that can reach the top k
 constexpr int kHeapPad = kM + 1;
+constexpr int kCellSlots = 128;   // >= the cells (i+1)(j+1) <= 32 (119)
 constexpr int kCombOff = (2 * kMaxK * kHeapPad * 6 + 255) / 256 * 256;
-static_assert(kCombOff + kBuf * kM * 8 <= kStages * kStageBytes,
-              "both halves' lists and the candidate buffers fit in the stage ring");
+static_assert(kCombOff + kCellSlots * 2 <= kStages * kStageBytes,
+              "both halves' lists and the cell table fit in the stage ring");
 constexpr int kListKeys = kMaxK * kM;  // keys of one (tile, head, half) list block [32][128]
 }  // namespace sl
 
@@ -217,9 +214,11 @@ __device__ __forceinline__ void flush_pending(float (&L)[32], uint32_t (&Lc)[32]
   float B[sl::kBuf];
   uint32_t Bc[sl::kBuf];
 #pragma unroll
-  for (int j = 0; j < sl::kBuf; ++j) {
-    B[j] = j < cnt ? canon(pp[j * sl::kM] * rowf) : -INFINITY;
-    Bc[j] = j < cnt ? (uint32_t)pc[j * sl::kM] : 0xffffffffu;
+  for (int j = 0; j < sl::kBuf; ++j) {  // all kBuf slots are read, those past cnt dropped
+    const float pv = pp[j * sl::kM];
+    const uint32_t pcv = pc[j * sl::kM];
+    B[j] = j < cnt ? canon(pv * rowf) : -INFINITY;
+    Bc[j] = j < cnt ? pcv : 0xffffffffu;
   }
   sort16_desc(B, Bc);
   merge16_desc(L, Lc, B, Bc);
@@ -234,79 +233,6 @@ __device__ __forceinline__ void flush_pending(float (&L)[32], uint32_t (&Lc)[32]
       if (i == k - 1) kth = L[i];
   }
   if (kth > -INFINITY) raise_threshold(thr_raw, kth, inv_rowf);
-}
-
-// One thread per (token, head); all kM threads of the group call it (its
-// merges are warp-collective), `live` says whether the row is a token.
-// s1/a1: the first half's k best (scores, positions; best first), s2/b2 the
-// second half's, at a stride of kHeapPad.  In the k x k grid S[i][j] =
-// s1[i] + s2[j] (non-increasing along rows and columns) cell (i, j) is beaten
-// by the (i+1)(j+1) - 1 cells above and left of it, so
-//   tau = max over i of S[i][ceil(k/(i+1)) - 1]
-// is at most the k-th best cell, and only cells with (i+1)(j+1) <= k and
-// S >= tau can be among the k best.  Those candidates go through the same
-// buffer, sort and merge steps as the per-half top-k (the score, carrying
-// the row id a*n+b); ps / pi are the row's buffer (stride kM).
-// Writes the k row ids and softmax weights.
-template <bool K32>
-__device__ void combine_row(const float* s1, const uint16_t* a1, const float* s2,
-                            const uint16_t* b2, int n, int k, bool live, float* ps, int* pi,
-                            int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
-  constexpr int P = sl::kHeapPad;
-  float tau = -INFINITY;
-  for (int i = 0; i < k; ++i) tau = fmaxf(tau, s1[i * P] + s2[((k + i) / (i + 1) - 1) * P]);
-  float L[32];
-  uint32_t Lc[32];
-#pragma unroll
-  for (int q = 0; q < 32; ++q) {
-    L[q] = -INFINITY;
-    Lc[q] = 0xffffffffu;
-  }
-  int cnt = 0;
-  auto merge = [&]() {
-    float B[sl::kBuf];
-    uint32_t Bc[sl::kBuf];
-#pragma unroll
-    for (int j = 0; j < sl::kBuf; ++j) {
-      B[j] = j < cnt ? ps[j * sl::kM] : -INFINITY;
-      Bc[j] = j < cnt ? (uint32_t)pi[j * sl::kM] : 0xffffffffu;
-    }
-    sort16_desc(B, Bc);
-    merge16_desc(L, Lc, B, Bc);
-    cnt = 0;
-  };
-  for (int i = 0; i < k; ++i) {
-    const float si = s1[i * P];
-    if (!__any_sync(0xffffffffu, live && si + s2[0] >= tau)) break;  // later rows are no larger
-    const int ai = (int)a1[i * P] * n;
-    const int m = k / (i + 1);
-    for (int j = 0; j < m; ++j) {
-      const float S = si + s2[j * P];
-      if (live && S >= tau) {
-        ps[cnt * sl::kM] = canon(S);
-        pi[cnt * sl::kM] = ai + (int)b2[j * P];
-        ++cnt;
-      }
-      if (__any_sync(0xffffffffu, cnt == sl::kBuf)) merge();
-    }
-  }
-  if (__any_sync(0xffffffffu, cnt > 0)) merge();
-  if (!live) return;
-  // softmax over the k kept scores; the first is the maximum
-  const float mx = L[0];
-  float z = 0.f;
-#pragma unroll
-  for (int r = 0; r < 32; ++r)
-    if (r < k) z += expf(L[r] - mx);
-  const float inv = 1.0f / z;
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    if (r < k) {
-      idx_out[r] = (int32_t)Lc[r];
-      w_out[r] = expf(L[r] - mx) * inv;
-    }
-  }
-  (void)K32;
 }
 
 // bounded wait that also gives up when another role of the CTA aborted
@@ -472,24 +398,25 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     bool ok = true;
 
     // 1. the row's query norm from the first chunk's stages
-    float ss = 0.f;
+    float ss[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums: short FMA chains
     for (int kb = 0; kb < KB; ++kb) {
       const int stage = kb % kStages;
       const bool got = wait_sel(&ctl->full[stage], (kb / kStages) & 1, ctl, status);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      // piece u ^ (row & 7) at step u: neighbouring rows on different banks
       const uint4* arow = reinterpret_cast<const uint4*>(stages + stage * kStageBytes + row * 128);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const uint4 v = arow[u];
+        const uint4 v = arow[u ^ (row & 7)];
         float f[8];
         unpack16<PKM_BF16>(v, f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+        for (int e = 0; e < 8; ++e) ss[e & 3] = fmaf(f[e], f[e], ss[e & 3]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->aread[stage]);
     }
-    const float rq = 1.0f / fmaxf(sqrtf(ss), kNormEps);
+    const float rq = 1.0f / fmaxf(sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3])), kNormEps);
     const float rowf = sqrtf((float)dh) * rq;
     const float inv_rowf = 1.0f / rowf;
 
@@ -604,6 +531,9 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
         float p[8];
         products8(cur, rkv, g, ncols, p);
         const int col0 = c0 + g * 8;
+        // predicated appends (unconditional stores at the next free slot
+        // measured slower: the extra shared-memory writes compete with the
+        // MMAs' operand reads)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (p[j] > thr_raw) {
@@ -658,9 +588,10 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
     constexpr int P = kHeapPad;
     float* sv = reinterpret_cast<float*>(stages);                    // [2][32][P] scores
     uint16_t* cv = reinterpret_cast<uint16_t*>(sv + 2 * kMaxK * P);  // [2][32][P] positions
-    float* cps = reinterpret_cast<float*>(stages + kCombOff);        // candidates [16][128]
-    int* cpi = reinterpret_cast<int*>(cps + kBuf * kM);
+    uint16_t* cells = reinterpret_cast<uint16_t*>(stages + kCombOff);  // [128]
     const uint64_t* pl = lists + ((int64_t)blockIdx.x * gridDim.y + 2 * h) * kListKeys;
+    // the cells (i, j) with (i+1)(j+1) <= k, row-major
+    if (threadIdx.x < kCellSlots) cells[threadIdx.x] = topk_cell(threadIdx.x, k);
     // both halves' lists of the tile's rows (L2): half c's entry j of row r at sv[c][j][r]
     for (int e = threadIdx.x; e < 2 * k * kM; e += kThreads) {
       const int half = e / (k * kM);
@@ -671,12 +602,14 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
       cv[(half * kMaxK + j) * P + r] = (uint16_t)entry_id(ent);
     }
     __syncthreads();
-    if (threadIdx.x < kM) {
-      const int r = threadIdx.x;
-      const int64_t t = m0 + r;
-      const int64_t o = (t * H + h) * k;
-      combine_row<K32>(sv + r, cv + r, sv + kMaxK * P + r, cv + kMaxK * P + r, n, k, t < T,
-                       cps + r, cpi + r, idx + o, wout + o);
+    const int rows = T - m0 < kM ? (int)(T - m0) : kM;
+    for (int r = warp; r < rows; r += kThreads / 32) {
+      const int64_t o = ((m0 + r) * H + h) * k;
+      const bool in = lane < k;
+      const int e = lane * P + r;
+      combine_lists_warp(in ? sv[e] : -INFINITY, in ? cv[e] : 0u,
+                         in ? sv[kMaxK * P + e] : -INFINITY, in ? cv[kMaxK * P + e] : 0u, cells,
+                         n, k, idx + o, wout + o);
     }
   }
 }

@@ -12,6 +12,25 @@ namespace pkm {
 // Host-side count of kernels this library has launched (instrumentation).
 void note_launch(int n = 1);
 
+// Launch `kern` with programmatic stream serialization (it may start while
+// the previous kernel of the stream still runs; it calls pdl_wait() before
+// touching that kernel's results) when `pdl`, as an ordinary launch otherwise.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_maybe_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                             size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Device address of the current device's sticky status word.
 int32_t* status_ptr();
 
@@ -46,14 +65,17 @@ cudaError_t launch_score_topk_tc(const void* q, const void* K, int64_t T, int H,
                                  int k, int splits, const float* rq, const float* rk, float* hv,
                                  int32_t* hi, int32_t* status, cudaStream_t stream);
 
-// Per-half top-k lists for batches of at most 32 tokens (k_score_small.cu):
-// one CTA per (head, half, 256-column chunk), lists hv/hi
-// [chunks][T, H, 2, k] merged by the combine step (splits = chunks).
-bool score_small_supported(pkm_dtype dt, int64_t T, int dh, int n, int k);
-int score_small_chunks(int n);
-cudaError_t launch_score_topk_small(const void* q, const void* K, int64_t T, int H, int dh,
-                                    int n, int k, const float* rq, const float* rk, float* hv,
-                                    int32_t* hi, int32_t* status, cudaStream_t stream);
+// The whole selection in one kernel for batches of at most 32 tokens
+// (k_select_small.cu): sub-key and query norms, scores on the tensor cores,
+// per-chunk and per-half top-k, k x k combine, top-k and softmax ->
+// idx [T,H,k], w [T,H,k].  bf16, d_half % 64 == 0, 256 <= n, n % 4 == 0,
+// at most 32 chunks of 256 columns, k <= 32.  `workspace` holds
+// select_small_workspace(T, H, n) bytes (lists and counters).
+bool select_small_supported(pkm_dtype dt, int64_t T, int dh, int n, int k);
+size_t select_small_workspace(int64_t T, int H, int n);
+cudaError_t launch_select_small(const void* q, const void* K, int64_t T, int H, int dh, int n,
+                                int k, int32_t* idx, float* w, void* workspace, int32_t* status,
+                                cudaStream_t stream);
 
 // The whole selection in one kernel (k_select_tc.cu): query norms, scores
 // on the tensor cores, per-half top-k, k x k combine, top-k and softmax ->
@@ -88,12 +110,14 @@ cudaError_t launch_embbag_range(const void* table, int64_t row_lo, int64_t n_loc
                                 pkm_dtype dt, const int32_t* idx, const float* w, int64_t n_bags,
                                 int B, float* out, cudaStream_t stream);
 
+// pdl: both kernels by programmatic dependent launch (each waits for the
+// previous kernel's results before reading idx / w / the partial sums).
 constexpr int64_t kSplitGatherMaxBags = 64;
 size_t embbag_split_workspace(int64_t n_bags, int B, int d);
 cudaError_t launch_embbag_fwd_split(const void* table, int64_t n_rows, int d, pkm_dtype dt,
                                     const int32_t* idx, const float* w, int64_t n_bags, int B,
                                     const void* gate, void* out, float* part, int32_t* status,
-                                    cudaStream_t stream);
+                                    cudaStream_t stream, bool pdl = false);
 
 // Memory+ helpers (bf16).
 // z = y ⊙ g elementwise (bf16, one rounding)
@@ -104,9 +128,13 @@ cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst
                                   cudaStream_t stream, int ld = 0);
 // C[M,N] = epi(A[M,K] * B[N,K]^T) in bf16; epi: 0 none, 1 silu.  A is
 // [M][K]; B is [N][K], or [K][N] with b_mn (a weight [d_in, d_out] used as x W).
+// pdl_mode (few-row batches only; ignored otherwise): 0 ordinary launch;
+// programmatic dependent launch with 1 -- A comes from the previous kernel,
+// 2 -- A and B do not (the kernel overlaps the previous one).
 bool gemm_tc_supported(int64_t M, int N, int K);
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
-                             void* C, int32_t* status, cudaStream_t stream, bool b_mn = false);
+                             void* C, int32_t* status, cudaStream_t stream, bool b_mn = false,
+                             int pdl_mode = 0);
 // C[M,N] (fp32) = A B^T, or C += it when accumulate; A [M][K] or, with a_mn,
 // [K][M]; B [N][K] or, with b_mn, [K][N].
 cudaError_t launch_gemm_f32(const void* A, const void* B, int64_t M, int N, int K,

@@ -41,7 +41,7 @@ struct FwdLayout {
   int splits;
   bool tc;
   bool fused;  // the one-kernel selection (k_select_tc.cu)
-  bool small;  // decode-sized batches: per-chunk lists (k_score_small.cu)
+  bool small;  // decode-sized batches: the one-kernel selection of k_select_small.cu
 };
 
 static bool has_memplus(const pkm_fwd_args* a) { return a->x || a->W1 || a->W2; }
@@ -54,10 +54,9 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
   // split the sub-key columns over CTAs (score_topk_tc) and combine apart
   L.fused = select_tc_supported(a->dtype, a->d_half, a->n_sub, a->k) &&
             a->T > kSplitGatherMaxBags;
-  L.small = !L.fused && score_small_supported(a->dtype, a->T, a->d_half, a->n_sub, a->k);
+  L.small = !L.fused && select_small_supported(a->dtype, a->T, a->d_half, a->n_sub, a->k);
   L.tc = !L.fused && !L.small && score_tc_supported(a->dtype, a->d_half, a->n_sub, a->k);
-  L.splits = L.small ? score_small_chunks(a->n_sub)
-                     : (L.tc ? score_tc_splits(a->T, a->H, a->n_sub) : 1);
+  L.splits = L.tc ? score_tc_splits(a->T, a->H, a->n_sub) : 1;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -65,9 +64,11 @@ static FwdLayout fwd_layout(const pkm_fwd_args* a) {
     return o;
   };
   // padded by one chunk of columns: the scoring epilogues read 8 at a time
-  L.rk = take((H * 2 * n + 256) * sizeof(float));
+  if (!L.small) L.rk = take((H * 2 * n + 256) * sizeof(float));
   if (L.fused) {
     L.sel = take(select_tc_workspace((int64_t)T, (int)H));
+  } else if (L.small) {
+    L.sel = take(select_small_workspace((int64_t)T, (int)H, (int)n));
   } else {
     L.rq = take(T * H * 2 * sizeof(float));
     L.hv = take((size_t)L.splits * T * H * 2 * k * sizeof(float));
@@ -156,10 +157,12 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
   char* g = mp ? ws + L.g : nullptr;
   char* z = mp ? ws + L.z : nullptr;
 
-  // a1: qk-normalisation factors (the query's inside the one-kernel selection)
+  // a1: qk-normalisation factors (inside the one-kernel selections: the
+  // query's in both, the sub-keys' too in the small-batch one)
   mark(a, 0, st);
-  if (!L.fused) PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
-  PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
+  if (!L.fused && !L.small) PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
+  if (!L.small)
+    PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
   mark(a, 1, st);
 
   if (L.fused) {
@@ -167,12 +170,14 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
     PKM_TRY(launch_select_tc(a->query, a->subkeys, T, H, dh, n, k, rk, a->idx, a->weights,
                              ws + L.sel, status, st));
     mark(a, 2, st);
+  } else if (L.small) {
+    // a1 .. a5 in one kernel
+    PKM_TRY(launch_select_small(a->query, a->subkeys, T, H, dh, n, k, a->idx, a->weights,
+                                ws + L.sel, status, st));
+    mark(a, 2, st);
   } else {
     // a2 + a3: sub-key scores and per-half top-k
-    if (L.small)
-      PKM_TRY(launch_score_topk_small(a->query, a->subkeys, T, H, dh, n, k, rq, rk, hv, hi,
-                                      status, st));
-    else if (L.tc)
+    if (L.tc)
       PKM_TRY(launch_score_topk_tc(a->query, a->subkeys, T, H, dh, n, k, L.splits, rq, rk, hv,
                                    hi, status, st));
     else
@@ -184,24 +189,31 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
   }
   mark(a, 3, st);
   if (select_only) return PKM_OK;
+  // Few-token batches chain their kernels by programmatic dependent launch:
+  // the gate GEMM runs beside the selection (it reads neither idx nor w),
+  // and each later kernel waits in-kernel for its predecessor's results
+  // instead of at the launch.
+  const bool few = T <= kSplitGatherMaxBags;
   // (a7) gate GEMM, a6 bag gather over the H*k selected rows of each token
   if (mp)  // g = silu(x W1), W1 [d_model][d_v] read as it is held
-    PKM_TRY(launch_gemm_bf16(a->x, a->W1, T, dv, dm, /*silu*/ 1, g, status, st, /*b_mn*/ true));
+    PKM_TRY(launch_gemm_bf16(a->x, a->W1, T, dv, dm, /*silu*/ 1, g, status, st, /*b_mn*/ true,
+                             few ? 2 : 0));
   mark(a, 4, st);
   // with y_out the bag output is kept and the gate applied in a second pass
   const void* gate = a->y_out ? nullptr : g;
   void* bag_out = a->y_out ? a->y_out : (mp ? z : a->out);
-  if (T <= kSplitGatherMaxBags)
+  if (few)
     PKM_TRY(launch_embbag_fwd_split(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k,
                                     gate, bag_out, reinterpret_cast<float*>(ws + L.part),
-                                    status, st));
+                                    status, st, /*pdl*/ true));
   else
     PKM_TRY(launch_embbag_fwd(a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, gate,
                               bag_out, status, st));
   if (a->y_out) PKM_TRY(launch_gate_mul_bf16(a->y_out, g, T * dv, z, st));
   mark(a, 5, st);
   if (mp)  // out = z W2, W2 [d_v][d_model] read as it is held
-    PKM_TRY(launch_gemm_bf16(z, a->W2, T, dm, dv, /*none*/ 0, a->out, status, st, true));
+    PKM_TRY(launch_gemm_bf16(z, a->W2, T, dm, dv, /*none*/ 0, a->out, status, st, true,
+                             few && !a->y_out ? 1 : 0));
   mark(a, 6, st);
   return PKM_OK;
 }

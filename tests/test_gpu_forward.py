@@ -108,15 +108,21 @@ def test_forward_fused_selection(case):
     run_forward(w)
 
 
-# Batches of at most 32 tokens (decode steps) score each 256-column chunk of
-# a (head, half) in its own CTA and sort the chunk's scores per token across a
-# warp; 33..64 tokens keep the column-split kernel with per-thread top-k.
+# Batches of at most 32 tokens (decode steps) run the one-kernel small-batch
+# selection: each 256-column chunk of a (head, half) in its own CTA (sub-key
+# and query norms from the staged tiles, the chunk's scores sorted per token
+# across a warp), the last CTA of a half merging the chunks' lists and the
+# last half of a head combining; 33..64 tokens keep the column-split kernel
+# with per-thread top-k.
 SMALL_T = [
     # name, T, H, d_half, n_sub, k, d_v
     ("small-t8", 8, 4, 64, 1024, 32, 64),
     ("small-t32-ragged-chunk", 32, 2, 128, 300, 16, 32),
     ("small-t1-k1", 1, 1, 64, 256, 1, 16),
     ("small-t5-k7", 5, 3, 192, 700, 7, 24),
+    ("small-t3-32-chunks", 3, 2, 64, 8192, 32, 8),
+    ("small-t8-wide", 8, 2, 512, 4096, 32, 32),
+    ("small-t17-k31-ragged", 17, 1, 256, 1100, 31, 16),
     ("split-t40", 40, 2, 64, 512, 32, 32),
 ]
 
@@ -142,6 +148,21 @@ def test_forward_fused_launches():
     torch.cuda.synchronize()
     assert lib.pkm_launch_count() - c0 == 3
     assert skv.device_error() == 0
+
+def test_forward_small_launches():
+    """A decode-sized batch launches three kernels in all: the one-kernel
+    selection and the two steps of the row-group gather."""
+    w = WORKLOADS["pkm"].scaled(T=8, H=2, d_half=64, n_sub=512, k=32, d_v=64)
+    inp = make_inputs(w, "cuda")
+    lib = skv.load()
+    skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k)
+    torch.cuda.synchronize()
+    c0 = lib.pkm_launch_count()
+    skv.pkm_forward(inp["query"], inp["subkeys"], inp["values"], w.k)
+    torch.cuda.synchronize()
+    assert lib.pkm_launch_count() - c0 == 3
+    assert skv.device_error() == 0
+
 
 @pytest.mark.parametrize("sign", [1.0, -1.0], ids=["aligned", "anti-aligned"])
 def test_forward_extreme_scores(sign):
