@@ -166,108 +166,109 @@ static bool tc_ok(int64_t M, int N, int K, bool a_mn, bool b_mn) {
 
 // Few rows (decode batches): C[M,N] = epi(A[M,K] W) with W [K][N] held
 // N-contiguous, on the SIMT cores.  A 128-row tensor-core tile would be
-// mostly padding and a handful of CTAs would stream all of W, so here every
-// CTA reads a 32-column strip of W exactly once for up to 8 rows of A: its
-// 8 warps split K; lane l takes 8 columns (one 16-byte vector) of the strip
-// and every 8th k of its warp's range, keeping 8 weight loads in flight, and
-// FMAs each vector into 8 rows x 8 columns of fp32 partials; the 8 lanes
-// sharing columns are summed with shuffles, the 8 warps' sums in warp order
-// through shared memory (a fixed order: the result is reproducible).  A^T
-// [K][8] is staged in shared memory so one 16-byte load gives A[0..7][k].
+// mostly padding, and the work is reading W once, so W is spread over many
+// CTAs: each reads an 8-column strip (one 16-byte vector per k) for up to 8
+// rows of A.  Its 8 warps split K; lane l takes every 32nd k of its warp's
+// range with all of its weight loads in flight at once, and FMAs each vector
+// into 8 rows x 8 columns of fp32 partials.  The 32 lanes' partials are
+// summed by a butterfly that halves the values a lane holds at each of its
+// five exchange steps (lane l ends with outputs 2l and 2l+1), the 8 warps'
+// sums in warp order through shared memory: a fixed order, so the result is
+// reproducible.  A^T [K][8] is staged in shared memory (one 16-byte load
+// gives A[0..7][k]), every 8 k-lines padded by 16 bytes so that the
+// staging threads' stores spread over the banks.
 constexpr int kSmallM = 8;
-constexpr int kSmallCols = 32;
-constexpr int kSmallMaxK = 1024;  // A^T and the partial sums stay within 48 KiB of static shared memory
-constexpr int kSmallBatch = 8;    // weight loads in flight per thread
+constexpr int kSmallCols = 8;
+constexpr int kSmallMaxK = 1024;            // A^T fits 18 KiB of static shared memory
+constexpr int kSmallWarps = 8;
+constexpr int kSmallRowsPerLane = kSmallMaxK / kSmallWarps / 32;  // weight loads in flight
+
+__device__ __forceinline__ int at_index(int k) { return k * kSmallM + (k >> 3) * kSmallM; }
 
 // pdl_mode (programmatic dependent launch): 1 -- A is the previous kernel's
 // output, wait for it first; 2 -- the inputs do not depend on the previous
 // kernel, wait for it only before finishing (so that this kernel's completion
 // still implies that one's); 0 -- ordinary launch.
-__global__ void __launch_bounds__(256) gemm_small_m_kernel(const __nv_bfloat16* __restrict__ A,
-                                                           const __nv_bfloat16* __restrict__ W,
-                                                           int M, int N, int K, int epi,
-                                                           __nv_bfloat16* __restrict__ C,
-                                                           int pdl_mode) {
-  __shared__ __align__(16) uint16_t at[kSmallMaxK * kSmallM];  // A^T: [k][m] bf16 bits
-  __shared__ float part[8][kSmallM][kSmallCols];               // per-warp sums
+__global__ void __launch_bounds__(kSmallWarps * 32) gemm_small_m_kernel(
+    const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ W, int M, int N, int K,
+    int epi, __nv_bfloat16* __restrict__ C, int pdl_mode) {
+  __shared__ __align__(16) uint16_t at[kSmallMaxK * kSmallM + kSmallMaxK];  // A^T, padded
+  __shared__ float part[kSmallWarps][kSmallM * kSmallCols];
   const int n0 = blockIdx.x * kSmallCols;
   const int m0 = blockIdx.y * kSmallM;
   const int mc = min(kSmallM, M - m0);
-  pdl_launch_dependents();
-  if (pdl_mode == 1) pdl_wait();
-  // stage A^T: 16-byte row pieces of A, scattered by k (K % 8 == 0)
-  for (int i = threadIdx.x; i < kSmallM * (K / 8); i += blockDim.x) {
-    const int m = i / (K / 8), kc = i % (K / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (m < mc) v = *reinterpret_cast<const uint4*>(A + (int64_t)(m0 + m) * K + kc * 8);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      at[(kc * 8 + 2 * e) * kSmallM + m] = (uint16_t)(w[e] & 0xffffu);
-      at[(kc * 8 + 2 * e + 1) * kSmallM + m] = (uint16_t)(w[e] >> 16);
-    }
-  }
-  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cv = lane & 3, kq = lane >> 2;  // column vector, k phase
-  const int ncol = n0 + cv * 8;
-  const int kw = (K + 7) / 8;  // k range of a warp
+  pdl_launch_dependents();
+  // this lane's weight vectors, loaded before anything waits
+  const int kw = (K + kSmallWarps - 1) / kSmallWarps;
   const int kb = warp * kw, ke = min(K, kb + kw);
-  float acc[kSmallM][8];
+  uint4 wv[kSmallRowsPerLane];
 #pragma unroll
-  for (int m = 0; m < kSmallM; ++m)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[m][c] = 0.f;
-  if (ncol < N) {
-    for (int k0 = kb + kq; k0 < ke; k0 += 8 * kSmallBatch) {
-      uint4 wv[kSmallBatch];
-#pragma unroll
-      for (int u = 0; u < kSmallBatch; ++u) {
-        const int kk = k0 + 8 * u;
-        wv[u] = kk < ke ? ldg_nc_16(W + (int64_t)kk * N + ncol) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < kSmallBatch; ++u) {
-        const int kk = k0 + 8 * u;
-        if (kk < ke) {
-          const uint4 av = *reinterpret_cast<const uint4*>(at + kk * kSmallM);
-          float wf[8], af[8];
-          unpack16<PKM_BF16>(wv[u], wf);
-          unpack16<PKM_BF16>(av, af);
-#pragma unroll
-          for (int m = 0; m < kSmallM; ++m)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) acc[m][c] = fmaf(af[m], wf[c], acc[m][c]);
-        }
-      }
-    }
+  for (int r = 0; r < kSmallRowsPerLane; ++r) {
+    const int kk = kb + lane + 32 * r;
+    wv[r] = kk < ke ? ldg_nc_16(W + (int64_t)kk * N + n0) : make_uint4(0u, 0u, 0u, 0u);
   }
-  // lanes cv, cv+4, ..., cv+28 hold the same columns: sum them
+  if (pdl_mode == 1) pdl_wait();
+  // stage A^T: thread kc transposes the 8 x 8 block A[0..7][8 kc .. 8 kc + 7]
+  for (int kc = threadIdx.x; kc < K / 8; kc += blockDim.x) {
+    uint32_t u[kSmallM][4];
 #pragma unroll
-  for (int m = 0; m < kSmallM; ++m)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float v = acc[m][c];
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 16);
-      acc[m][c] = v;
+    for (int m = 0; m < kSmallM; ++m) {
+      const uint4 v = m < mc ? *reinterpret_cast<const uint4*>(A + (int64_t)(m0 + m) * K + kc * 8)
+                             : make_uint4(0u, 0u, 0u, 0u);
+      u[m][0] = v.x;
+      u[m][1] = v.y;
+      u[m][2] = v.z;
+      u[m][3] = v.w;
     }
-  if (kq == 0) {
 #pragma unroll
-    for (int m = 0; m < kSmallM; ++m)
+    for (int j = 0; j < 8; ++j) {
+      uint32_t o[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) part[warp][m][cv * 8 + c] = acc[m][c];
+      for (int q = 0; q < 4; ++q)
+        o[q] = __byte_perm(u[2 * q][j >> 1], u[2 * q + 1][j >> 1], (j & 1) ? 0x7632 : 0x5410);
+      *reinterpret_cast<uint4*>(at + at_index(kc * 8 + j)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kSmallM * kSmallCols; i += blockDim.x) {
-    const int m = i / kSmallCols, c = i % kSmallCols;
-    if (m >= mc || n0 + c >= N) continue;
+  float acc[kSmallM * kSmallCols];  // [m][c]
+#pragma unroll
+  for (int i = 0; i < kSmallM * kSmallCols; ++i) acc[i] = 0.f;
+#pragma unroll
+  for (int r = 0; r < kSmallRowsPerLane; ++r) {
+    const int kk = kb + lane + 32 * r;
+    if (kk < ke) {
+      float wf[8], af[8];
+      unpack16<PKM_BF16>(wv[r], wf);
+      unpack16<PKM_BF16>(*reinterpret_cast<const uint4*>(at + at_index(kk)), af);
+#pragma unroll
+      for (int m = 0; m < kSmallM; ++m)
+#pragma unroll
+        for (int c = 0; c < kSmallCols; ++c) acc[m * kSmallCols + c] = fmaf(af[m], wf[c], acc[m * kSmallCols + c]);
+    }
+  }
+  // butterfly over the lanes: at the step with mask h the lanes with bit h
+  // keep the upper half of their values and add their partner's copy of it
+#pragma unroll
+  for (int h = 16, cnt = kSmallM * kSmallCols; h > 0; h >>= 1, cnt >>= 1) {
+    const bool upper = (lane & h) != 0;
+#pragma unroll
+    for (int i = 0; i < cnt / 2; ++i) {
+      const float send = upper ? acc[i] : acc[i + cnt / 2];
+      const float keep = upper ? acc[i + cnt / 2] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, h);
+    }
+  }
+  part[warp][2 * lane] = acc[0];
+  part[warp][2 * lane + 1] = acc[1];
+  __syncthreads();
+  if (threadIdx.x < kSmallM * kSmallCols) {
+    const int m = threadIdx.x / kSmallCols, c = threadIdx.x % kSmallCols;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += part[w][m][c];
+    for (int w = 0; w < kSmallWarps; ++w) v += part[w][threadIdx.x];
     if (epi == 1) v = silu_f(v);
-    C[(int64_t)(m0 + m) * N + n0 + c] = __float2bfloat16_rn(v);
+    if (m < mc && n0 + c < N) C[(int64_t)(m0 + m) * N + n0 + c] = __float2bfloat16_rn(v);
   }
   if (pdl_mode == 2) pdl_wait();
 }
@@ -279,7 +280,7 @@ cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int
   if (b_mn && M <= 64 && K <= kSmallMaxK && K % 8 == 0 && N % 8 == 0) {
     dim3 grid((unsigned)((N + kSmallCols - 1) / kSmallCols), (unsigned)((M + kSmallM - 1) / kSmallM));
     const cudaError_t e = launch_maybe_pdl(
-        pdl_mode != 0, gemm_small_m_kernel, grid, dim3(256), 0, stream,
+        pdl_mode != 0, gemm_small_m_kernel, grid, dim3(kSmallWarps * 32), 0, stream,
         static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), (int)M, N, K,
         epi, static_cast<__nv_bfloat16*>(C), pdl_mode);
     note_launch();

@@ -15,6 +15,7 @@
 //              (bf16, 128-byte swizzle) into a 4-stage ring.
 //   warp 1     TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128,
 //              N=256, fp32 accumulator in 256 TMEM columns.
+//   warps 6-7  the table of the k x k cells the combine reads.
 //   warps 2-5  norms: while each k-block sits in shared memory they add the
 //              squares of the chunk's 256 sub-key rows and of the token rows
 //              (the swizzle only permutes 16-byte pieces within a row); the
@@ -53,7 +54,7 @@ constexpr int kStages = 4;
 constexpr int kABytes = kM * kKB * 2;
 constexpr int kBBytes = kN * kKB * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;      // 8 warps: up to 8 tokens per round of the list phases
 constexpr int kWarps = kThreads / 32;
 constexpr int kNormThreads = 128;  // warps 2..5
 constexpr int kMaxRows = 32;
@@ -246,6 +247,10 @@ __global__ void __launch_bounds__(ssm::kThreads, 1) select_small_kernel(
       for (unsigned long long i = 0; i < kSpinLimit; ++i)
         if (mbar_try_wait(&ctl->drain, 0)) break;
     }
+  } else if (warp >= 6) {
+    // ------------------------------------- the k x k cells (for the combine)
+    if (run)
+      for (int e = threadIdx.x - 192; e < kCellSlots; e += 64) cells[e] = topk_cell(e, k);
   } else if (run) {
     // ------------------------------------------------ norms, then scores
     const int tid = threadIdx.x - 64;  // 0..127
@@ -367,8 +372,6 @@ __global__ void __launch_bounds__(ssm::kThreads, 1) select_small_kernel(
   if (!ctl->combine) return;
 
   // ------------------ the second half of the head to arrive: k x k combine
-  if (threadIdx.x < kCellSlots) cells[threadIdx.x] = topk_cell(threadIdx.x, k);
-  __syncthreads();
   for (int t = warp; t < T; t += kWarps) {
     const bool in = lane < k;
     const uint64_t e1 = ld_cg_u64(half_lists + ((int64_t)(2 * h) * T + t) * kList + lane);
