@@ -291,8 +291,9 @@ def graph_launches(lib, step) -> int:
 
 
 def traffic_record(workload: str):
-    """dram bytes per gather launch from the committed ncu summary, or None
-    when the gather kernel's source changed since it was captured."""
+    """dram bytes per launch of a kernel ("<workload>" the gather,
+    "<workload>:select" the selection) from the committed ncu summaries, or
+    None when the kernel's source changed since it was captured."""
     path = os.path.join(PROFILES, "traffic.json")
     if not os.path.exists(path):
         return None
@@ -405,22 +406,37 @@ def run_ours(args, rank, world, local):
         for i in range(K):
             if flush_between:
                 flush.zero_()  # L2 flush between timed steps (outside the events)
+            ev[i][0].record()
             if graph is not None:
-                ev[i][0].record()
                 graph.replay()
-                ev[i][6].record()
             else:
-                step(ev[i], bev[i] if train else None)
+                step()
+            ev[i][6].record()
         torch.cuda.synchronize()
     launches = lib.pkm_launch_count() - launches0
     if graph is not None:  # kernels replayed from the graph: one step's launches x K
         launches = graph_launches(lib, step) * K
     barrier(world)
-    step_ms = [(e[0].elapsed_time(e[6]) if not train else e[0].elapsed_time(b[1]))
-               for e, b in zip(ev, bev)]
-    phase_ms = None if graph is not None else \
-        [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(6)]
+    step_ms = [e[0].elapsed_time(e[6]) for e in ev]
     total_ms = max_over_ranks(sum(step_ms), world)
+    # Phases from separate (untimed) steps with the library's phase events:
+    # an event recorded between two kernels serialises them, so the timed
+    # steps above run without any (their kernels overlap by programmatic
+    # dependent launch) and these give the per-phase split.
+    phase_ms = None
+    if graph is None:
+        P = min(K, 20)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(P)]
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(P)]
+        for e in sum(ev, []) + sum(bev, []):
+            e.record()
+        torch.cuda.synchronize()
+        for i in range(P):
+            if flush_between:
+                flush.zero_()
+            step(ev[i], bev[i] if train else None)
+        torch.cuda.synchronize()
+        phase_ms = [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(6)]
     assert skv.device_error() == 0
     ms_per_step = total_ms / K
     value = whole_job_tokens_per_s(T, world, ms_per_step)
@@ -442,7 +458,7 @@ def run_ours(args, rank, world, local):
         phases = dict(zip(["norms", "score_topk", "combine_softmax", "gate_gemm", "gather",
                            "out_gemm"], [round(statistics.mean(p) * 1e3, 2) for p in phase_ms]))
         sel = selection_roofline(w, statistics.mean(phase_ms[1]) + statistics.mean(phase_ms[2]),
-                                 peaks, peak_kind)
+                                 peaks, peak_kind, traffic_record(args.workload + ":select"))
     else:  # graph replay: only whole steps are timed
         achieved = bytes_per_launch / (ms_per_step / 1e3) / 1e9
         roof = {"kernel": "whole step (graph replay)", "bound": "hbm",
@@ -538,9 +554,11 @@ def selection_flops(w) -> int:
     return 2 * w.T * w.H * 2 * w.n_sub * w.d_half
 
 
-def selection_roofline(w, sel_ms: float, peaks, peak_kind):
+def selection_roofline(w, sel_ms: float, peaks, peak_kind, traffic=None):
     """The selection (sub-key norms and the selection kernel(s)) against the
-    measured bf16 tensor peak: the scoring GEMM is its dense contraction."""
+    measured bf16 tensor peak: the scoring GEMM is its dense contraction.
+    `traffic`: the selection kernel's DRAM bytes per launch from the committed
+    ncu summary (None when its source changed since the capture)."""
     flops = selection_flops(w)
     tf = flops / (sel_ms / 1e3) / 1e12
     pk = float(peaks["bf16_tflops"])
@@ -548,7 +566,7 @@ def selection_roofline(w, sel_ms: float, peaks, peak_kind):
                       "softmax) after the sub-key norms", "bound": "tensor",
             "achieved": round(tf, 1), "peak": pk, "unit": "TFLOP/s", "frac": round(tf / pk, 4),
             "peak_source": f"{peak_kind} bf16_tflops", "flops_per_launch": flops,
-            "traffic": None, "select_us": round(sel_ms * 1e3, 2)}
+            "traffic": traffic, "select_us": round(sel_ms * 1e3, 2)}
 
 
 def dist_stats(ms):

@@ -154,7 +154,7 @@ cudaError_t launch_gemm_simt(const void* A, const void* B, int64_t M, int N, int
 }
 cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
                            int out_mode, void* C, int32_t* status, cudaStream_t stream,
-                           int splits, int64_t c_split, bool a_mn, bool b_mn);
+                           int splits, int64_t c_split, bool a_mn, bool b_mn, int pdl_mode = 0);
 
 // Shapes the tensor-core GEMM takes: the TMA rows of every operand are a
 // multiple of 16 bytes (K for a K-major operand, M / N for an MN-major one).
@@ -287,7 +287,7 @@ cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int
     return e != cudaSuccess ? e : cudaGetLastError();
   }
   if (tc_ok(M, N, K, false, b_mn))
-    return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream, 1, 0, false, b_mn);
+    return launch_gemm_tc(A, B, M, N, K, epi, 0, C, status, stream, 1, 0, false, b_mn, pdl_mode);
   return launch_gemm_simt(A, B, M, N, K, epi, 0, C, stream, false, b_mn);
 }
 

@@ -88,11 +88,15 @@ template <int EPI, int OUT, bool AMN, bool BMN>
 __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int64_t M,
     int N, int K, void* __restrict__ Cv, int kb_per_split, int nz, int64_t c_split,
-    int32_t* status) {
+    int32_t* status, int pdl_mode) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* stages = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmCtl* ctl = reinterpret_cast<GemmCtl*>(stages + gm::kStages * gm::kStageBytes);
+  // programmatic dependent launch: 1 -- an operand is the previous kernel's
+  // output, wait for it first; 2 -- none is, wait only before finishing
+  pdl_launch_dependents();
+  if (pdl_mode == 1) pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (int)((M + gm::kM - 1) / gm::kM);
   const int tiles_n = (N + gm::kN - 1) / gm::kN;
@@ -289,6 +293,7 @@ __global__ void __launch_bounds__(gm::kThreads, 1) gemm_tc_kernel(
     tc_fence_after();
     tmem_dealloc(tmem, gm::kAcc * gm::kN);
   }
+  if (pdl_mode == 2) pdl_wait();
 }
 
 bool gemm_tc_supported(int64_t M, int N, int K) {
@@ -313,8 +318,14 @@ static int num_sms() {
 // a_mn / b_mn: A is [K][M] / B is [K][N] (M / N contiguous) instead of [M][K] / [N][K].
 cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K, int epi,
                            int out_mode, void* C, int32_t* status, cudaStream_t stream,
-                           int splits, int64_t c_split, bool a_mn, bool b_mn) {
+                           int splits, int64_t c_split, bool a_mn, bool b_mn, int pdl_mode) {
   if (M <= 0) return cudaSuccess;
+  // more than one 128-row tile: pairs of SMs share 256 x 256 tiles (k_gemm_tc2.cu)
+  if (gemm_tc2_useful(M)) {
+    const cudaError_t e2 = launch_gemm_tc2(A, B, M, N, K, epi, out_mode, C, status, stream,
+                                           splits, c_split, a_mn, b_mn, pdl_mode);
+    if (e2 != cudaErrorNotSupported) return e2;
+  }
   CUtensorMap tmA, tmB;
   if (a_mn) {
     if (M % 8) return cudaErrorInvalidValue;  // the row stride of [K][M] is 16-byte aligned
@@ -352,8 +363,8 @@ cudaError_t launch_gemm_tc(const void* A, const void* B, int64_t M, int N, int K
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)gm::kSmemBytes);
     if (e != cudaSuccess) return;
-    kern<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(tmA, tmB, M, N, K, C, kbps, nz, c_split,
-                                                         status);
+    e = launch_maybe_pdl(pdl_mode != 0, kern, dim3(grid), dim3(gm::kThreads), gm::kSmemBytes,
+                         stream, tmA, tmB, M, N, K, C, kbps, nz, c_split, status, pdl_mode);
   };
 #define PKM_GEMM_LAYOUTS(E_, O_)                                   \
   if (a_mn && b_mn) go(gemm_tc_kernel<E_, O_, true, true>);        \

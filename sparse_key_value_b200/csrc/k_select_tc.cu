@@ -288,6 +288,9 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
   const int nch = (n + kN - 1) / kN;
   const int KB = dh / kKB;
   const bool misaligned = (smem_u32(smem_raw) & 1023u) != 0;  // the same in every CTA
+  // the next kernel (the Memory+ gate GEMM, which reads neither idx nor w)
+  // may start on SMs this grid's last wave leaves free
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {

@@ -99,7 +99,7 @@ cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64
 cudaError_t launch_embbag_fwd(const void* table, int64_t n_rows, int d, pkm_dtype dt,
                               const int32_t* idx, const float* w, int64_t n_bags, int B,
                               const void* gate, void* out, int32_t* status, cudaStream_t stream,
-                              int ctas_per_sm = 4);
+                              int ctas_per_sm = 4, bool pdl = false);
 
 // The same gather for small batches (see k_embbag_split.cu): fp32 partial
 // sums of row groups in `part` (embbag_split_workspace bytes), then an
@@ -128,9 +128,15 @@ cudaError_t launch_transpose_bf16(const void* src, int rows, int cols, void* dst
                                   cudaStream_t stream, int ld = 0);
 // C[M,N] = epi(A[M,K] * B[N,K]^T) in bf16; epi: 0 none, 1 silu.  A is
 // [M][K]; B is [N][K], or [K][N] with b_mn (a weight [d_in, d_out] used as x W).
-// pdl_mode (few-row batches only; ignored otherwise): 0 ordinary launch;
-// programmatic dependent launch with 1 -- A comes from the previous kernel,
-// 2 -- A and B do not (the kernel overlaps the previous one).
+// pdl_mode: 0 ordinary launch; programmatic dependent launch with 1 -- A
+// comes from the previous kernel, 2 -- A and B do not (the kernel overlaps
+// the previous one and waits for it only before finishing).
+// The same GEMMs on CTA pairs (tcgen05 cta_group::2, 256 x 256 tiles);
+// cudaErrorNotSupported (nothing launched) when no pair can be resident.
+bool gemm_tc2_useful(int64_t M);
+cudaError_t launch_gemm_tc2(const void* A, const void* B, int64_t M, int N, int K, int epi,
+                            int out_mode, void* C, int32_t* status, cudaStream_t stream,
+                            int splits, int64_t c_split, bool a_mn, bool b_mn, int pdl_mode = 0);
 bool gemm_tc_supported(int64_t M, int N, int K);
 cudaError_t launch_gemm_bf16(const void* A, const void* B, int64_t M, int N, int K, int epi,
                              void* C, int32_t* status, cudaStream_t stream, bool b_mn = false,

@@ -189,15 +189,17 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
   }
   mark(a, 3, st);
   if (select_only) return PKM_OK;
-  // Few-token batches chain their kernels by programmatic dependent launch:
-  // the gate GEMM runs beside the selection (it reads neither idx nor w),
-  // and each later kernel waits in-kernel for its predecessor's results
-  // instead of at the launch.
+  // Programmatic dependent launch: the gate GEMM runs beside the selection
+  // (it reads neither idx nor w) on the SMs the selection's last wave leaves
+  // free.  Few-token batches chain the later kernels the same way (each
+  // waits in-kernel for its predecessor's results instead of at the launch);
+  // for large batches an early-launched gather measured slower (its waiting
+  // CTAs crowd the SMs as the selection drains), so those launch as usual.
   const bool few = T <= kSplitGatherMaxBags;
   // (a7) gate GEMM, a6 bag gather over the H*k selected rows of each token
   if (mp)  // g = silu(x W1), W1 [d_model][d_v] read as it is held
     PKM_TRY(launch_gemm_bf16(a->x, a->W1, T, dv, dm, /*silu*/ 1, g, status, st, /*b_mn*/ true,
-                             few ? 2 : 0));
+                             /*pdl: overlap*/ 2));
   mark(a, 4, st);
   // with y_out the bag output is kept and the gate applied in a second pass
   const void* gate = a->y_out ? nullptr : g;
@@ -213,7 +215,7 @@ static pkm_status forward_impl(const pkm_fwd_args* a, cudaStream_t st,
   mark(a, 5, st);
   if (mp)  // out = z W2, W2 [d_v][d_model] read as it is held
     PKM_TRY(launch_gemm_bf16(z, a->W2, T, dm, dv, /*none*/ 0, a->out, status, st, true,
-                             few && !a->y_out ? 1 : 0));
+                             few && !a->y_out ? /*pdl: z from the gather*/ 1 : 0));
   mark(a, 6, st);
   return PKM_OK;
 }

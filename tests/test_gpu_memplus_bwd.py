@@ -73,7 +73,13 @@ def test_memplus_backward_deterministic():
         assert torch.equal(a[key], b[key]), key
 
 
-@pytest.mark.parametrize("T,dm,dq", [(300, 128, 256), (50, 32, 64)])
+# (T, d_model, d_q): more than 128 tokens runs the GEMMs on SM pairs (256-row
+# tiles, a ragged last pair); 50 tokens the single-SM tensor-core kernel;
+# 4100 x 1024 x 1024 many tiles per pair with a ragged tail
+QPROJ = [(300, 128, 256), (50, 32, 64), (1000, 640, 520), (4100, 1024, 1024)]
+
+
+@pytest.mark.parametrize("T,dm,dq", QPROJ)
 def test_qproj_matches_oracle(T, dm, dq):
     import oracle
 
