@@ -25,8 +25,6 @@ __global__ void __launch_bounds__(kBagThreads, 4) embbag_fwd_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ w, int64_t n_bags, int B,
     const typename Elem<DT>::T* __restrict__ gate, typename Elem<DT>::T* __restrict__ out,
     int bags_per_cta, int32_t* status) {
-  pdl_launch_dependents();
-  pdl_wait();  // idx, w and the gate come from the kernels before this one
   constexpr int V = Elem<DT>::kVec;
   extern __shared__ unsigned char smem_raw[];
   int32_t* s_idx = reinterpret_cast<int32_t*>(smem_raw);       // [bags_per_cta][B]
@@ -121,7 +119,7 @@ template <pkm_dtype DT, bool GATE>
 static cudaError_t launch_embbag_t(const void* table, int64_t n_rows, int d, const int32_t* idx,
                                    const float* w, int64_t n_bags, int B, const void* gate,
                                    void* out, int ctas_per_sm, int32_t* status,
-                                   cudaStream_t stream, bool pdl) {
+                                   cudaStream_t stream) {
   using T = typename Elem<DT>::T;
   const int chunks = d / Elem<DT>::kVec;
   // several bags per CTA when a row has fewer 16-byte chunks than threads
@@ -139,27 +137,26 @@ static cudaError_t launch_embbag_t(const void* table, int64_t n_rows, int d, con
   const int64_t groups = (n_bags + bags_per_cta - 1) / bags_per_cta;
   const int64_t cap = (int64_t)sm_count() * ctas_per_sm;
   dim3 grid((unsigned)(groups < cap ? groups : cap));
-  const cudaError_t e = launch_maybe_pdl(pdl, fn, grid, dim3(kBagThreads), smem, stream,
-                                         (const T*)table, n_rows, d, idx, w, n_bags, B,
-                                         (const T*)gate, (T*)out, bags_per_cta, status);
+  fn<<<grid, kBagThreads, smem, stream>>>((const T*)table, n_rows, d, idx, w, n_bags, B,
+                                          (const T*)gate, (T*)out, bags_per_cta, status);
   note_launch();
-  return e != cudaSuccess ? e : cudaGetLastError();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_embbag_fwd(const void* table, int64_t n_rows, int d, pkm_dtype dt,
                               const int32_t* idx, const float* w, int64_t n_bags, int B,
                               const void* gate, void* out, int32_t* status, cudaStream_t stream,
-                              int ctas_per_sm, bool pdl) {
+                              int ctas_per_sm) {
   if (n_bags <= 0) return cudaSuccess;
   if (dt == PKM_BF16)
     return gate ? launch_embbag_t<PKM_BF16, true>(table, n_rows, d, idx, w, n_bags, B, gate,
-                                                  out, ctas_per_sm, status, stream, pdl)
+                                                  out, ctas_per_sm, status, stream)
                 : launch_embbag_t<PKM_BF16, false>(table, n_rows, d, idx, w, n_bags, B, nullptr,
-                                                   out, ctas_per_sm, status, stream, pdl);
+                                                   out, ctas_per_sm, status, stream);
   return gate ? launch_embbag_t<PKM_F32, true>(table, n_rows, d, idx, w, n_bags, B, gate, out,
-                                               ctas_per_sm, status, stream, pdl)
+                                               ctas_per_sm, status, stream)
               : launch_embbag_t<PKM_F32, false>(table, n_rows, d, idx, w, n_bags, B, nullptr,
-                                                out, ctas_per_sm, status, stream, pdl);
+                                                out, ctas_per_sm, status, stream);
 }
 
 }  // namespace pkm

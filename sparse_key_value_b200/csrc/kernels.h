@@ -99,7 +99,7 @@ cudaError_t launch_combine(const float* hv, const int32_t* hi, int splits, int64
 cudaError_t launch_embbag_fwd(const void* table, int64_t n_rows, int d, pkm_dtype dt,
                               const int32_t* idx, const float* w, int64_t n_bags, int B,
                               const void* gate, void* out, int32_t* status, cudaStream_t stream,
-                              int ctas_per_sm = 4, bool pdl = false);
+                              int ctas_per_sm = 4);
 
 // The same gather for small batches (see k_embbag_split.cu): fp32 partial
 // sums of row groups in `part` (embbag_split_workspace bytes), then an
