@@ -294,15 +294,43 @@ def traffic_record(workload: str):
     """dram bytes per launch of a kernel ("<workload>" the gather,
     "<workload>:select" the selection) from the committed ncu summaries, or
     None when the kernel's source changed since it was captured."""
+    rec = traffic_entry(workload)
+    return rec["dram_bytes_per_launch"] if rec else None
+
+
+def traffic_entry(workload: str):
+    """The committed ncu record of `workload` in profiles/traffic.json, or None
+    when it is missing or any of its kernels' sources changed since."""
     path = os.path.join(PROFILES, "traffic.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(workload)
     if not rec:
         return None
-    src = os.path.join(ROOT, "sparse_key_value_b200", "csrc", rec["source"])
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["dram_bytes_per_launch"] if sha == rec["source_sha"] else None
+    sources = rec.get("sources") or {rec["source"]: rec["source_sha"]}
+    for name, want in sources.items():
+        src = os.path.join(ROOT, "sparse_key_value_b200", "csrc", name)
+        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != want:
+            return None
+    return rec
+
+
+def l2_read_gbs() -> float:
+    """Measured L2 read bandwidth for the L2-bound kernels' second roofline:
+    GB/s of torch's sum over a 64 MiB fp32 tensor that stays L2-resident
+    (an L2 reference, like the HBM copy of MEASURED_PEAKS.json)."""
+    x = torch.ones(16 << 20, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        x.sum()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 50
+    e0.record()
+    for _ in range(reps):
+        x.sum()
+    e1.record()
+    torch.cuda.synchronize()
+    return x.numel() * 4 * reps / (e0.elapsed_time(e1) / 1e3) / 1e9
 
 
 # ------------------------------------------------------------ our arm --
@@ -484,6 +512,20 @@ def run_ours(args, rank, world, local):
                              "algorithmic_bytes": bbytes,
                              "GBps": round(bbytes / (bwd_ms / 1e3) / 1e9, 1),
                              "frac": round(bbytes / (bwd_ms / 1e3) / 1e9 / peak, 4)}
+        # the kernels' own DRAM and L2 bytes (ncu record): repeated (Zipf-hot)
+        # rows are L2 hits, so the backward is bound by L2 traffic more than
+        # by DRAM; both bounds side by side
+        rec = traffic_entry(args.workload + ":backward")
+        if rec:
+            l2bw = l2_read_gbs()
+            db, lb = rec["dram_bytes_per_launch"], rec["l2_bytes_per_launch"]
+            extra["backward"].update(
+                dram_bytes=db, dram_GBps=round(db / (bwd_ms / 1e3) / 1e9, 1),
+                dram_frac=round(db / (bwd_ms / 1e3) / 1e9 / peak, 4),
+                hbm_bound_us=round(db / (peak * 1e9) * 1e6, 1),
+                l2_bytes=lb, l2_read_GBps_measured=round(l2bw, 1),
+                l2_bound_us=round(lb / (l2bw * 1e9) * 1e6, 1),
+                traffic_capture=rec["capture"])
         if mp_train:
             # five GEMMs of 2*T*d_model*d_v FLOPs: a, dz, dx, dW1, dW2
             mp_ms = statistics.mean([b[0].elapsed_time(b[2]) for b in bev])
@@ -505,8 +547,8 @@ def run_ours(args, rank, world, local):
         roof = {"kernel": "pkm_backward (sort, segmented value-gradient sum, dw/dS, dq, dK)",
                 "bound": "hbm", "achieved": b["GBps"], "peak": peak, "unit": "GB/s",
                 "frac": b["frac"], "peak_source": f"{peak_kind} hbm_gbs",
-                "algorithmic_bytes_per_launch": b["algorithmic_bytes"], "traffic": None,
-                "backward_us": b["us"]}
+                "algorithmic_bytes_per_launch": b["algorithmic_bytes"],
+                "traffic": b.get("dram_bytes"), "backward_us": b["us"]}
 
     if train:
         # optimiser step on the touched rows (not part of the timed training
