@@ -144,6 +144,37 @@ cudaError_t launch_bag_dw(const void* dy, const void* table, int64_t n_rows, int
   return cudaGetLastError();
 }
 
+// ----------------------------------------------------------- softmax bwd
+// One warp per group of k <= 64 entries (a token's head): dS = w (dw - <w, dw>).
+__global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* __restrict__ w,
+                                                          const float* __restrict__ dw,
+                                                          int slices, int64_t groups, int k,
+                                                          float* __restrict__ dS) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (g >= groups) return;
+  const int64_t o = g * k, R = groups * k;
+  const bool v0 = lane < k, v1 = lane + 32 < k;
+  const float w0 = v0 ? w[o + lane] : 0.f, w1 = v1 ? w[o + lane + 32] : 0.f;
+  float d0 = 0.f, d1 = 0.f;
+  for (int s = 0; s < slices; ++s) {
+    if (v0) d0 += dw[s * R + o + lane];
+    if (v1) d1 += dw[s * R + o + lane + 32];
+  }
+  const float sum = warp_sum(w0 * d0 + w1 * d1);
+  if (v0) dS[o + lane] = w0 * (d0 - sum);
+  if (v1) dS[o + lane + 32] = w1 * (d1 - sum);
+}
+
+cudaError_t launch_softmax_bwd(const float* w, const float* dw, int slices, int64_t groups, int k,
+                               float* dS, cudaStream_t stream) {
+  if (groups <= 0) return cudaSuccess;
+  softmax_bwd_kernel<<<(unsigned)((groups + 7) / 8), 256, 0, stream>>>(w, dw, slices, groups, k,
+                                                                       dS);
+  note_launch();
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------- dq
 // One warp per (token, head); lane l holds elements [l*E, (l+1)*E) of the
 // d_half-long vectors for E = d_half / 32 (a multiple of 8 up to 64).

@@ -10,6 +10,8 @@
 // segment that crosses chunk boundaries go to per-chunk carry rows and a
 // fix-up kernel adds them in chunk order.  The work per CTA is fixed, so a
 // hot key with many entries (Zipf popularity) spreads over many CTAs.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -241,6 +243,220 @@ __global__ void __launch_bounds__(kThreads) segsum_chunk_kernel(
   }
 }
 
+// ------------------------------------------------ value rows with dw ----
+// The value gradient of the bf16 backward with the softmax's upstream
+// gradient in the same walk: for each sorted (value row r, slot e) entry,
+// grad[r] += w[e] * dy[t(e)] and dw[e] = <dy[t(e)], V[r]> ("Memory Layers at
+// Scale" digest, "병렬 EmbeddingBag 구현": the backward of the weighted bag).
+// One warp per chunk of kChunk entries (same chunks, segment ids and carry
+// rows as segsum_chunk_kernel), holding whole rows: lane l owns the 16-byte
+// column chunks l, l + 32, ...  The rows come through shared memory by bulk
+// copies (cp.async.bulk, one per 16-bit row) into per-warp rings: dy rows
+// kDwRing entries ahead of the warp, the table row of each segment as soon as
+// a ring slot is free (each distinct value row is read once per chunk, not
+// once per slot).  The dot products reduce within the warp, in a fixed order.
+constexpr int kDwRing = 4;   // dy rows in flight per warp
+constexpr int kDwVRing = 4;  // table rows in flight per warp (segments may be one entry long)
+
+__device__ __forceinline__ void bulk_row(void* smem_dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(smem_dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__host__ __device__ inline size_t segsum_dw_warp_smem(int d) {
+  return (size_t)(kDwRing + kDwVRing) * d * 2 + (size_t)kChunk * 16 +
+         (size_t)(kDwRing + kDwVRing) * 8;
+}
+
+// Rows wider than 512 are cut into `slices` column slices, each walked by
+// its own warp; slice s writes its partial dot products to dw_out[s][entry]
+// (summed in slice order by the softmax backward).
+template <int Q>  // 16-byte (8 x bf16) column chunks per lane: d / slices = 256 Q
+__global__ void __launch_bounds__(256) segsum_dw_kernel(
+    const uint32_t* __restrict__ skey, const uint32_t* __restrict__ sval, int64_t n,
+    uint32_t mark, const float* __restrict__ coef, const __nv_bfloat16* __restrict__ src,
+    int64_t div, int d, int slices, SegWs ws, SegOutDev out,
+    const __nv_bfloat16* __restrict__ table, float* __restrict__ dw_out, int32_t* status) {
+  constexpr int E = 8 * Q;
+  extern __shared__ __align__(16) unsigned char smem_dw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const int64_t gw = (int64_t)blockIdx.x * nwarps + warp;
+  const int64_t c = gw / slices;   // chunk
+  const int sl = (int)(gw % slices);
+  const int ds = d / slices;       // this slice's columns
+  const int64_t chunks = (n + kChunk - 1) / kChunk;
+  const size_t per_warp = segsum_dw_warp_smem(ds);
+  unsigned char* base = smem_dw + (size_t)warp * per_warp;
+  __nv_bfloat16* dring = reinterpret_cast<__nv_bfloat16*>(base);
+  __nv_bfloat16* vring = dring + (size_t)kDwRing * ds;
+  uint32_t* key_s = reinterpret_cast<uint32_t*>(vring + (size_t)kDwVRing * ds);
+  uint32_t* row_s = key_s + kChunk;
+  uint32_t* e_s = row_s + kChunk;
+  float* cf_s = reinterpret_cast<float*>(e_s + kChunk);
+  uint64_t* dbar = reinterpret_cast<uint64_t*>(cf_s + kChunk);
+  uint64_t* vbar = dbar + kDwRing;
+  if (c >= chunks) return;  // whole warp
+  const int64_t i0 = c * kChunk;
+  const int len = (int)min((int64_t)kChunk, n - i0);
+  const uint32_t div32 = (uint32_t)div;
+  const uint32_t row_bytes = (uint32_t)ds * 2;
+  const int64_t col0 = (int64_t)sl * ds;  // first column of the slice
+
+  if (lane == 0) {
+    for (int s2 = 0; s2 < kDwRing; ++s2) mbar_init(&dbar[s2], 1);
+    for (int s2 = 0; s2 < kDwVRing; ++s2) mbar_init(&vbar[s2], 1);
+    fence_barrier_init();
+  }
+  int nvalid = 0;
+  for (int j = lane; j < kChunk; j += 32) {
+    const int64_t i = i0 + j;
+    const uint32_t key = j < len ? skey[i] : mark;
+    const uint32_t e = j < len ? sval[i] : 0u;
+    key_s[j] = key;
+    e_s[j] = e;
+    row_s[j] = e / div32;
+    cf_s[j] = key != mark ? coef[e] : 0.f;
+    nvalid += key != mark && j < len;
+  }
+  const int lv = (int)warp_sum((float)nvalid);  // valid entries come first (the mark sorts last)
+  const uint32_t nextk = i0 + len < n ? skey[i0 + len] : mark;
+  const uint32_t prev_key = i0 > 0 ? skey[i0 - 1] : mark;
+  __syncwarp();
+  const uint32_t seg_base = ws.seg_base[c];
+  if (lane == 0 && sl == 0) {
+    ws.first_end[c] = 1;
+    ws.last_seg[c] = 0xffffffffu;
+  }
+  const bool cont0 = key_s[0] != mark && prev_key == key_s[0];
+  volatile int abort_flag = 0;
+
+  // producer state (lane 0 issues): next entry to fetch, table rows fetched
+  int pj = 0, ps = 0;
+  int cs = 0;  // table rows consumed (segments started) so far
+  auto produce = [&](int j) {
+    if (lane == 0) {
+      fence_proxy_async_smem();  // the warp's reads of the freed slots come first
+      while (pj < lv && pj < j + kDwRing) {
+        const bool starts = pj == 0 || key_s[pj] != key_s[pj - 1];
+        if (starts && ps - cs >= kDwVRing) break;  // its table-row slot is still in use
+        const int slot = pj % kDwRing;
+        mbar_arrive_expect_tx(&dbar[slot], row_bytes);
+        bulk_row(dring + (size_t)slot * ds, src + (int64_t)row_s[pj] * d + col0, row_bytes,
+                 &dbar[slot]);
+        if (starts) {
+          const int vs = ps % kDwVRing;
+          mbar_arrive_expect_tx(&vbar[vs], row_bytes);
+          bulk_row(vring + (size_t)vs * ds, table + (int64_t)key_s[pj] * d + col0, row_bytes,
+                   &vbar[vs]);
+          ++ps;
+        }
+        ++pj;
+      }
+    }
+    __syncwarp();
+  };
+
+  float acc[E];
+#pragma unroll
+  for (int q = 0; q < E; ++q) acc[q] = 0.f;
+  uint32_t vr[E / 2];  // the segment's table row, packed bf16 pairs
+  uint32_t heads = 0;
+  bool part_starts = !cont0;
+  int j = 0;
+  for (; j < lv; ++j) {
+    produce(j);
+    const uint32_t key = key_s[j];
+    if (j == 0 || key != key_s[j - 1]) {
+      const int vs = cs % kDwVRing;
+      const bool got = mbar_wait_or_abort(&vbar[vs], (uint32_t)(cs / kDwVRing) & 1,
+                                          &abort_flag, status);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const uint4* vrow = reinterpret_cast<const uint4*>(vring + (size_t)vs * ds);
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        const uint4 t = vrow[lane + 32 * q];
+        vr[4 * q] = t.x;
+        vr[4 * q + 1] = t.y;
+        vr[4 * q + 2] = t.z;
+        vr[4 * q + 3] = t.w;
+      }
+      ++cs;
+    }
+    const int slot = j % kDwRing;
+    const bool got = mbar_wait_or_abort(&dbar[slot], (uint32_t)(j / kDwRing) & 1, &abort_flag,
+                                        status);
+    if (!__all_sync(0xffffffffu, got)) break;
+    const uint4* drow = reinterpret_cast<const uint4*>(dring + (size_t)slot * ds);
+    const float cf = cf_s[j];
+    const float2 w2 = make_float2(cf, cf);
+    float pd[4] = {0.f, 0.f, 0.f, 0.f};  // four partial dot products: short FMA chains
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      const uint4 t = drow[lane + 32 * q];
+      float f[8];
+      unpack16<PKM_BF16>(t, f);
+#pragma unroll
+      for (int e2 = 0; e2 < 8; e2 += 2) {
+        const float2 r = __ffma2_rn(w2, make_float2(f[e2], f[e2 + 1]),
+                                    make_float2(acc[8 * q + e2], acc[8 * q + e2 + 1]));
+        acc[8 * q + e2] = r.x;
+        acc[8 * q + e2 + 1] = r.y;
+        const uint32_t vp = vr[4 * q + e2 / 2];
+        pd[e2 >> 1] = fmaf(f[e2], bf16_lo(vp), pd[e2 >> 1]);
+        pd[e2 >> 1] = fmaf(f[e2 + 1], bf16_hi(vp), pd[e2 >> 1]);
+      }
+    }
+    const float pdot = warp_sum((pd[0] + pd[1]) + (pd[2] + pd[3]));
+    if (lane == 0) dw_out[(int64_t)sl * n + e_s[j]] = pdot;
+    // segment bookkeeping, as in segsum_chunk_kernel
+    const uint32_t nk = j + 1 < len ? key_s[j + 1] : nextk;
+    if (j + 1 < len && nk == key) {
+      __syncwarp();  // every lane is done with slot j before it is refilled
+      continue;
+    }
+    const bool seg_ends = nk != key;
+    if (part_starts) ++heads;
+    const uint32_t seg = seg_base + heads - 1;
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      const int ch = (int)(col0 / 8) + lane + 32 * q;  // 16-byte column chunk of the row
+      if (part_starts && seg_ends) {
+        emit_final<8>(out, seg, key, d, ch, acc + 8 * q, status);
+      } else if (!part_starts) {
+        store_row<8>(ws.carry_first + c * d + (int64_t)ch * 8, acc + 8 * q);
+      } else {
+        store_row<8>(ws.carry_last + c * d + (int64_t)ch * 8, acc + 8 * q);
+      }
+    }
+    if (lane == 0 && sl == 0) {
+      if (!part_starts) ws.first_end[c] = seg_ends ? 1u : 0u;
+      else if (!seg_ends) ws.last_seg[c] = seg;
+    }
+#pragma unroll
+    for (int q = 0; q < E; ++q) acc[q] = 0.f;
+    part_starts = true;
+    __syncwarp();
+  }
+  if (j < lv && lane == 0) {
+    // a wait ran out: let every copy issued land before the warp leaves
+    for (int jj = j; jj < pj; ++jj)
+      for (unsigned long long it = 0; it < kSpinLimit; ++it)
+        if (mbar_try_wait(&dbar[jj % kDwRing], (uint32_t)(jj / kDwRing) & 1)) break;
+    for (int ss = cs; ss < ps; ++ss)
+      for (unsigned long long it = 0; it < kSpinLimit; ++it)
+        if (mbar_try_wait(&vbar[ss % kDwVRing], (uint32_t)(ss / kDwVRing) & 1)) break;
+  }
+  // entries with an invalid row id get dw = 0
+  for (int jj = lv + lane; jj < len; jj += 32) dw_out[(int64_t)sl * n + e_s[jj]] = 0.f;
+}
+
 // Adds the carried pieces of every segment that crosses chunk boundaries.
 template <int V>
 __global__ void __launch_bounds__(kThreads) segsum_fixup_kernel(const uint32_t* __restrict__ skey,
@@ -271,6 +487,14 @@ __global__ void __launch_bounds__(kThreads) segsum_fixup_kernel(const uint32_t* 
 cudaError_t launch_scan_exclusive(uint32_t* data, int64_t len, uint32_t* total, int64_t* total64,
                                   cudaStream_t stream);
 
+bool segsum_has_dw(pkm_dtype dt, int d) {
+  return dt == PKM_BF16 && d % 256 == 0 && d <= 2048 && (d / segsum_dw_slices(d)) % 256 == 0;
+}
+// column slices of the dw walk: 512 columns per warp (narrower slices put more
+// warps on a chunk: each warp's walk over its entries is a chain of dependent
+// steps)
+int segsum_dw_slices(int d) { return d > 512 ? d / 512 : 1; }
+
 // Segmented sums of coef[e] * src[e / div] over the sorted pairs; entries
 // with key == mark (sorted last) are ignored.  Outputs: sparse rows
 // (uniq_rows/grad_rows, capacity cap; n_uniq receives the number of keys),
@@ -279,7 +503,7 @@ cudaError_t launch_segsum(const uint32_t* skey, const uint32_t* sval, int64_t n,
                           const float* coef, const void* src, pkm_dtype dt, int64_t div, int d,
                           int32_t* uniq_rows, float* grad_rows, int64_t cap, int64_t* n_uniq,
                           float* dense_add, float* dense_set, void* workspace, int32_t* status,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, const void* table, float* dw) {
   if (n <= 0) {
     if (n_uniq) return cudaMemsetAsync(n_uniq, 0, sizeof(int64_t), stream);
     return cudaSuccess;
@@ -292,6 +516,37 @@ cudaError_t launch_segsum(const uint32_t* skey, const uint32_t* sval, int64_t n,
   cudaError_t e = launch_scan_exclusive(ws.seg_base, chunks, nullptr, n_uniq, stream);
   if (e != cudaSuccess) return e;
   SegOutDev out{uniq_rows, grad_rows, cap, dense_add, dense_set};
+  if (table && dw && segsum_has_dw(dt, d)) {
+    // value rows with dw: one warp per chunk, rows through bulk-copy rings
+    const int slices = segsum_dw_slices(d);
+    const int ds = d / slices;
+    const size_t per_warp = segsum_dw_warp_smem(ds);
+    const int nw = (int)std::min<size_t>(8, (200u << 10) / per_warp);
+    const size_t smem = per_warp * nw;
+    const unsigned grid = (unsigned)((chunks * slices + nw - 1) / nw);
+    auto go = [&](auto kern) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return;
+      kern<<<grid, 32 * nw, smem, stream>>>(skey, sval, n, mark, coef,
+                                              (const __nv_bfloat16*)src, div, d, slices, ws, out,
+                                              (const __nv_bfloat16*)table, dw, status);
+    };
+    switch (ds / 256) {
+      case 1: go(segsum_dw_kernel<1>); break;
+      case 2: go(segsum_dw_kernel<2>); break;
+      case 3: go(segsum_dw_kernel<3>); break;
+      case 4: go(segsum_dw_kernel<4>); break;
+      case 5: go(segsum_dw_kernel<5>); break;
+      case 6: go(segsum_dw_kernel<6>); break;
+      case 7: go(segsum_dw_kernel<7>); break;
+      default: go(segsum_dw_kernel<8>); break;
+    }
+    if (e != cudaSuccess) return e;
+    segsum_fixup_kernel<8><<<(unsigned)chunks, min(kThreads, ((d / 8) + 31) / 32 * 32), 0,
+                             stream>>>(skey, n, d, ws, out, status);
+    note_launch(2);
+    return cudaGetLastError();
+  }
   const int V = dt == PKM_BF16 ? 8 : 4;
   // two 16-byte column vectors per thread when they divide the row
   const int NV = (d / V) % 2 == 0 ? 2 : 1;

@@ -188,13 +188,23 @@ cudaError_t launch_dk_entries(const int32_t* idx, const float* dS, const float* 
 cudaError_t launch_dk_jacobian(const void* K, pkm_dtype dt, const float* rk, int64_t rows, int dh,
                                float* g, cudaStream_t stream);
 
-// Deterministic segmented sums over sorted (key, entry) pairs.
+// Deterministic segmented sums over sorted (key, entry) pairs.  With `table`
+// and `dw` (bf16, d a multiple of 256 up to 2048): also dw[entry] =
+// <src[entry / div], table[key]>, each segment's table row read once;
+// entries with an invalid key get 0.  segsum_has_dw says whether a shape
+// takes that path.
 size_t segsum_workspace(int64_t n, int d);
+bool segsum_has_dw(pkm_dtype dt, int d);
+int segsum_dw_slices(int d);  // dw comes as [slices][entries] partial sums
 cudaError_t launch_segsum(const uint32_t* skey, const uint32_t* sval, int64_t n, uint32_t mark,
                           const float* coef, const void* src, pkm_dtype dt, int64_t div, int d,
                           int32_t* uniq_rows, float* grad_rows, int64_t cap, int64_t* n_uniq,
                           float* dense_add, float* dense_set, void* workspace, int32_t* status,
-                          cudaStream_t stream);
+                          cudaStream_t stream, const void* table = nullptr, float* dw = nullptr);
+// dS = w (dw - sum over the group of w dw), groups of k consecutive entries;
+// dw = the sum of `slices` partials [slices][groups * k], in slice order
+cudaError_t launch_softmax_bwd(const float* w, const float* dw, int slices, int64_t groups, int k,
+                               float* dS, cudaStream_t stream);
 cudaError_t launch_scan_exclusive(uint32_t* data, int64_t len, uint32_t* total, int64_t* total64,
                                   cudaStream_t stream);
 
