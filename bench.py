@@ -563,7 +563,7 @@ def run_ours(args, rank, world, local):
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world,
+        e2e = run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world, use_graph=use_graph,
                       backward=(lambda: (
                           skv.check(lib.pkm_memplus_backward(skv.ctypes.byref(margs), sptr),
                                     "pkm_memplus_backward") if mp_train else None,
@@ -834,13 +834,15 @@ def time_sparse_adam(skv, table, rows, grads, count, U, w, peak, peak_kind, reps
             "peak_source": f"{peak_kind} hbm_gbs"}
 
 
-def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world, backward=None):
+def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world, backward=None, use_graph=False):
     """Same metric through the public API with host buffers: every step
     copies the step's query (and x, and for training dy) from pinned host
     memory, runs the step and copies the output back.  The copies run on
     their own streams with two device buffers, so the host-to-device copy of
     step i+1 and the device-to-host copy of step i-1 overlap the compute of
-    step i (each step still moves all its bytes inside the timed region)."""
+    step i (each step still moves all its bytes inside the timed region).
+    With `use_graph` (decode) the step's forward on each buffer is a CUDA
+    graph captured once from the same calls and replayed every step."""
     import sparse_key_value_b200 as skv
 
     hq = inp["query"].cpu().pin_memory()
@@ -861,6 +863,26 @@ def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world, backward=None):
     for e in used + drained:
         e.record(comp)
 
+    def forward(b):
+        kw2 = dict(kw)
+        if dx is not None:
+            kw2["x"] = dx[b]
+        skv.pkm_forward(dq[b], inp["subkeys"], inp["values"], w.k, out=dout[b], idx=idx,
+                        weights=wts, workspace=ws, **kw2)
+
+    graphs = None
+    if use_graph and backward is None:
+        for b in range(2):  # eager calls first (workspace lookups happen outside capture)
+            forward(b)
+        torch.cuda.synchronize()
+        graphs = []
+        for b in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                forward(b)
+            graphs.append(g)
+        torch.cuda.synchronize()
+
     def step(i):
         b = i % 2
         h2d.wait_event(used[b])
@@ -873,13 +895,12 @@ def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world, backward=None):
         loaded[b].record(h2d)
         comp.wait_event(loaded[b])
         comp.wait_event(drained[b])
-        kw2 = dict(kw)
-        if dx is not None:
-            kw2["x"] = dx[b]
         if ddy is not None:
             inp["dy"].copy_(ddy[b])  # the backward reads dy from its fixed buffer
-        skv.pkm_forward(dq[b], inp["subkeys"], inp["values"], w.k, out=dout[b], idx=idx,
-                        weights=wts, workspace=ws, **kw2)
+        if graphs is not None:
+            graphs[b].replay()
+        else:
+            forward(b)
         used[b].record(comp)
         if backward is not None:
             backward()
@@ -908,10 +929,14 @@ def run_e2e(args, w, inp, kw, out, idx, wts, ws, flush, world, backward=None):
     nbytes = lambda t: t.numel() * t.element_size()  # noqa: E731
     h2d_b = sum(nbytes(t) for t in (hq, hx, hdy) if t is not None)
     d2h_b = nbytes(hout[0])
-    return {"value": round(world * w.T / (ms / 1e3), 1), "unit": UNIT,
-            "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "ms_per_step": round(ms, 4),
-            "pipeline": "host-to-device copies, compute and device-to-host copies on three "
-                        "streams with two device buffers; one timed region over all steps"}
+    res = {"value": round(world * w.T / (ms / 1e3), 1), "unit": UNIT,
+           "h2d_bytes_per_step": h2d_b, "d2h_bytes_per_step": d2h_b, "ms_per_step": round(ms, 4),
+           "pipeline": "host-to-device copies, compute and device-to-host copies on three "
+                       "streams with two device buffers; one timed region over all steps"
+                       + ("; the forward replayed from a CUDA graph per buffer"
+                          if graphs is not None else "")}
+    del graphs
+    return res
 
 
 # ---------------------------------------------------------- Engram lookup --

@@ -94,3 +94,38 @@ def test_engram_workload_and_bytes():
     assert torch.equal(other["table"], inp["table"]) and not torch.equal(other["tokens"],
                                                                           inp["tokens"])
     assert small.scaled(seed=small.seed + 1).seeds == small.seeds
+
+
+def test_traffic_records_follow_their_sources(tmp_path, monkeypatch):
+    """bench.py reports an ncu traffic record only while every kernel source
+    it names is unchanged (by hash); multi-source records need all of them."""
+    import hashlib
+    import json
+    import os
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+
+    def sha(name):
+        path = os.path.join(root, "sparse_key_value_b200", "csrc", name)
+        return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+    rec = {
+        "a": {"source": "k_embbag.cu", "source_sha": sha("k_embbag.cu"),
+              "dram_bytes_per_launch": 11},
+        "b": {"source": "k_embbag.cu", "source_sha": "0" * 16, "dram_bytes_per_launch": 12},
+        "c:backward": {"sources": {"k_segsum.cu": sha("k_segsum.cu"),
+                                   "k_sort.cu": sha("k_sort.cu")},
+                       "dram_bytes_per_launch": 13, "l2_bytes_per_launch": 14},
+        "d:backward": {"sources": {"k_segsum.cu": sha("k_segsum.cu"), "k_sort.cu": "1" * 16},
+                       "dram_bytes_per_launch": 15, "l2_bytes_per_launch": 16},
+    }
+    (tmp_path / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    assert bench.traffic_record("a") == 11
+    assert bench.traffic_record("b") is None          # its kernel changed since the capture
+    assert bench.traffic_record("missing") is None
+    assert bench.traffic_entry("c:backward")["l2_bytes_per_launch"] == 14
+    assert bench.traffic_entry("d:backward") is None  # one of its sources changed
