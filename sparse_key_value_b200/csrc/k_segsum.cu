@@ -457,6 +457,176 @@ __global__ void __launch_bounds__(256) segsum_dw_kernel(
   for (int jj = lv + lane; jj < len; jj += 32) dw_out[(int64_t)sl * n + e_s[jj]] = 0.f;
 }
 
+// ------------------------------------------- wide rows through a ring ----
+// The same segmented sum for bf16 source rows of d % 512 == 0 columns (the
+// value gradient: src = dy): one CTA per chunk, the chunk's source rows
+// brought into a deep ring of shared-memory slots by bulk copies
+// (cp.async.bulk, one per row) that a producer lane issues up to R rows ahead,
+// so the L2 sees many whole-row reads in flight per SM instead of a few
+// 16-byte loads per thread.  Consumer warp w, lane l owns the 16-byte column
+// chunks (w Q + q) 32 + l, q < Q; each warp releases a slot once its lanes
+// have read it.  Sums run entry by entry in sorted order (bitwise the same as
+// segsum_chunk_kernel).
+constexpr int kRingQ = 2;                  // 16-byte column chunks per consumer lane
+constexpr size_t kRingBytes = 32u << 10;   // ring slots per CTA: six CTAs per SM
+constexpr int kRingMaxSlots = 32;
+
+__device__ __forceinline__ void bulk_row_hint(void* smem_dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_u32(smem_dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
+__host__ __device__ inline int segsum_ring_slots(int d) {
+  const int r = (int)(kRingBytes / ((size_t)d * 2));
+  return r < kRingMaxSlots ? r : kRingMaxSlots;
+}
+__host__ __device__ inline size_t segsum_ring_smem(int d) {
+  return (size_t)segsum_ring_slots(d) * d * 2 + (size_t)(kChunk + 4) * 4 * 3 +
+         (size_t)kRingMaxSlots * 16;
+}
+
+__global__ void __launch_bounds__(32 * 9) segsum_ring_kernel(
+    const uint32_t* __restrict__ skey, const uint32_t* __restrict__ sval, int64_t n,
+    uint32_t mark, const float* __restrict__ coef, const __nv_bfloat16* __restrict__ src,
+    int64_t div, int d, SegWs ws, SegOutDev out, int32_t* status) {
+  constexpr int Q = kRingQ;
+  constexpr int E = 8 * Q;
+  extern __shared__ __align__(16) unsigned char smem_ring[];
+  const int R = segsum_ring_slots(d);
+  const int nw = (int)(blockDim.x >> 5) - 1;  // consumer warps; warp nw produces
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(smem_ring);  // [R][d]
+  uint32_t* key_s = reinterpret_cast<uint32_t*>(smem_ring + (size_t)R * d * 2);  // [kChunk + 1]
+  uint32_t* row_s = key_s + kChunk + 4;
+  float* cf_s = reinterpret_cast<float*>(row_s + kChunk + 4);
+  uint64_t* full = reinterpret_cast<uint64_t*>(cf_s + kChunk + 4);
+  uint64_t* empty = full + kRingMaxSlots;
+  __shared__ int n_valid;
+  __shared__ volatile int abort_flag;
+
+  const int64_t c = blockIdx.x;
+  const int64_t i0 = c * kChunk;
+  const int len = (int)min((int64_t)kChunk, n - i0);
+  const uint32_t div32 = (uint32_t)div;
+  if (threadIdx.x == 0) {
+    n_valid = 0;
+    abort_flag = 0;
+    for (int s = 0; s < R; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], (uint32_t)nw);
+    }
+    fence_barrier_init();
+  }
+  for (int j = threadIdx.x; j <= len; j += blockDim.x) {
+    const int64_t i = i0 + j;
+    key_s[j] = i < n ? skey[i] : mark;
+    if (j < len) {
+      const uint32_t e = sval[i];
+      row_s[j] = e / div32;
+      cf_s[j] = key_s[j] != mark ? coef[e] : 0.f;
+    }
+  }
+  const uint32_t prev_key = i0 > 0 ? skey[i0 - 1] : mark;
+  __syncthreads();
+  {
+    int cnt = 0;
+    for (int j = threadIdx.x; j < len; j += blockDim.x) cnt += key_s[j] != mark;
+    if (cnt) atomicAdd(&n_valid, cnt);
+  }
+  const uint32_t base = ws.seg_base[c];
+  if (threadIdx.x == 0) {
+    ws.first_end[c] = 1;
+    ws.last_seg[c] = 0xffffffffu;
+  }
+  __syncthreads();
+  const int lv = n_valid;  // valid entries come first (the mark sorts last)
+  const uint32_t row_bytes = (uint32_t)d * 2;
+
+  if (warp == nw) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t keep = l2_policy_keep();  // dy rows are re-read by many chunks
+      int j = 0;
+      for (int slot = 0, round = 0; j < lv; ++j) {
+        if (round > 0 &&
+            !mbar_wait_or_abort(&empty[slot], (uint32_t)(round - 1) & 1, &abort_flag, status))
+          break;
+        fence_proxy_async_smem();  // the consumers' reads of the slot come first
+        mbar_arrive_expect_tx(&full[slot], row_bytes);
+        bulk_row_hint(ring + (size_t)slot * d, src + (int64_t)row_s[j] * d, row_bytes,
+                      &full[slot], keep);
+        if (++slot == R) { slot = 0; ++round; }
+      }
+      if (j < lv) {
+        // a wait gave up: every copy issued lands before the CTA leaves
+        for (int jj = j > R ? j - R : 0; jj < j; ++jj)
+          for (unsigned long long it = 0; it < kSpinLimit; ++it)
+            if (mbar_try_wait(&full[jj % R], (uint32_t)(jj / R) & 1)) break;
+      }
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- consumers
+  float acc[E];
+#pragma unroll
+  for (int q = 0; q < E; ++q) acc[q] = 0.f;
+  uint32_t heads = 0;
+  bool part_starts = !(key_s[0] != mark && prev_key == key_s[0]);
+  for (int j = 0, slot = 0, round = 0; j < lv; ++j) {
+    const bool got = mbar_wait_or_abort(&full[slot], (uint32_t)round & 1, &abort_flag, status);
+    if (!__all_sync(0xffffffffu, got)) break;
+    const uint4* rowp = reinterpret_cast<const uint4*>(ring + (size_t)slot * d);
+    uint4 v[Q];
+#pragma unroll
+    for (int q = 0; q < Q; ++q) v[q] = rowp[(warp * Q + q) * 32 + lane];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    if (++slot == R) { slot = 0; ++round; }
+    const float cf = cf_s[j];
+    const float2 w2 = make_float2(cf, cf);
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      float f[8];
+      unpack16<PKM_BF16>(v[q], f);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float2 r = __ffma2_rn(w2, make_float2(f[e], f[e + 1]),
+                                    make_float2(acc[8 * q + e], acc[8 * q + e + 1]));
+        acc[8 * q + e] = r.x;
+        acc[8 * q + e + 1] = r.y;
+      }
+    }
+    const uint32_t key = key_s[j];
+    if (j + 1 < len && key_s[j + 1] == key) continue;  // the part goes on in this chunk
+    const bool seg_ends = key_s[j + 1] != key;  // key_s[len] is the next chunk's first
+    if (part_starts) ++heads;
+    const uint32_t seg = base + heads - 1;
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      const int ch = (warp * Q + q) * 32 + lane;  // 16-byte column chunk of the row
+      if (part_starts && seg_ends) {
+        emit_final<8>(out, seg, key, d, ch, acc + 8 * q, status);
+      } else if (!part_starts) {
+        store_row<8>(ws.carry_first + c * d + (int64_t)ch * 8, acc + 8 * q);
+      } else {
+        store_row<8>(ws.carry_last + c * d + (int64_t)ch * 8, acc + 8 * q);
+      }
+    }
+    if (warp == 0 && lane == 0) {
+      if (!part_starts) ws.first_end[c] = seg_ends ? 1u : 0u;
+      else if (!seg_ends) ws.last_seg[c] = seg;
+    }
+#pragma unroll
+    for (int q = 0; q < E; ++q) acc[q] = 0.f;
+    part_starts = true;
+  }
+}
+
 // Adds the carried pieces of every segment that crosses chunk boundaries.
 template <int V>
 __global__ void __launch_bounds__(kThreads) segsum_fixup_kernel(const uint32_t* __restrict__ skey,
@@ -489,6 +659,12 @@ cudaError_t launch_scan_exclusive(uint32_t* data, int64_t len, uint32_t* total, 
 
 bool segsum_has_dw(pkm_dtype dt, int d) {
   return dt == PKM_BF16 && d % 256 == 0 && d <= 2048 && (d / segsum_dw_slices(d)) % 256 == 0;
+}
+// the ring kernel: bf16 rows of 1024..4096 columns in steps of 512, whose
+// bulk copies start 16-byte aligned
+static bool segsum_ring_ok(pkm_dtype dt, int d, const void* src) {
+  return dt == PKM_BF16 && d % (256 * kRingQ) == 0 && d >= 1024 && d <= 4096 &&
+         (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
 }
 // column slices of the dw walk: 512 columns per warp (narrower slices put more
 // warps on a chunk: each warp's walk over its entries is a chain of dependent
@@ -542,6 +718,21 @@ cudaError_t launch_segsum(const uint32_t* skey, const uint32_t* sval, int64_t n,
       default: go(segsum_dw_kernel<8>); break;
     }
     if (e != cudaSuccess) return e;
+    segsum_fixup_kernel<8><<<(unsigned)chunks, min(kThreads, ((d / 8) + 31) / 32 * 32), 0,
+                             stream>>>(skey, n, d, ws, out, status);
+    note_launch(2);
+    return cudaGetLastError();
+  }
+  if (segsum_ring_ok(dt, d, src)) {
+    // wide bf16 rows: the ring kernel, 2 consumer lanes' worth of 16-byte
+    // chunks per 512 columns
+    const int nw = d / (256 * kRingQ);
+    const size_t smem = segsum_ring_smem(d);
+    e = cudaFuncSetAttribute(segsum_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    segsum_ring_kernel<<<(unsigned)chunks, 32 * (nw + 1), smem, stream>>>(
+        skey, sval, n, mark, coef, (const __nv_bfloat16*)src, div, d, ws, out, status);
     segsum_fixup_kernel<8><<<(unsigned)chunks, min(kThreads, ((d / 8) + 31) / 32 * 32), 0,
                              stream>>>(skey, n, d, ws, out, status);
     note_launch(2);

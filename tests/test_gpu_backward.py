@@ -178,3 +178,29 @@ def test_embbag_backward(n_bags, B, d, dt):
     ref_dw = np.einsum("td,tbd->tb", dy.double().cpu().numpy(),
                        table.double().cpu().numpy()[idx.numpy()])
     close(res["dw"].cpu().numpy(), ref_dw, RTOL[dt], "dw")
+
+
+# bf16 rows of 1024..4096 columns take the segmented sum whose source rows come
+# through a ring of whole-row bulk copies (one CTA per chunk of sorted entries,
+# a producer lane up to 12..32 rows ahead): hot rows span many chunks, the last
+# chunk is ragged, 1536 columns puts three consumer warps on a row
+@pytest.mark.parametrize("n_bags,B,d", [(700, 47, 1024), (130, 64, 1536), (90, 40, 4096)])
+def test_embbag_backward_wide_rows(n_bags, B, d):
+    import oracle
+
+    n_rows = 3000
+    g = torch.Generator().manual_seed(n_bags + d)
+    dy = torch.randn(n_bags, d, generator=g).to(torch.bfloat16).cuda()
+    idx, w = random_bags(n_bags, B, n_rows, seed=d + 1, zipf=1.1)
+    dense = torch.zeros(n_rows, d, device="cuda")
+    res = skv.embbag_backward(dy, idx.cuda(), w.cuda(), n_rows=n_rows, dense=dense)
+    idx64 = idx.numpy().astype(np.int64).reshape(n_bags, 1, B)
+    w64 = w.double().numpy().reshape(n_bags, 1, B)
+    rows = np.unique(idx64)
+    ref_rows = oracle.value_grad_rows(idx64, w64, dy.cpu(), rows)
+    np.testing.assert_array_equal(res["uniq_rows"].cpu().numpy(), rows)
+    close(res["grad_rows"].cpu().numpy(), ref_rows, RTOL["bf16"], "grad_rows")
+    close(dense[torch.from_numpy(rows).cuda()].cpu().numpy(), ref_rows, RTOL["bf16"], "dense")
+    # summed in sorted order: a second run gives the same bits
+    res2 = skv.embbag_backward(dy, idx.cuda(), w.cuda(), n_rows=n_rows)
+    assert torch.equal(res["grad_rows"], res2["grad_rows"])
