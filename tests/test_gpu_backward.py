@@ -76,7 +76,9 @@ def run_backward(wl, dense=False, sample_rows=None):
 # bf16 with d_v a multiple of 256 (up to 2048) and at most a quarter as many
 # slots as table rows takes the value-gradient walk that also yields dw (one
 # warp per chunk of sorted entries and 512-column slice, rows through
-# bulk-copy rings); other shapes re-gather the value rows for dw
+# bulk-copy rings); other shapes re-gather the value rows for dw, and their
+# bf16 rows of 1024..4096 columns (multiples of 512) are summed by the ring
+# walk (one CTA per chunk, whole rows through bulk copies)
 SMALL = [
     # name, T, H, d_half, n_sub, k, d_v, dtype, zipf
     ("bf16-small", 200, 2, 256, 64, 16, 128, "bf16", False),
@@ -85,6 +87,10 @@ SMALL = [
     ("bf16-dw-768-ragged", 70, 3, 256, 96, 7, 768, "bf16", False),
     ("bf16-dw-2048-zipf", 40, 2, 256, 128, 16, 2048, "bf16", True),
     ("bf16-redo-2048-zipf", 257, 2, 256, 64, 32, 2048, "bf16", True),
+    # re-gathered dw, value rows of 1024..4096 columns summed by the ring walk
+    ("bf16-ring-1024-zipf", 300, 2, 256, 64, 16, 1024, "bf16", True),
+    ("bf16-ring-1536-ragged", 77, 3, 256, 40, 7, 1536, "bf16", False),
+    ("bf16-ring-4096-zipf", 33, 1, 256, 32, 32, 4096, "bf16", True),
     ("f32-small", 130, 3, 128, 16, 8, 32, "f32", False),
     ("bf16-k1", 64, 1, 256, 8, 1, 16, "bf16", False),
     ("f32-k64", 50, 1, 128, 64, 64, 24, "f32", False),
