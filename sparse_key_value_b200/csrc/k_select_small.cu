@@ -377,9 +377,11 @@ __global__ void __launch_bounds__(ssm::kThreads, 1) select_small_kernel(
     const uint64_t e1 = ld_cg_u64(half_lists + ((int64_t)(2 * h) * T + t) * kList + lane);
     const uint64_t e2 = ld_cg_u64(half_lists + ((int64_t)(2 * h + 1) * T + t) * kList + lane);
     const int64_t o = ((int64_t)t * H + h) * k;
-    combine_lists_warp(in ? entry_score(e1) : -INFINITY, entry_id(e1),
-                       in ? entry_score(e2) : -INFINITY, entry_id(e2), cells, n, k, idx + o,
-                       wout + o);
+    const float v1 = in ? entry_score(e1) : -INFINITY, v2 = in ? entry_score(e2) : -INFINITY;
+    if (k == 32)  // the grid's first row is already in order
+      combine_lists_warp<true>(v1, entry_id(e1), v2, entry_id(e2), cells, n, k, idx + o, wout + o);
+    else
+      combine_lists_warp<false>(v1, entry_id(e1), v2, entry_id(e2), cells, n, k, idx + o, wout + o);
   }
 }
 

@@ -610,9 +610,9 @@ __global__ void __launch_bounds__(sl::kThreads, 2) select_tc_kernel(
       const int64_t o = ((m0 + r) * H + h) * k;
       const bool in = lane < k;
       const int e = lane * P + r;
-      combine_lists_warp(in ? sv[e] : -INFINITY, in ? cv[e] : 0u,
-                         in ? sv[kMaxK * P + e] : -INFINITY, in ? cv[kMaxK * P + e] : 0u, cells,
-                         n, k, idx + o, wout + o);
+      combine_lists_warp<K32>(in ? sv[e] : -INFINITY, in ? cv[e] : 0u,
+                              in ? sv[kMaxK * P + e] : -INFINITY, in ? cv[kMaxK * P + e] : 0u,
+                              cells, n, k, idx + o, wout + o);
     }
   }
 }

@@ -77,7 +77,10 @@ __device__ __forceinline__ uint16_t topk_cell(int e, int k) {
 // cells l, l+32, l+64, l+96 of `cells`; each group of 32 is sorted across
 // the warp, the four groups are merged keeping the top 32, and lane l < k
 // writes the l-th best: row id a*n + b and its softmax weight over the k
-// kept scores.
+// kept scores.  With k = 32 the first group is the grid's first row
+// v1[0] + v2[j], j = 0..31, already in order (fp32 addition of a common
+// term keeps the order of the v2[j]): its sort is skipped.
+template <bool K32 = false>
 __device__ __forceinline__ void combine_lists_warp(float v1, uint32_t a1, float v2, uint32_t b2,
                                                    const uint16_t* cells, int n, int k,
                                                    int32_t* __restrict__ idx_out,
@@ -98,7 +101,7 @@ __device__ __forceinline__ void combine_lists_warp(float v1, uint32_t a1, float 
     id[g] = valid ? ai * (uint32_t)n + bj : 0xffffffffu;
   }
 #pragma unroll
-  for (int g = 0; g < 4; ++g) warp_sort32_desc(v[g], id[g]);
+  for (int g = K32 ? 1 : 0; g < 4; ++g) warp_sort32_desc(v[g], id[g]);
   warp_merge32_desc(v[0], id[0], v[1], id[1]);
   warp_merge32_desc(v[2], id[2], v[3], id[3]);
   warp_merge32_desc(v[0], id[0], v[2], id[2]);

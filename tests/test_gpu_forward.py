@@ -85,9 +85,9 @@ def test_forward_small(case):
 
 # Batches of more than 64 tokens with bf16, d_half % 64 == 0, n >= 256,
 # n % 4 == 0 and k <= 32 run the one-kernel selection (query norms, scores,
-# per-half top-k, k x k combine and softmax in one launch, the two halves of
-# a head in a cluster of two CTAs); smaller batches split the sub-key columns
-# over CTAs and combine in a second kernel.
+# per-half top-k, k x k combine and softmax in one launch; one CTA per (token
+# tile, head, half), the second CTA of a (tile, head) to finish combines; k = 32
+# skips sorting the combine's first group, the grid's already ordered first row).
 FUSED = [
     # name, T, H, d_half, n_sub, k, d_v
     ("fused-k32-ragged-tile", 333, 2, 64, 512, 32, 64),
