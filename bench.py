@@ -62,6 +62,9 @@ def parse():
     p.add_argument("--engram-rows", type=int, default=0,
                    help="engram workload: rows per head table (0: the workload's own, about "
                         "2^20; smaller tables for profiling captures)")
+    p.add_argument("--select-only", action="store_true",
+                   help="profiling aid for the pkm-style workloads: run only the selection "
+                        "(no value table on the device) and print its mean time per launch")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--sharded", action="store_true",
@@ -1220,6 +1223,40 @@ def engram_reference(args, world):
     }
 
 
+def run_select_only(args):
+    """The selection alone on the workload's queries and sub-keys (no value
+    table is allocated): a small-footprint command for kernel captures.  Its
+    line reports the selection's time per launch, not the lookup metric."""
+    import sparse_key_value_b200 as skv
+    from sparse_key_value_b200.inputs import WORKLOADS, make_inputs
+
+    skv.load()
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, "cuda", with_values=False)
+    idx = torch.empty(w.T, w.H, w.k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(w.T, w.H, w.k, dtype=torch.float32, device="cuda")
+
+    def once():
+        skv.pkm_select(inp["query"], inp["subkeys"], w.k, d_v=w.d_v, idx=idx, weights=wts)
+
+    for _ in range(args.warmup):
+        once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        once()
+    e1.record()
+    torch.cuda.synchronize()
+    err = skv.device_error()
+    if err:
+        raise SystemExit(f"bench.py --select-only: device status {err}")
+    return {"metric": "selection time per launch (profiling aid)",
+            "value": round(e0.elapsed_time(e1) * 1e3 / max(1, args.steps), 2), "unit": "us",
+            "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+            "config": {"workload": args.workload, "select_only": True, **w.describe()}}
+
+
 def main():
     args = parse()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
@@ -1232,6 +1269,11 @@ def main():
             res = run_reference(args, rank, world)
         elif args.sharded:
             res = run_sharded(args, rank, world, local)
+        elif args.select_only:
+            if args.workload in ("engram", "tiny") or world > 1:
+                raise SystemExit("bench.py: --select-only is for one GPU and the product-key "
+                                 "workloads with bf16 tensor-core selection")
+            res = run_select_only(args)
         elif args.workload == "engram":
             res, w, inp = run_engram(args, rank, world, local)
             res["cpu_baseline"] = engram_cpu_baseline(args, w, inp) \
