@@ -1,5 +1,7 @@
 // pkm_capi_bwd.cu -- C ABI of the backward entry points: validation,
 // workspace carving and the launch sequence (see include/pkm.h).
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -16,8 +18,21 @@ int bits_for(uint64_t max_value) {  // bits needed to hold values 0..max_value
 }
 
 struct BwdLayout {
-  size_t rq, rk, dS, dwp, iota, skeys, svals, ekeys, ecoef, radix, seg, total;
+  size_t rq, rk, dS, dwp, iota, skeys, svals, ekeys, ecoef, radix, seg;
+  // the value-gradient branch's own sort and segment buffers when it runs
+  // beside the rest of the backward (see backward_impl)
+  size_t vkeys, vskeys, vsvals, vradix, vseg, total;
 };
+
+// dw = <dy, V[idx]> from the value-gradient walk (each distinct value row
+// read once) instead of a per-slot re-gather of the value rows: for batches
+// with few slots per table row -- rows then rarely repeat; with many slots per
+// row (R > N/4) the repeated rows make the re-gather cheap in L2 and the plain
+// walk faster (measured: Memory+ shapes 3.78 ms against 4.28 ms, PKM training
+// shapes 2.31 ms against 1.73 ms)
+bool fused_value_dw(pkm_dtype dt, int d_v, size_t R, size_t N) {
+  return segsum_has_dw(dt, d_v) && 4 * R <= N;
+}
 
 BwdLayout bwd_layout(const pkm_bwd_args* a) {
   BwdLayout L{};
@@ -34,8 +49,8 @@ BwdLayout bwd_layout(const pkm_bwd_args* a) {
   L.rk = take(H * 2 * n * 4);
   L.dS = take(R * 4);
   // partial dot products dw [slices][R] of the value-gradient walk
-  L.dwp = segsum_has_dw(a->dtype, a->d_v) && 4 * R <= n * n
-              ? take((size_t)segsum_dw_slices(a->d_v) * R * 4) : 0;
+  const bool fused = fused_value_dw(a->dtype, a->d_v, R, n * n);
+  L.dwp = fused ? take((size_t)segsum_dw_slices(a->d_v) * R * 4) : 0;
   L.iota = take(R2 * 4);
   L.skeys = take(R2 * 4);
   L.svals = take(R2 * 4);
@@ -44,7 +59,16 @@ BwdLayout bwd_layout(const pkm_bwd_args* a) {
   L.radix = take(radix_sort_workspace((int64_t)R2));
   const size_t s1 = segsum_workspace((int64_t)R, a->d_v);
   const size_t s2 = segsum_workspace((int64_t)R2, a->d_half);
-  L.seg = take(s1 > s2 ? s1 : s2);
+  if (fused) {  // one branch: the buffers are shared in turn
+    L.seg = take(s1 > s2 ? s1 : s2);
+  } else {
+    L.seg = take(s2);
+    L.vkeys = take(R * 4);
+    L.vskeys = take(R * 4);
+    L.vsvals = take(R * 4);
+    L.vradix = take(radix_sort_workspace((int64_t)R));
+    L.vseg = take(s1);
+  }
   L.total = off;
   return L;
 }
@@ -81,6 +105,27 @@ pkm_status validate_bwd(const pkm_bwd_args* a) {
     if (e_ != cudaSuccess) return PKM_ERR_CUDA; \
   } while (0)
 
+// The library's second stream on the current device (created once), where
+// the backward runs its value-gradient branch beside the rest; null -- the
+// branch then runs in line -- while `st` is being captured into a graph or
+// if the stream cannot be created.
+cudaStream_t side_stream(cudaStream_t st) {
+  static cudaStream_t streams[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+    return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    cudaStream_t s = nullptr;
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    streams[dev] = s;
+  }
+  return streams[dev];
+}
+
 pkm_status backward_impl(const pkm_bwd_args* a, cudaStream_t st) {
   int32_t* status = status_ptr();
   if (!status) return PKM_ERR_CUDA;
@@ -104,27 +149,68 @@ pkm_status backward_impl(const pkm_bwd_args* a, cudaStream_t st) {
   // qk-normalisation factors (recomputed)
   PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
   PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
-  // value gradient: sort the (row, slot) pairs, then segmented sums of w * dy.
-  // dw = <dy, V[idx]> and the softmax backward dS: from the same sorted walk
-  // (each distinct value row read once) when the batch has few slots per
-  // table row -- rows then rarely repeat, and the walk saves a whole second
-  // pass over the selected rows; with many slots per row (R >= N/4) the
-  // repeated rows make a per-slot re-gather cheap in L2 and the plain walk
-  // faster (measured: Memory+ shapes 3.78 ms against 4.28 ms, PKM training
-  // shapes 2.31 ms against 1.73 ms)
-  const bool fused_dw = segsum_has_dw(a->dtype, dv) && 4 * R <= N;
-  if (!fused_dw)
-    PKM_TRY(launch_bag_dw(a->dy, a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, k,
-                          nullptr, dS, status, st));
   PKM_TRY(launch_iota(iota, 2 * R, st));
-  PKM_TRY(launch_sanitize_keys(a->idx, R, N, ekeys, status, st));
-  PKM_TRY(launch_radix_sort(ekeys, iota, R, bits_for((uint64_t)N), skeys, svals, radix, st));
-  PKM_TRY(launch_segsum(skeys, svals, R, (uint32_t)N, a->weights, a->dy, a->dtype, (int64_t)H * k,
-                        dv, a->uniq_rows, a->grad_rows, a->grad_rows ? a->uniq_cap : 0, a->n_uniq,
-                        a->dvalues_dense, nullptr, seg, status, st,
-                        fused_dw ? a->values : nullptr, fused_dw ? dwp : nullptr));
+  // value gradient: sort the (row, slot) pairs, then segmented sums of w * dy;
+  // dw and the softmax backward dS from the same walk where fused_value_dw
+  // says so.  Otherwise dS comes from a per-slot re-gather of the value rows,
+  // and the value-gradient branch (sort + walk, its own buffers) needs
+  // nothing the rest of the backward computes: it runs on the library's
+  // second stream beside the re-gather and the query and sub-key gradients,
+  // and the caller's stream waits for it at the end.
+  const bool fused_dw = fused_value_dw(a->dtype, dv, (size_t)R, (size_t)N);
+  // the caller's stream waits for the side branch on every way out
+  struct SideJoin {
+    cudaStream_t st = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    bool pending = false;  // join recorded on the side stream, not yet waited for
+    cudaError_t finish() {
+      const cudaError_t e = pending ? cudaStreamWaitEvent(st, join, 0) : cudaSuccess;
+      pending = false;
+      return e;
+    }
+    ~SideJoin() {
+      finish();
+      if (fork) cudaEventDestroy(fork);
+      if (join) cudaEventDestroy(join);
+    }
+  } sj;
+  sj.st = st;
+  cudaStream_t vst = st;
+  if (!fused_dw) {
+    cudaStream_t side = side_stream(st);
+    if (side && cudaEventCreateWithFlags(&sj.fork, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&sj.join, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventRecord(sj.fork, st) == cudaSuccess &&
+        cudaStreamWaitEvent(side, sj.fork, 0) == cudaSuccess)
+      vst = side;
+  }
+  uint32_t* vkeys = fused_dw ? ekeys : reinterpret_cast<uint32_t*>(ws + L.vkeys);
+  uint32_t* vskeys = fused_dw ? skeys : reinterpret_cast<uint32_t*>(ws + L.vskeys);
+  uint32_t* vsvals = fused_dw ? svals : reinterpret_cast<uint32_t*>(ws + L.vsvals);
+  void* vradix = fused_dw ? radix : ws + L.vradix;
+  void* vseg = fused_dw ? seg : ws + L.vseg;
+  cudaError_t ve = launch_sanitize_keys(a->idx, R, N, vkeys, status, vst);
+  if (ve == cudaSuccess)
+    ve = launch_radix_sort(vkeys, iota, R, bits_for((uint64_t)N), vskeys, vsvals, vradix, vst);
+  if (ve == cudaSuccess)
+    ve = launch_segsum(vskeys, vsvals, R, (uint32_t)N, a->weights, a->dy, a->dtype,
+                       (int64_t)H * k, dv, a->uniq_rows, a->grad_rows,
+                       a->grad_rows ? a->uniq_cap : 0, a->n_uniq, a->dvalues_dense, nullptr, vseg,
+                       status, vst, fused_dw ? a->values : nullptr, fused_dw ? dwp : nullptr);
+  if (vst != st) {
+    if (cudaEventRecord(sj.join, vst) == cudaSuccess) {
+      sj.pending = true;
+    } else {  // no event to wait on: let the side branch finish before returning
+      cudaStreamSynchronize(vst);
+      return PKM_ERR_CUDA;
+    }
+  }
+  if (ve != cudaSuccess) return PKM_ERR_CUDA;
   if (fused_dw)
     PKM_TRY(launch_softmax_bwd(a->weights, dwp, segsum_dw_slices(dv), T * H, k, dS, st));
+  else
+    PKM_TRY(launch_bag_dw(a->dy, a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, k,
+                          nullptr, dS, status, st));
   // query gradient
   PKM_TRY(launch_dq(a->query, a->subkeys, a->dtype, rq, rk, a->idx, dS, T, H, dh, n, k, a->dquery,
                     st));
@@ -137,6 +223,7 @@ pkm_status backward_impl(const pkm_bwd_args* a, cudaStream_t st) {
   PKM_TRY(launch_segsum(skeys, svals, 2 * R, mark, ecoef, a->query, a->dtype, k, dh, nullptr,
                         nullptr, 0, nullptr, nullptr, a->dsubkeys, seg, status, st));
   PKM_TRY(launch_dk_jacobian(a->subkeys, a->dtype, rk, (int64_t)H * 2 * n, dh, a->dsubkeys, st));
+  PKM_TRY(sj.finish());
   return PKM_OK;
 }
 

@@ -210,3 +210,49 @@ def test_embbag_backward_wide_rows(n_bags, B, d):
     # summed in sorted order: a second run gives the same bits
     res2 = skv.embbag_backward(dy, idx.cuda(), w.cuda(), n_rows=n_rows)
     assert torch.equal(res["grad_rows"], res2["grad_rows"])
+
+
+def test_backward_side_stream_caller_stream_and_graph():
+    """With dw from the per-slot re-gather, the value-gradient branch (sort and
+    walk) runs on the library's second stream beside the rest of the
+    backward and the caller's stream waits for it; inside a CUDA-graph
+    capture it runs in line.  On a caller stream other than the default, and
+    replayed from a graph, the results equal the eager ones bit for bit."""
+    wl = WORKLOADS["train"].scaled(name="side-stream", T=300, H=2, d_half=256, n_sub=64, k=16,
+                                   d_v=1024, seed=5)
+    inp = make_inputs(wl, "cuda")
+    q, K, V, dy = inp["query"], inp["subkeys"], inp["values"], inp["dy"]
+    out, idx, w = skv.pkm_forward(q, K, V, wl.k)
+    N = wl.n_sub ** 2
+    assert wl.T * wl.H * wl.k * 4 > N  # the re-gather path, where the branches split
+
+    def run(dense):
+        return skv.pkm_backward(q, K, V, idx, w, dy, sparse=False, dense=dense)
+
+    d0 = torch.zeros(N, wl.d_v, device="cuda")
+    a = run(d0)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    d1 = torch.zeros(N, wl.d_v, device="cuda")
+    with torch.cuda.stream(s):
+        b = run(d1)
+    s.synchronize()
+    d2 = torch.zeros(N, wl.d_v, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run(torch.zeros(N, wl.d_v, device="cuda"))  # warm the allocator outside the capture
+    side.synchronize()
+    with torch.cuda.graph(g):
+        c = run(d2)
+    d2.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    for key in ("dquery", "dsubkeys"):
+        assert torch.equal(a[key], b[key]), key
+        assert torch.equal(a[key], c[key]), key
+    assert torch.equal(d0, d1)
+    assert torch.equal(d0, d2)
+    assert skv.device_error() == 0
