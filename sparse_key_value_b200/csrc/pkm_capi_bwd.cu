@@ -146,9 +146,6 @@ pkm_status backward_impl(const pkm_bwd_args* a, cudaStream_t st) {
   const int H = a->H, dh = a->d_half, n = a->n_sub, k = a->k, dv = a->d_v;
   const int64_t N = (int64_t)n * n, R = T * H * k;
 
-  // qk-normalisation factors (recomputed)
-  PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
-  PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
   PKM_TRY(launch_iota(iota, 2 * R, st));
   // value gradient: sort the (row, slot) pairs, then segmented sums of w * dy;
   // dw and the softmax backward dS from the same walk where fused_value_dw
@@ -211,6 +208,9 @@ pkm_status backward_impl(const pkm_bwd_args* a, cudaStream_t st) {
   else
     PKM_TRY(launch_bag_dw(a->dy, a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, k,
                           nullptr, dS, status, st));
+  // qk-normalisation factors (recomputed), for dq and dK
+  PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
+  PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
   // query gradient
   PKM_TRY(launch_dq(a->query, a->subkeys, a->dtype, rq, rk, a->idx, dS, T, H, dh, n, k, a->dquery,
                     st));
