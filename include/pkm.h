@@ -185,6 +185,13 @@ PKM_API pkm_status pkm_select(const pkm_fwd_args *args, pkm_stream_t stream);
  *   Either may be NULL (not both).  dscores [T,H,k] fp32 (optional) gets dS.
  * Every sum runs in a fixed order: results are bitwise reproducible.
  *
+ * Streams: when dw comes from a per-slot re-gather of the value rows (more
+ * slots than a quarter of the table rows), the value-gradient sort and
+ * segmented sum run on a library-owned stream of the current device, forked
+ * from `stream` by an event and joined back to it by another before the
+ * call's last work item, so every output is ordered on `stream` as usual.
+ * While `stream` is being captured into a CUDA graph all work stays on it.
+ *
  * Limits beyond the forward's: d_half a multiple of 256 (bf16) or 128 (fp32)
  * and at most 2048 (one warp holds a query half in registers, 16 bytes per
  * lane per step); T*H*k*2 < 2^32.  Other sizes return PKM_ERR_UNSUPPORTED
