@@ -256,3 +256,31 @@ def test_backward_side_stream_caller_stream_and_graph():
     assert torch.equal(d0, d1)
     assert torch.equal(d0, d2)
     assert skv.device_error() == 0
+
+
+def test_embbag_backward_wide_rows_invalid_ids():
+    """Out-of-range row ids (negative or past the table) in the ring walk's
+    value gradient: those entries are dropped (sorted last, never summed), the
+    device status records the anomaly, and every valid row's gradient is
+    exact against the oracle on the valid entries alone."""
+    import oracle
+
+    n_bags, B, d, n_rows = 500, 40, 1024, 2000
+    g = torch.Generator().manual_seed(77)
+    dy = torch.randn(n_bags, d, generator=g).to(torch.bfloat16).cuda()
+    idx, w = random_bags(n_bags, B, n_rows, seed=78, zipf=1.1)
+    bad = torch.rand(n_bags, B, generator=g) < 0.01
+    idx[bad & (torch.rand(n_bags, B, generator=g) < 0.5)] = -1
+    idx[bad & (idx >= 0)] = n_rows + 5
+    assert int(bad.sum()) > 0
+    res = skv.embbag_backward(dy, idx.cuda(), w.cuda(), n_rows=n_rows)
+    assert skv.device_error() == 4  # PKM_ERR_DEVICE: an out-of-range row id
+    idx64 = idx.numpy().astype(np.int64)
+    valid = (idx64 >= 0) & (idx64 < n_rows)
+    rows = np.unique(idx64[valid])
+    # the invalid entries contribute nothing: weight 0 on a row that is present anyway
+    idx_ok = np.where(valid, idx64, rows[0]).reshape(n_bags, 1, B)
+    w_ok = np.where(valid, w.double().numpy(), 0.0).reshape(n_bags, 1, B)
+    ref_rows = oracle.value_grad_rows(idx_ok, w_ok, dy.cpu(), rows)
+    np.testing.assert_array_equal(res["uniq_rows"].cpu().numpy(), rows)
+    close(res["grad_rows"].cpu().numpy(), ref_rows, RTOL["bf16"], "grad_rows")
