@@ -96,11 +96,11 @@ __device__ __forceinline__ uint64_t pack_entry(float s, uint32_t id) {
 __device__ __forceinline__ float entry_score(uint64_t e) { return __uint_as_float((uint32_t)e); }
 __device__ __forceinline__ uint32_t entry_id(uint64_t e) { return (uint32_t)(e >> 32); }
 
-// L2-coherent load (skips L1): other CTAs wrote these
+// L2-coherent load (skips L1): other CTAs wrote these.  A plain load with the
+// .cg hint, so that a warp's loads of all chunks can be in flight together
+// (the __syncthreads after the count keeps them below it)
 __device__ __forceinline__ uint64_t ld_cg_u64(const uint64_t* p) {
-  uint64_t v;
-  asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
+  return __ldcg(reinterpret_cast<const unsigned long long*>(p));
 }
 
 // wait for the TMEM loads in flight; names the registers of the load being
