@@ -341,3 +341,28 @@ def test_decode_steps():
         run_forward(w, inp=inp)
     del base
     torch.cuda.empty_cache()
+
+
+# The selection at the largest supported sizes: n_sub^2 < 2^31 allows n_sub =
+# 46340 (a multiple of 4, so the tensor-core selection takes it: 363 chunks,
+# the last one ragged), and d_half = 2048 is the widest query half (32
+# k-blocks per chunk); two token tiles, the second ragged
+@pytest.mark.parametrize("n,dh", [(46340, 64), (1024, 2048)], ids=["n-46340", "dh-2048"])
+def test_select_maximum_sizes(n, dh):
+    import oracle
+    from parity import check_selection, weights_close, W_RTOL
+
+    w = WORKLOADS["pkm"].scaled(name=f"max-{n}-{dh}", T=130, H=1, d_half=dh, n_sub=n, k=32,
+                                d_v=8, seed=n + dh)
+    inp = make_inputs(w, "cuda", with_values=False)
+    idx, wts = skv.pkm_select(inp["query"], inp["subkeys"], w.k, d_v=w.d_v)
+    torch.cuda.synchronize()
+    assert skv.device_error() == 0
+    q, K = inp["query"].cpu(), inp["subkeys"].cpu()
+    idx_o, S_o, w_o, _ = oracle.pkm_select(q, K, w.k)
+    s_half = oracle.half_scores(q, K)
+    G = idx.cpu().numpy().astype(np.int64)
+    exempt = check_selection(G, idx_o, s_half, n)
+    assert exempt <= 1, f"{exempt} tie exemptions"
+    weights_close(wts.cpu().numpy(), oracle.softmax(oracle.full_scores(s_half, G, n)),
+                  W_RTOL["bf16"])
