@@ -11,6 +11,7 @@
 //   du_c      = sqrt(d_half) sum_j dS_j kappa_c[a_j]
 //   dq_c      = (du_c - u_c <u_c, du_c>) / max(|q_c|, eps)   (dq_kernel)
 //   dkappa_c[a] = sqrt(d_half) sum over (t,h,j) with a_j = a of dS_j u_c
+//               (its entries written by dq_kernel too)
 //   dK        = (dkappa - kappa <kappa, dkappa>) / max(|K|, eps)
 // The value gradient and dkappa are sums over sorted keys (k_sort.cu,
 // k_segsum.cu); this file holds the per-token kernels.
@@ -178,12 +179,20 @@ cudaError_t launch_softmax_bwd(const float* w, const float* dw, int slices, int6
 // ---------------------------------------------------------------------- dq
 // One warp per (token, head); lane l holds elements [l*E, (l+1)*E) of the
 // d_half-long vectors for E = d_half / 32 (a multiple of 8 up to 64).
+// With `keys` the same pass also writes the sub-key gradient's entries: for
+// each half c, every distinct sub-key position a among the k selected rows
+// becomes one entry
+//   key  = (h*2 + c) * n + a,
+//   coef = sqrt(d_half) * (sum of dS_j with a_j = a) / max(|q_c|, eps)
+// (the sum in j order, the same one du uses); the other slots get key =
+// mark.  Entry e = ((t*H + h)*2 + c)*k + j, whose source row is query row e / k.
 template <pkm_dtype DT, int E>
 __global__ void __launch_bounds__(256) dq_kernel(
     const typename Elem<DT>::T* __restrict__ q, const typename Elem<DT>::T* __restrict__ K,
-    const float* __restrict__ rq, const float* __restrict__ rk, const int32_t* __restrict__ idx,
+    const float* __restrict__ rk, const int32_t* __restrict__ idx,
     const float* __restrict__ dS, int64_t T, int H, int dh, int n, int k,
-    float* __restrict__ dq) {
+    float* __restrict__ dq, uint32_t mark, uint32_t* __restrict__ keys,
+    float* __restrict__ coef) {
   constexpr int V = Elem<DT>::kVec;
   constexpr int NC = E / V;  // 16-byte chunks per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -201,6 +210,20 @@ __global__ void __launch_bounds__(256) dq_kernel(
   for (int c = 0; c < 2; ++c) {
     const int hc = h * 2 + c;
     const typename Elem<DT>::T* Kc = K + (int64_t)hc * n * dh;
+    // the query row's elements (held packed until the end) and its norm
+    const int64_t qrow = th * 2 + c;
+    const typename Elem<DT>::T* qp = q + qrow * dh + (int64_t)lane * E;
+    uint4 qv[NC > 0 ? NC : 1];  // (NC = 0: an instance the launcher never runs)
+    float ss = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < NC; ++cc) {
+      qv[cc] = ldg_nc_16(qp + cc * V);
+      float f[V];
+      unpack16<DT>(qv[cc], f);
+#pragma unroll
+      for (int e = 0; e < V; ++e) ss = fmaf(f[e], f[e], ss);
+    }
+    const float r = 1.0f / fmaxf(sqrtf(warp_sum(ss)), kNormEps);
     // sub-key positions of this half, each distinct one once with the sum of
     // its dS (in slot order), compacted into the warp's list
     const bool ok0 = lane < k && i0 >= 0 && (int64_t)i0 < N;
@@ -221,6 +244,18 @@ __global__ void __launch_bounds__(256) dq_kernel(
         if (j >= lane + 32) s1 += gj;
       }
     }
+    if (keys) {
+      // the sub-key gradient's entries of this (token, head, half): the same
+      // distinct positions with their dS sums, scaled by the query's factor
+      if (lane < k) {
+        keys[qrow * k + lane] = lead0 ? (uint32_t)(hc * n + a0) : mark;
+        coef[qrow * k + lane] = lead0 ? scale * s0 * r : 0.f;
+      }
+      if (lane + 32 < k) {
+        keys[qrow * k + lane + 32] = lead1 ? (uint32_t)(hc * n + a1) : mark;
+        coef[qrow * k + lane + 32] = lead1 ? scale * s1 * r : 0.f;
+      }
+    }
     const unsigned m0 = __ballot_sync(0xffffffffu, lead0);
     const unsigned m1 = __ballot_sync(0xffffffffu, lead1);
     const unsigned lt = (1u << lane) - 1u;
@@ -236,6 +271,8 @@ __global__ void __launch_bounds__(256) dq_kernel(
     }
     __syncwarp();
     const int m = __popc(m0) + __popc(m1);
+    // the sub-key rows stay in L2 while the query rows and dq stream past
+    const uint64_t keep = l2_policy_keep();
     float du[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) du[e] = 0.f;
@@ -247,20 +284,17 @@ __global__ void __launch_bounds__(256) dq_kernel(
 #pragma unroll
       for (int cc = 0; cc < NC; ++cc) {
         float f[V];
-        unpack16<DT>(ldg_nc_16(row + cc * V), f);
+        unpack16<DT>(ldg_nc_16_hint(row + cc * V, keep), f);
 #pragma unroll
         for (int e = 0; e < V; ++e) du[cc * V + e] = fmaf(coef, f[e], du[cc * V + e]);
       }
     }
     __syncwarp();
-    const int64_t qrow = th * 2 + c;
-    const float r = rq[qrow];
     float u[E];
-    const typename Elem<DT>::T* qp = q + qrow * dh + (int64_t)lane * E;
 #pragma unroll
     for (int cc = 0; cc < NC; ++cc) {
       float f[V];
-      unpack16<DT>(ldg_nc_16(qp + cc * V), f);
+      unpack16<DT>(qv[cc], f);
 #pragma unroll
       for (int e = 0; e < V; ++e) u[cc * V + e] = f[e] * r;
     }
@@ -283,15 +317,16 @@ __global__ void __launch_bounds__(256) dq_kernel(
 }
 
 template <pkm_dtype DT>
-static cudaError_t launch_dq_t(const void* q, const void* K, const float* rq, const float* rk,
+static cudaError_t launch_dq_t(const void* q, const void* K, const float* rk,
                                const int32_t* idx, const float* dS, int64_t T, int H, int dh,
-                               int n, int k, float* dq, cudaStream_t stream) {
+                               int n, int k, float* dq, uint32_t mark, uint32_t* keys,
+                               float* coef, cudaStream_t stream) {
   using Tp = typename Elem<DT>::T;
   const unsigned grid = (unsigned)((T * H + 7) / 8);
   const int E = dh / 32;
 #define PKM_DQ(EE)                                                                              \
-  dq_kernel<DT, EE><<<grid, 256, 0, stream>>>((const Tp*)q, (const Tp*)K, rq, rk, idx, dS, T, H, \
-                                              dh, n, k, dq)
+  dq_kernel<DT, EE><<<grid, 256, 0, stream>>>((const Tp*)q, (const Tp*)K, rk, idx, dS, T, H,     \
+                                              dh, n, k, dq, mark, keys, coef)
   if (E % Elem<DT>::kVec != 0) return cudaErrorInvalidValue;
   switch (E) {
     case 4: PKM_DQ(4); break;
@@ -315,76 +350,15 @@ bool backward_dh_supported(pkm_dtype dt, int dh) {
   return dh % (32 * V) == 0 && dh / 32 <= 64;
 }
 
-cudaError_t launch_dq(const void* q, const void* K, pkm_dtype dt, const float* rq,
-                      const float* rk, const int32_t* idx, const float* dS, int64_t T, int H,
-                      int dh, int n, int k, float* dq, cudaStream_t stream) {
+cudaError_t launch_dq(const void* q, const void* K, pkm_dtype dt, const float* rk, const int32_t* idx, const float* dS, int64_t T, int H,
+                      int dh, int n, int k, float* dq, uint32_t mark, uint32_t* keys,
+                      float* coef, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
-  return dt == PKM_BF16 ? launch_dq_t<PKM_BF16>(q, K, rq, rk, idx, dS, T, H, dh, n, k, dq, stream)
-                        : launch_dq_t<PKM_F32>(q, K, rq, rk, idx, dS, T, H, dh, n, k, dq, stream);
-}
-
-// ----------------------------------------------------------- dK entries
-// One warp per (token, head).  For each half c, every distinct sub-key
-// position a among the k selected rows becomes one entry
-//   key = (h*2 + c) * n + a,  coef = sqrt(d_half) * rq * (sum of dS_j with a_j = a)
-// (the sum in j order); the other slots get key = mark.  Entry e =
-// ((t*H + h)*2 + c)*k + j, whose source row is query row e / k.
-__global__ void __launch_bounds__(256) dk_entries_kernel(
-    const int32_t* __restrict__ idx, const float* __restrict__ dS, const float* __restrict__ rq,
-    int64_t T, int H, int dh, int n, int k, uint32_t mark, uint32_t* __restrict__ keys,
-    float* __restrict__ coef) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t th = (int64_t)blockIdx.x * (blockDim.x / 32) + warp;
-  if (th >= T * H) return;
-  const int h = (int)(th % H);
-  const float scale = sqrtf((float)dh);
-  const int32_t id0 = lane < k ? idx[th * k + lane] : 0;
-  const int32_t id1 = lane + 32 < k ? idx[th * k + lane + 32] : 0;
-  const float g0 = lane < k ? dS[th * k + lane] : 0.f;
-  const float g1 = lane + 32 < k ? dS[th * k + lane + 32] : 0.f;
-  for (int c = 0; c < 2; ++c) {
-    const int64_t N = (int64_t)n * n;
-    const bool ok0 = id0 >= 0 && (int64_t)id0 < N, ok1 = id1 >= 0 && (int64_t)id1 < N;
-    const int32_t a0 = ok0 ? (c == 0 ? id0 / n : id0 % n) : -1;
-    const int32_t a1 = ok1 ? (c == 0 ? id1 / n : id1 % n) : -1;
-    bool lead0 = true, lead1 = true;
-    float s0 = 0.f, s1 = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int32_t aj = __shfl_sync(0xffffffffu, j < 32 ? a0 : a1, j & 31);
-      const float gj = __shfl_sync(0xffffffffu, j < 32 ? g0 : g1, j & 31);
-      if (aj == a0) {
-        if (j < lane) lead0 = false;
-        if (j >= lane) s0 += gj;
-      }
-      if (aj == a1) {
-        if (j < lane + 32) lead1 = false;
-        if (j >= lane + 32) s1 += gj;
-      }
-    }
-    const int64_t row = th * 2 + c;
-    const float r = rq[row];
-    const int hc = h * 2 + c;
-    lead0 = lead0 && ok0;
-    lead1 = lead1 && ok1;
-    if (lane < k) {
-      keys[row * k + lane] = lead0 ? (uint32_t)(hc * n + a0) : mark;
-      coef[row * k + lane] = lead0 ? scale * s0 * r : 0.f;
-    }
-    if (lane + 32 < k) {
-      keys[row * k + lane + 32] = lead1 ? (uint32_t)(hc * n + a1) : mark;
-      coef[row * k + lane + 32] = lead1 ? scale * s1 * r : 0.f;
-    }
-  }
-}
-
-cudaError_t launch_dk_entries(const int32_t* idx, const float* dS, const float* rq, int64_t T,
-                              int H, int dh, int n, int k, uint32_t mark, uint32_t* keys,
-                              float* coef, cudaStream_t stream) {
-  if (T <= 0) return cudaSuccess;
-  dk_entries_kernel<<<(unsigned)((T * H + 7) / 8), 256, 0, stream>>>(idx, dS, rq, T, H, dh, n, k,
-                                                                     mark, keys, coef);
-  note_launch();
-  return cudaGetLastError();
+  return dt == PKM_BF16
+             ? launch_dq_t<PKM_BF16>(q, K, rk, idx, dS, T, H, dh, n, k, dq, mark, keys, coef,
+                                     stream)
+             : launch_dq_t<PKM_F32>(q, K, rk, idx, dS, T, H, dh, n, k, dq, mark, keys, coef,
+                                    stream);
 }
 
 // ---------------------------------------------------- sub-key Jacobian

@@ -174,17 +174,16 @@ cudaError_t launch_iota(uint32_t* v, int64_t n, cudaStream_t stream);
 cudaError_t launch_sanitize_keys(const int32_t* idx, int64_t n, int64_t limit, uint32_t* keys,
                                  int32_t* status, cudaStream_t stream);
 
-// dq of one (token, head) per warp: d_half must be a multiple of 32 x
-// (elements per 16 bytes), at most 2048.
+// dq of one (token, head) per warp (the query norms computed in the same
+// pass): d_half must be a multiple of 32 x (elements per 16 bytes), at most
+// 2048.  With `keys` (2 T H k entries) it
+// also writes the sub-key gradient's entries (distinct positions per token,
+// head and half; the other slots get `mark`) and their coefficients.
 bool backward_dh_supported(pkm_dtype dt, int dh);
-cudaError_t launch_dq(const void* q, const void* K, pkm_dtype dt, const float* rq,
-                      const float* rk, const int32_t* idx, const float* dS, int64_t T, int H,
-                      int dh, int n, int k, float* dq, cudaStream_t stream);
-
-// Sub-key gradient entries (distinct positions per token, head and half).
-cudaError_t launch_dk_entries(const int32_t* idx, const float* dS, const float* rq, int64_t T,
-                              int H, int dh, int n, int k, uint32_t mark, uint32_t* keys,
-                              float* coef, cudaStream_t stream);
+cudaError_t launch_dq(const void* q, const void* K, pkm_dtype dt, const float* rk,
+                      const int32_t* idx, const float* dS, int64_t T, int H, int dh, int n,
+                      int k, float* dq, uint32_t mark, uint32_t* keys, float* coef,
+                      cudaStream_t stream);
 cudaError_t launch_dk_jacobian(const void* K, pkm_dtype dt, const float* rk, int64_t rows, int dh,
                                float* g, cudaStream_t stream);
 

@@ -18,7 +18,7 @@ int bits_for(uint64_t max_value) {  // bits needed to hold values 0..max_value
 }
 
 struct BwdLayout {
-  size_t rq, rk, dS, dwp, iota, skeys, svals, ekeys, ecoef, radix, seg;
+  size_t rk, dS, dwp, iota, skeys, svals, ekeys, ecoef, radix, seg;
   // the value-gradient branch's own sort and segment buffers when it runs
   // beside the rest of the backward (see backward_impl)
   size_t vkeys, vskeys, vsvals, vradix, vseg, total;
@@ -45,7 +45,6 @@ BwdLayout bwd_layout(const pkm_bwd_args* a) {
     off += round_up(bytes);
     return o;
   };
-  L.rq = take(T * H * 2 * 4);
   L.rk = take(H * 2 * n * 4);
   L.dS = take(R * 4);
   // partial dot products dw [slices][R] of the value-gradient walk
@@ -131,7 +130,6 @@ pkm_status backward_impl(const pkm_bwd_args* a, cudaStream_t st) {
   if (!status) return PKM_ERR_CUDA;
   const BwdLayout L = bwd_layout(a);
   char* ws = static_cast<char*>(a->workspace);
-  float* rq = reinterpret_cast<float*>(ws + L.rq);
   float* rk = reinterpret_cast<float*>(ws + L.rk);
   float* dS = a->dscores ? a->dscores : reinterpret_cast<float*>(ws + L.dS);
   float* dwp = reinterpret_cast<float*>(ws + L.dwp);
@@ -208,16 +206,14 @@ pkm_status backward_impl(const pkm_bwd_args* a, cudaStream_t st) {
   else
     PKM_TRY(launch_bag_dw(a->dy, a->values, N, dv, a->dtype, a->idx, a->weights, T, H * k, k,
                           nullptr, dS, status, st));
-  // qk-normalisation factors (recomputed), for dq and dK
-  PKM_TRY(launch_row_rnorm(a->query, a->dtype, T * H * 2, dh, rq, st));
+  // the sub-keys' normalisation factors (recomputed; the query's come with dq)
   PKM_TRY(launch_row_rnorm(a->subkeys, a->dtype, (int64_t)H * 2 * n, dh, rk, st));
-  // query gradient
-  PKM_TRY(launch_dq(a->query, a->subkeys, a->dtype, rq, rk, a->idx, dS, T, H, dh, n, k, a->dquery,
-                    st));
-  // sub-key gradient: entries per distinct (head, half, sub-key) and token,
-  // sorted, summed into the dense output, then the normalisation Jacobian
+  // query gradient, and the sub-key gradient's entries per distinct (head,
+  // half, sub-key) and token in the same pass; then the entries sorted,
+  // summed into the dense output, and the normalisation Jacobian
   const uint32_t mark = (uint32_t)(2 * H * n);
-  PKM_TRY(launch_dk_entries(a->idx, dS, rq, T, H, dh, n, k, mark, ekeys, ecoef, st));
+  PKM_TRY(launch_dq(a->query, a->subkeys, a->dtype, rk, a->idx, dS, T, H, dh, n, k, a->dquery,
+                    mark, ekeys, ecoef, st));
   PKM_TRY(launch_radix_sort(ekeys, iota, 2 * R, bits_for(mark), skeys, svals, radix, st));
   PKM_TRY(cudaMemsetAsync(a->dsubkeys, 0, sizeof(float) * (size_t)H * 2 * n * dh, st));
   PKM_TRY(launch_segsum(skeys, svals, 2 * R, mark, ecoef, a->query, a->dtype, k, dh, nullptr,
