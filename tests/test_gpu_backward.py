@@ -94,6 +94,11 @@ SMALL = [
     ("f32-small", 130, 3, 128, 16, 8, 32, "f32", False),
     ("bf16-k1", 64, 1, 256, 8, 1, 16, "bf16", False),
     ("f32-k64", 50, 1, 128, 64, 64, 24, "f32", False),
+    # wide query halves: the dq pass holds 16..64 query elements per lane
+    ("bf16-dh1024", 40, 2, 1024, 32, 8, 64, "bf16", False),
+    ("bf16-dh2048-k64", 24, 1, 2048, 64, 64, 32, "bf16", False),
+    ("f32-dh512", 30, 2, 512, 32, 16, 48, "f32", False),
+    ("f32-dh2048", 16, 1, 2048, 16, 8, 16, "f32", False),
 ]
 
 
