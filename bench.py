@@ -62,6 +62,11 @@ def parse():
     p.add_argument("--engram-rows", type=int, default=0,
                    help="engram workload: rows per head table (0: the workload's own, about "
                         "2^20; smaller tables for profiling captures)")
+    p.add_argument("--n-sub", type=int, default=0,
+                   help="profiling aid for the product-key workloads: this many sub-keys per "
+                        "(head, half) and a value table of n_sub^2 rows instead of the "
+                        "workload's own (0), for kernel captures that fit a few GB; its line is "
+                        "not the workload's metric and carries no ncu traffic record")
     p.add_argument("--select-only", action="store_true",
                    help="profiling aid for the pkm-style workloads: run only the selection "
                         "(no value table on the device) and print its mean time per launch")
@@ -346,6 +351,8 @@ def run_ours(args, rank, world, local):
     w = WORKLOADS[args.workload]
     if args.workload == "decode":
         w = w.scaled(T=8)
+    if args.n_sub > 0:
+        w = w.scaled(n_sub=args.n_sub)
     inp = make_inputs(rank_workload(w, rank), "cuda")
     mp = w.memplus
     kw = dict(x=inp["x"], W1=inp["W1"], W2=inp["W2"]) if mp else {}
@@ -476,7 +483,9 @@ def run_ours(args, rank, world, local):
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
     bytes_per_launch = gather_bytes_per_token(w) * T
-    traffic = traffic_record(args.workload)
+    # the committed records hold the workloads' own sizes
+    rec_key = args.workload if args.n_sub <= 0 else None
+    traffic = traffic_record(rec_key) if rec_key else None
     sel = None
     if phase_ms is not None:
         gather_ms = statistics.mean(phase_ms[4])
@@ -489,7 +498,8 @@ def run_ours(args, rank, world, local):
         phases = dict(zip(["norms", "score_topk", "combine_softmax", "gate_gemm", "gather",
                            "out_gemm"], [round(statistics.mean(p) * 1e3, 2) for p in phase_ms]))
         sel = selection_roofline(w, statistics.mean(phase_ms[1]) + statistics.mean(phase_ms[2]),
-                                 peaks, peak_kind, traffic_record(args.workload + ":select"))
+                                 peaks, peak_kind,
+                                 traffic_record(rec_key + ":select") if rec_key else None)
     else:  # graph replay: only whole steps are timed
         achieved = bytes_per_launch / (ms_per_step / 1e3) / 1e9
         roof = {"kernel": "whole step (graph replay)", "bound": "hbm",
@@ -518,7 +528,7 @@ def run_ours(args, rank, world, local):
         # the kernels' own DRAM and L2 bytes (ncu record): repeated (Zipf-hot)
         # rows are L2 hits, so the backward is bound by L2 traffic more than
         # by DRAM; both bounds side by side
-        rec = traffic_entry(args.workload + ":backward")
+        rec = traffic_entry(rec_key + ":backward") if rec_key else None
         if rec:
             l2bw = l2_read_gbs()
             db, lb = rec["dram_bytes_per_launch"], rec["l2_bytes_per_launch"]
@@ -1232,6 +1242,8 @@ def run_select_only(args):
 
     skv.load()
     w = WORKLOADS[args.workload]
+    if args.n_sub > 0:
+        w = w.scaled(n_sub=args.n_sub)
     inp = make_inputs(w, "cuda", with_values=False)
     idx = torch.empty(w.T, w.H, w.k, dtype=torch.int32, device="cuda")
     wts = torch.empty(w.T, w.H, w.k, dtype=torch.float32, device="cuda")
