@@ -323,24 +323,6 @@ def traffic_entry(workload: str):
     return rec
 
 
-def l2_read_gbs() -> float:
-    """Measured L2 read bandwidth for the L2-bound kernels' second roofline:
-    GB/s of torch's sum over a 64 MiB fp32 tensor that stays L2-resident
-    (an L2 reference, like the HBM copy of MEASURED_PEAKS.json)."""
-    x = torch.ones(16 << 20, dtype=torch.float32, device="cuda")
-    for _ in range(3):
-        x.sum()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 50
-    e0.record()
-    for _ in range(reps):
-        x.sum()
-    e1.record()
-    torch.cuda.synchronize()
-    return x.numel() * 4 * reps / (e0.elapsed_time(e1) / 1e3) / 1e9
-
-
 # ------------------------------------------------------------ our arm --
 
 def run_ours(args, rank, world, local):
@@ -526,18 +508,17 @@ def run_ours(args, rank, world, local):
                              "GBps": round(bbytes / (bwd_ms / 1e3) / 1e9, 1),
                              "frac": round(bbytes / (bwd_ms / 1e3) / 1e9 / peak, 4)}
         # the kernels' own DRAM and L2 bytes (ncu record): repeated (Zipf-hot)
-        # rows are L2 hits, so the backward is bound by L2 traffic more than
-        # by DRAM; both bounds side by side
+        # rows are L2 hits, so DRAM moves well under the algorithmic bytes; the
+        # L2 bytes are reported without a time floor (no library-independent
+        # L2 copy reaches the L2 throughput these kernels reach)
         rec = traffic_entry(rec_key + ":backward") if rec_key else None
         if rec:
-            l2bw = l2_read_gbs()
             db, lb = rec["dram_bytes_per_launch"], rec["l2_bytes_per_launch"]
             extra["backward"].update(
                 dram_bytes=db, dram_GBps=round(db / (bwd_ms / 1e3) / 1e9, 1),
                 dram_frac=round(db / (bwd_ms / 1e3) / 1e9 / peak, 4),
                 hbm_bound_us=round(db / (peak * 1e9) * 1e6, 1),
-                l2_bytes=lb, l2_read_GBps_measured=round(l2bw, 1),
-                l2_bound_us=round(lb / (l2bw * 1e9) * 1e6, 1),
+                l2_bytes=lb, l2_GBps=round(lb / (bwd_ms / 1e3) / 1e9, 1),
                 traffic_capture=rec["capture"])
         if mp_train:
             # five GEMMs of 2*T*d_model*d_v FLOPs: a, dz, dx, dW1, dW2
