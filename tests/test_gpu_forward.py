@@ -124,6 +124,9 @@ SMALL_T = [
     ("small-t8-wide", 8, 2, 512, 4096, 32, 32),
     ("small-t17-k31-ragged", 17, 1, 256, 1100, 31, 16),
     ("split-t40", 40, 2, 64, 512, 32, 32),
+    # the first and last batch sizes of the column-split path
+    ("split-t33", 33, 2, 64, 512, 32, 32),
+    ("split-t64-ragged", 64, 1, 128, 300, 16, 48),
 ]
 
 
