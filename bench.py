@@ -67,6 +67,10 @@ def parse():
                         "(head, half) and a value table of n_sub^2 rows instead of the "
                         "workload's own (0), for kernel captures that fit a few GB; its line is "
                         "not the workload's metric and carries no ncu traffic record")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="profiling aid for the product-key workloads: this many tokens per "
+                        "step instead of the workload's own (0); like --n-sub, its line is not "
+                        "the workload's metric and carries no ncu traffic record")
     p.add_argument("--select-only", action="store_true",
                    help="profiling aid for the pkm-style workloads: run only the selection "
                         "(no value table on the device) and print its mean time per launch")
@@ -335,6 +339,8 @@ def run_ours(args, rank, world, local):
         w = w.scaled(T=8)
     if args.n_sub > 0:
         w = w.scaled(n_sub=args.n_sub)
+    if args.tokens > 0:
+        w = w.scaled(T=args.tokens)
     inp = make_inputs(rank_workload(w, rank), "cuda")
     mp = w.memplus
     kw = dict(x=inp["x"], W1=inp["W1"], W2=inp["W2"]) if mp else {}
@@ -466,7 +472,7 @@ def run_ours(args, rank, world, local):
     peak = float(peaks["hbm_gbs"])
     bytes_per_launch = gather_bytes_per_token(w) * T
     # the committed records hold the workloads' own sizes
-    rec_key = args.workload if args.n_sub <= 0 else None
+    rec_key = args.workload if args.n_sub <= 0 and args.tokens <= 0 else None
     traffic = traffic_record(rec_key) if rec_key else None
     sel = None
     if phase_ms is not None:
@@ -1225,6 +1231,8 @@ def run_select_only(args):
     w = WORKLOADS[args.workload]
     if args.n_sub > 0:
         w = w.scaled(n_sub=args.n_sub)
+    if args.tokens > 0:
+        w = w.scaled(T=args.tokens)
     inp = make_inputs(w, "cuda", with_values=False)
     idx = torch.empty(w.T, w.H, w.k, dtype=torch.int32, device="cuda")
     wts = torch.empty(w.T, w.H, w.k, dtype=torch.float32, device="cuda")
